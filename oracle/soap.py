@@ -1,0 +1,110 @@
+"""The SOAP step for one matrix, in float64, with a per-step basis refresh.
+
+Steps, in the order used by the per-step-refresh variant ("Reading notes on
+SOAP, Muon, and Beyond", section 4: the basis is re-orthogonalised every step
+with the current gradient folded in; "初探优化器（一）", section 6.2 steps 1-5;
+"LLM Optimizers: From SGD and AdamW to SOAP, Muon, and Scalable Training",
+section 11.1 equations):
+
+    1. L = bs L + (1 - bs) G G^T ;   R = bs R + (1 - bs) G^T G
+    2. Q_L = qr(L Q_L) ;             Q_R = qr(R Q_R)      (one power step)
+    3. M = b1 M + (1 - b1) G                            (original space)
+    4. M' = Q_L^T M Q_R ;            G' = Q_L^T G Q_R
+    5. V = b2 V + (1 - b2) G' * G'                      (rotated space)
+       Dbar = (M' / (1 - b1^t)) / (sqrt(V / (1 - b2^t)) + eps)
+    6. D = Q_L Dbar Q_R^T
+    7. W = (1 - lr wd) W - lr D
+
+A side whose factor is ``None`` uses the identity basis (one-sided SOAP for
+very large axes, section 11.2 of the LLM Optimizers guide); with both sides
+identity the step is AdamW.  Keeping M in the original space and rotating it
+with the current basis is the same as the section 11.1 change-of-basis rule
+for the stored first moment.  V is never re-rotated.
+
+``precision="bf16"`` reproduces the GPU path's declared rounding points:
+every tensor-core operand is rounded to bf16 (ties to even) and products are
+accumulated wide; the QR is exact (the GPU's is fp32-accurate).  With both
+sides present the two-sided products are taken left factor first:
+
+    s1: Gb = bf16(G);  L = bs L + (1 - bs) Gb Gb^T   (L itself is not rounded)
+    s2: Y = bf16(L) bf16(Q_L);  Q_L = qr(Y)
+    s4: T = bf16(bf16(Q_L)^T Mb);  M' = T bf16(Q_R)        (Mb = bf16(M))
+        T = bf16(bf16(Q_L)^T Gb);  G' = T bf16(Q_R)
+    s6: S = bf16(bf16(Q_L) bf16(Dbar));  D = S bf16(Q_R)^T
+  one-sided: M' = bf16(Q_L)^T Mb,  D = bf16(Q_L) bf16(Dbar)  (left), or
+             M' = Mb bf16(Q_R),    D = bf16(Dbar) bf16(Q_R)^T (right);
+  no side:   M' = M, G' = G, D = Dbar (no rounding: plain AdamW).
+"""
+
+import numpy as np
+
+from .bf16 import rnd
+from .qr import qr_positive
+
+
+def soap_step(W, G, M, V, L=None, QL=None, R=None, QR=None, *, t=1,
+              lr=3e-3, beta1=0.95, beta2=0.95, shampoo_beta=None, eps=1e-8,
+              weight_decay=0.0, bias_correction=True, precision="fp64",
+              refresh=True):
+    """One SOAP step.  Inputs are not modified; returns the new state.
+
+    ``shampoo_beta`` defaults to ``beta2`` (one beta for both second-order
+    statistics).  ``refresh=False`` skips steps 1-2 and uses the given bases
+    as they are (for checks against an exact eigenbasis).
+    """
+    if precision not in ("fp64", "bf16"):
+        raise ValueError(f"unknown precision {precision!r}")
+    r = rnd if precision == "bf16" else (lambda x: x)
+    f64 = lambda x: None if x is None else np.asarray(x, dtype=np.float64)
+    W, G, M, V = f64(W), f64(G), f64(M), f64(V)
+    L, QL, R, QR = f64(L), f64(QL), f64(R), f64(QR)
+    left = QL is not None
+    right = QR is not None
+    bs = beta2 if shampoo_beta is None else shampoo_beta
+
+    Gb = r(G)
+    # 1-2. factor EMAs with the current gradient, then one power step + QR
+    if refresh:
+        if left:
+            L = bs * L + (1.0 - bs) * (Gb @ Gb.T)
+            QL, _ = qr_positive(r(L) @ r(QL))
+        if right:
+            R = bs * R + (1.0 - bs) * (Gb.T @ Gb)
+            QR, _ = qr_positive(r(R) @ r(QR))
+    # 3. first moment, original space
+    M = beta1 * M + (1.0 - beta1) * G
+    Mb = r(M)
+    QLb = r(QL) if left else None
+    QRb = r(QR) if right else None
+
+    # 4. rotate into the basis
+    def rotate_in(X, Xb):
+        if left and right:
+            return r(QLb.T @ Xb) @ QRb
+        if left:
+            return QLb.T @ Xb
+        if right:
+            return Xb @ QRb
+        return X
+
+    Mr = rotate_in(M, Mb)
+    Gr = rotate_in(G, Gb)
+    # 5. Adam in the basis
+    V = beta2 * V + (1.0 - beta2) * Gr * Gr
+    bc1 = 1.0 - beta1 ** t if bias_correction else 1.0
+    bc2 = 1.0 - beta2 ** t if bias_correction else 1.0
+    Dbar = (Mr / bc1) / (np.sqrt(V / bc2) + eps)
+    # 6. rotate back
+    if left and right:
+        D = r(QLb @ r(Dbar)) @ QRb.T
+    elif left:
+        D = QLb @ r(Dbar)
+    elif right:
+        D = r(Dbar) @ QRb.T
+    else:
+        D = Dbar
+    # 7. decoupled weight decay and apply
+    decayed = (1.0 - lr * weight_decay) * W
+    W_new = decayed - lr * D
+    return {"W": W_new, "M": M, "V": V, "L": L, "QL": QL, "R": R, "QR": QR,
+            "Dbar": Dbar, "D": D, "dW": W_new - decayed, "Mr": Mr, "Gr": Gr}

@@ -1,0 +1,499 @@
+#!/usr/bin/env python
+"""Benchmark of the per-matrix optimizer step on B200.
+
+Default workload: one Muon step over every 2-D matrix of a 32-layer dense GPT
+(hidden 4096, 32 query / 8 KV heads of dim 128, FFN 14336): 224 fp32
+matrices, 6.98 G parameters, synthetic gradients (Gaussian N(0, 1e-3^2) plus
+a rank-16 spike with 10x its norm), random-init weights N(0, 0.02^2).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  ``value`` is whole-job TFLOP/s with the
+pages' Newton-Schulz count 5 (4 m'^2 n' + 2 m'^3) per matrix (m' <= n'),
+timed on the device with CUDA events over exactly K steps between a barrier
+and a synchronize, max over ranks.  Inputs are far larger than L2, so no
+flush is needed.  Multi-GPU runs are independent replicas (the step has no
+exchange on one matrix); ``scaling`` is weak.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Muon/SOAP step TFLOP/s and matrices/s on 1 B200; % of BF16 tensor peak & HBM BW"
+UNIT = "TFLOP/s"
+WORKLOAD = "muon_step dense GPT 32 layers (hidden 4096, kv 1024, ffn 14336): 224 fp32 matrices, 6.98 G params"
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def page_flops(m, n, steps=5):
+    """The pages' Newton-Schulz count per matrix: steps * (4 m'^2 n' + 2 m'^3)."""
+    mp, np_ = min(m, n), max(m, n)
+    return steps * (4.0 * mp * mp * np_ + 2.0 * mp ** 3)
+
+
+def gemm_alg_flops(m, n, steps=5):
+    """Necessary tensor-core flops of our NS products per matrix: the two
+    symmetric products only need their upper triangle (m'(m'+1)/2 entries)."""
+    mp, np_ = min(m, n), max(m, n)
+    gram = mp * (mp + 1) * np_
+    poly = mp * (mp + 1) * mp
+    update = 2.0 * mp * mp * np_
+    return steps * (gram + poly + update)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ----------------------------------------------------------------------------- workloads on the GPU
+
+def gpt_workload(device, layers=32, hidden=4096, kv=1024, ffn=14336, rank=16, noise=1e-3, ratio=10.0):
+    """Synthetic dense-GPT matrices generated on the device (seeded torch
+    generator; same recipe as workloads.gauss_spike)."""
+    import torch
+    import workloads as wl
+    Ws, Gs, Bs, shapes = [], [], [], []
+    for layer in range(layers):
+        for name, m, n in wl.gpt_shapes(hidden, kv, ffn):
+            g = torch.Generator(device=device)
+            g.manual_seed(wl.seed_of("bench-cfg2", layer, name))
+            W = torch.randn(m, n, generator=g, device=device) * 0.02
+            G = torch.randn(m, n, generator=g, device=device) * noise
+            P = torch.randn(m, rank, generator=g, device=device)
+            Q = torch.randn(n, rank, generator=g, device=device)
+            S = P @ Q.T
+            S *= ratio * G.norm() / S.norm()
+            G += S
+            del S, P, Q
+            Ws.append(W)
+            Gs.append(G)
+            Bs.append(torch.zeros_like(W))
+            shapes.append((m, n))
+    return Ws, Gs, Bs, shapes
+
+
+def moe_workload(device, layers=4, experts=128, hidden=2048, ffn=768, noise=1e-3):
+    import torch
+    import workloads as wl
+    Ws, Gs, Bs, shapes = [], [], [], []
+    for layer in range(layers):
+        for e in range(experts):
+            g = torch.Generator(device=device)
+            g.manual_seed(wl.seed_of("bench-cfg3", layer, e))
+            scale = float(torch.randn(1, generator=g, device=device).exp())
+            for m, n in ((ffn, hidden), (ffn, hidden), (hidden, ffn)):
+                Ws.append(torch.randn(m, n, generator=g, device=device) * 0.02)
+                Gs.append(torch.randn(m, n, generator=g, device=device) * (noise * scale))
+                Bs.append(torch.zeros(m, n, device=device))
+                shapes.append((m, n))
+    return Ws, Gs, Bs, shapes
+
+
+def time_steps(fn, steps, warmup, sync_all=None):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if sync_all:
+        sync_all()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+    from matrix_aware_optimizers_muon_b200 import OP_MUON, Context
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    peaks, peak_kind = load_peaks()
+    ctx = Context(local)
+    Ws, Gs, Bs, shapes = gpt_workload(dev)
+    ctx.reserve(OP_MUON, shapes)
+    torch.cuda.synchronize()
+    flops_page = sum(page_flops(m, n) for m, n in shapes)
+    flops_gemm = sum(gemm_alg_flops(m, n) for m, n in shapes)
+    params = sum(m * n for m, n in shapes)
+
+    def step():
+        ctx.muon_step(Ws, Gs, Bs, lr=0.02, weight_decay=0.01, momentum=0.95, reserve=False)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ctx.profile(True)
+    ctx.profile_read()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    clk = clocks.stop()
+    prof = ctx.profile_read()
+    ctx.profile(False)
+    status = ctx.device_status()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    gemm_ms = sum(prof[k][0] for k in ("gram", "poly", "update"))
+    gemm_exec = sum(prof[k][1] for k in ("gram", "poly", "update"))
+    gemm_launches = sum(prof[k][2] for k in ("gram", "poly", "update"))
+    ew_ms = prof["prep"][0] + prof["apply"][0]
+    launches = int(sum(v[2] for v in prof.values()))
+    gemm_tf = flops_gemm * args.steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    ew_bytes = 24.0 * params
+    ew_gbs = ew_bytes * args.steps / (ew_ms / 1e3) / 1e9 if ew_ms > 0 else None
+
+    value = flops_page * world / (ms / 1e3) / 1e12
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded gradients: N(0,1e-3^2) + rank-16 spike at 10x norm; W ~ N(0,0.02^2))",
+        "config": {"workload": WORKLOAD, "matrices": len(shapes), "params": params,
+                   "ns_steps": 5, "coeffs": [3.4445, -4.775, 2.0315],
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs (84 GB) far larger than L2; no flush"},
+        "matrices_per_s": round(len(shapes) * world / (ms / 1e3), 2),
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "gemm_bf16_kernel (tcgen05; Gram + polynomial + update, all NS products)",
+            "achieved": round(gemm_tf, 2) if gemm_tf else None,
+            "peak": peak_tf,
+            "unit": "TFLOP/s",
+            "frac": round(gemm_tf / peak_tf, 4) if gemm_tf else None,
+            "peak_source": f"{peak_kind} bf16_tflops_sustained",
+            "traffic": None,
+            "alg_flops_per_step": flops_gemm,
+            "exec_flops_per_step": gemm_exec / args.steps,
+            "launches_per_step": gemm_launches / args.steps,
+            "ms_per_step": round(gemm_ms / args.steps, 3),
+        },
+        "roofline_elementwise": {
+            "bound": "hbm",
+            "kernel": "prep_kernel + apply_kernel (24 B/param)",
+            "achieved": round(ew_gbs, 1) if ew_gbs else None,
+            "peak": peaks.get("hbm_gbs"),
+            "unit": "GB/s",
+            "frac": round(ew_gbs / peaks["hbm_gbs"], 4) if ew_gbs else None,
+            "ms_per_step": round(ew_ms / args.steps, 3),
+        },
+        "kernels_ms_per_step": {k: round(v[0] / args.steps, 3) for k, v in prof.items() if v[2]},
+        "gpu_launches": launches,
+        "device_status": status,
+        "clocks": clk,
+    }
+
+    # end to end through the public API with host buffers
+    if args.e2e:
+        out["e2e"] = e2e_measure(ctx, Ws, Gs, Bs, flops_page, world, barrier, args)
+    del Ws, Gs, Bs
+    ctx.workspace = None
+    torch.cuda.empty_cache()
+
+    if args.extras and world == 1:
+        out["extra"] = extras(ctx, dev, args)
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if world > 1:
+        dist.destroy_process_group()
+    return out
+
+
+def e2e_measure(ctx, Ws, Gs, Bs, flops_page, world, barrier, args):
+    import torch
+    steps = max(1, min(args.steps, 2))
+    try:
+        host = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in Gs]
+        for h, g in zip(host, Gs):
+            h.copy_(g)
+        flags = torch.zeros(len(Gs), dtype=torch.int32, device=Gs[0].device)
+        flags_h = torch.empty(len(Gs), dtype=torch.int32, pin_memory=True)
+    except RuntimeError as exc:
+        return {"value": None, "unit": UNIT, "reason": f"pinned host allocation failed: {exc}"[:200]}
+    h2d = sum(h.numel() * 4 for h in host)
+
+    def step():
+        for h, g in zip(host, Gs):
+            g.copy_(h, non_blocking=True)
+        ctx.muon_step(Ws, Gs, Bs, lr=0.02, weight_decay=0.01, momentum=0.95, nonfinite=flags,
+                      reserve=False)
+        flags_h.copy_(flags, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    barrier()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    del host
+    return {"value": round(flops_page * world / (ms / 1e3) / 1e12, 2), "unit": UNIT,
+            "ms_per_step": round(ms, 3), "steps": steps, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": len(Gs) * 4, "nonfinite": int(flags_h.sum())}
+
+
+def dyadic_gpu(n, dev, cond=1e4):
+    """The sweep's known-SVD square input (workloads.dyadic recipe), built on
+    the device: G[i, j] = g[i xor j]."""
+    import torch
+    import workloads as wl
+    d = wl.dyadic_spectrum(wl.rng_of("cfg5", n), n, cond)
+    g = torch.from_numpy(wl.fwht(d) / n).to(dev, torch.float32)
+    idx = torch.arange(n, device=dev)
+    return g[idx[:, None] ^ idx[None, :]].contiguous()
+
+
+def heads_gpu(count, dim, dev, cond=1e4):
+    """Batched per-head inputs U diag(s) V^T with Haar-random U, V."""
+    import torch
+    import workloads as wl
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed_of("bench-heads", count, dim))
+    s = torch.from_numpy(wl.geometric_spectrum(dim, cond)).to(dev, torch.float32)
+    s = s * (dim / s.norm())
+    U, _ = torch.linalg.qr(torch.randn(count, dim, dim, generator=g, device=dev))
+    V, _ = torch.linalg.qr(torch.randn(count, dim, dim, generator=g, device=dev))
+    G = (U * s) @ V.transpose(1, 2)
+    return [G[i].contiguous() for i in range(count)]
+
+
+def extras(ctx, dev, args):
+    """The other workloads, measured the same way (short runs)."""
+    import torch
+    import workloads as wl
+    res = {}
+    # single 256 x 512 Muon step (latency)
+    W, G, B = (torch.from_numpy(x).to(dev) for x in wl.cfg1())
+    ctx.reserve(0, [(256, 512)])
+    ms = time_steps(lambda: ctx.muon_step([W], [G], [B], reserve=False), 50, 5)
+    res["muon_256x512_us"] = round(ms * 1e3, 1)
+    ctx.workspace = None
+    # MoE experts, grouped
+    Ws, Gs, Bs, shapes = moe_workload(dev)
+    ctx.reserve(0, shapes)
+    ms = time_steps(lambda: ctx.muon_step(Ws, Gs, Bs, reserve=False), 5, 2)
+    fl = sum(page_flops(m, n) for m, n in shapes)
+    res["muon_moe_1536x768x2048"] = {"ms": round(ms, 3), "TFLOP/s": round(fl / (ms / 1e3) / 1e12, 1),
+                                     "matrices_per_s": round(len(shapes) / (ms / 1e3), 1)}
+    del Ws, Gs, Bs
+    ctx.workspace = None
+    torch.cuda.empty_cache()
+    # Newton-Schulz sweep on known-SVD inputs (condition number 1e4)
+    sweep = {}
+    for n in (512, 1024, 2048, 4096, 8192, 16384):
+        Gt = dyadic_gpu(n, dev)
+        out = torch.empty_like(Gt)
+        ctx.reserve(2, [(n, n)])
+        reps = 10 if n <= 4096 else 3
+        ms = time_steps(lambda: ctx.ns_orthogonalize([Gt], [out], reserve=False), reps, 2)
+        sweep[str(n)] = {"ms": round(ms, 3), "TFLOP/s": round(page_flops(n, n) / (ms / 1e3) / 1e12, 1)}
+        del Gt, out
+        ctx.workspace = None
+        torch.cuda.empty_cache()
+    Ht = heads_gpu(4096, 128, dev)
+    Ho = [torch.empty_like(h) for h in Ht]
+    ctx.reserve(2, [(128, 128)] * 4096)
+    ms = time_steps(lambda: ctx.ns_orthogonalize(Ht, Ho, reserve=False), 5, 2)
+    sweep["heads_4096x128x128"] = {"ms": round(ms, 3),
+                                   "TFLOP/s": round(4096 * page_flops(128, 128) / (ms / 1e3) / 1e12, 2)}
+    res["ns_sweep"] = sweep
+    del Ht, Ho
+    ctx.workspace = None
+    torch.cuda.empty_cache()
+    return res
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(seconds):
+    """The fp64 oracle as it stands, on this host's cores, on a bounded
+    sample of the same workload: Muon steps on layer-0 matrices of the dense
+    GPT (Wk, Wv: 1024 x 4096; then Wq if time allows)."""
+    import numpy as np
+    import workloads as wl
+    from oracle import muon as omuon
+    cores = len(os.sched_getaffinity(0))
+    done_flops, t_total, names = 0.0, 0.0, []
+    for name, m, n in [("wk", 1024, 4096), ("wv", 1024, 4096), ("wq", 4096, 4096)]:
+        W, G = wl.cfg2_matrix(0, name, m, n)
+        B = np.zeros_like(W)
+        t = time.perf_counter()
+        omuon.muon_step(W, G, B)
+        t_total += time.perf_counter() - t
+        done_flops += page_flops(m, n)
+        names.append(f"{name} {m}x{n}")
+        if t_total > seconds:
+            break
+    return {"value": round(done_flops / t_total / 1e12, 5), "unit": UNIT, "cores": cores,
+            "kind": "oracle", "seconds": round(t_total, 2),
+            "sample": "fp64 NumPy Muon steps on layer-0 matrices of the dense GPT: " + ", ".join(names)}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the oracle, timed on the host cores."""
+    if rank != 0:
+        return None
+    cores = len(os.sched_getaffinity(0))
+    import numpy as np
+    import workloads as wl
+    from oracle import muon as omuon
+    W, G = wl.cfg2_matrix(0, "wk", 1024, 4096)
+    B = np.zeros_like(W)
+    fl = page_flops(1024, 4096)
+    for _ in range(args.warmup):
+        omuon.muon_step(W, G, B)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        omuon.muon_step(W, G, B)
+    dt = (time.perf_counter() - t) / args.steps
+    value = round(fl / dt / 1e12, 5)
+    sample = "one fp64 NumPy Muon step on the layer-0 Wk matrix (1024 x 4096) per step"
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-extras", dest="extras", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        out = run_reference(args, world, rank)
+    else:
+        out = run_ours(args, world, rank, local)
+    if rank == 0 and out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

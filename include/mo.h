@@ -1,0 +1,219 @@
+/*
+ * mo.h - C ABI of the matrix-aware optimizer-step library (Muon, SOAP and
+ * the Newton-Schulz orthogonaliser) for NVIDIA B200 (sm_100a).
+ *
+ * Conventions for every call below
+ * --------------------------------
+ *  - Matrices are fp32, row-major and contiguous (leading dimension == cols)
+ *    and live in device memory of the context's GPU.  Base pointers must be
+ *    4-byte aligned; 16-byte alignment with cols % 4 == 0 enables the
+ *    vectorised path.
+ *  - The caller owns every buffer: parameters, gradients, optimizer state and
+ *    the workspace.  The library never allocates device memory; it owns only
+ *    the host-side context.  The workspace is attached with
+ *    mo_set_workspace() and must be at least mo_workspace_bytes(.., min) large.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are stream-ordered and asynchronous: they validate on
+ *    the host, enqueue kernels and return without synchronising.
+ *  - Parameters and state are updated in place; gradients are read only.  A
+ *    matrix whose gradient pointer is NULL is skipped entirely (its state is
+ *    not advanced), the "grad is None" rule of the LLM Optimizers guide,
+ *    section 6.2.
+ *  - Errors: invalid arguments are reported before any launch with a
+ *    negative status and a message from mo_last_error().  Nothing falls back
+ *    to the CPU: a call that cannot run on the GPU fails.
+ *  - Non-finite values propagate (as in the published recurrences).  The
+ *    optional `nonfinite` arrays receive, per matrix, 1 when the quantity
+ *    named in the config is not finite and 0 otherwise, written on the
+ *    device without a host synchronisation.
+ *  - Kernels never wait without a bound: a wait that exceeds two seconds
+ *    records a code in the context's device status word, read back with
+ *    mo_device_status().
+ *  - One context per host thread.
+ */
+#ifndef MO_H_
+#define MO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MO_API __attribute__((visibility("default")))
+#else
+#define MO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MO_OK = 0,
+  MO_ERR_INVALID_ARG = -1,   /* null pointer, bad size or hyperparameter */
+  MO_ERR_UNSUPPORTED = -2,   /* valid request this build cannot run */
+  MO_ERR_NO_WORKSPACE = -3,  /* no workspace attached, or too small */
+  MO_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
+  MO_ERR_DEVICE = -5         /* the device status word reports a timeout */
+} mo_status;
+
+typedef struct mo_ctx mo_ctx;
+
+/* Create a context bound to CUDA device `device`.  Host memory only. */
+MO_API mo_status mo_ctx_create(mo_ctx** ctx, int device);
+MO_API void mo_ctx_destroy(mo_ctx* ctx);
+
+/* Last error message of this context (host string, valid until the next
+ * call on the same context).  Never NULL. */
+MO_API const char* mo_last_error(const mo_ctx* ctx);
+
+/* Library version string. */
+MO_API const char* mo_version(void);
+
+/* ------------------------------------------------------------------ workspace
+ * Workspace needed by `op` (0 = muon_step, 1 = soap_step, 2 =
+ * ns_orthogonalize) for the n matrices of shapes rows[i] x cols[i] (host
+ * arrays).  *full_bytes lets every group of equal-shape matrices run in one
+ * batch; *min_bytes is the least that works (one matrix at a time).  Either
+ * output pointer may be NULL. */
+MO_API mo_status mo_workspace_bytes(mo_ctx* ctx, int op, const int64_t* rows, const int64_t* cols, int n,
+                             size_t* min_bytes, size_t* full_bytes);
+
+/* Attach caller-allocated device memory (256-byte aligned).  The library
+ * keeps the pointer until the next call; the caller keeps ownership and must
+ * not free it while work that uses it is in flight.  Attaching clears the
+ * device status word with a stream-ordered memset on `stream`. */
+MO_API mo_status mo_set_workspace(mo_ctx* ctx, void* dev_ptr, size_t bytes, void* stream);
+
+/* Copy the device status word to *status (0 = no timeout recorded) and clear
+ * it.  Synchronises `stream`.  Returns MO_ERR_DEVICE when the word was set. */
+MO_API mo_status mo_device_status(mo_ctx* ctx, void* stream, int32_t* status);
+
+/* ------------------------------------------------------------------ profiling
+ * With profiling enabled, every kernel the following calls launch is
+ * bracketed by a CUDA event pair on its stream.  mo_profile_read()
+ * synchronises those events and returns, per kernel kind k < nkinds (host
+ * arrays), the summed elapsed milliseconds, the executed tensor-core flops
+ * and the launch count, then forgets the records.  Kinds: 0 Muon momentum /
+ * cast, 1 norm finalize, 2 Gram X X^T, 3 polynomial b A + c A A, 4 update
+ * a X + P X, 5 apply / store, 6 SOAP elementwise, 7 SOAP products, 8 SOAP
+ * QR, 9 mo_gemm_bf16. */
+MO_API mo_status mo_profile_enable(mo_ctx* ctx, int enable);
+MO_API mo_status mo_profile_read(mo_ctx* ctx, double* ms, double* flops, int64_t* launches, int nkinds);
+
+/* ------------------------------------------------------------------ Muon
+ * One Muon step per matrix ("Matrix optimizers: K-FAC, Shampoo and Muon",
+ * section "Muon", steps 1-4; "LLM Optimizers: From SGD and AdamW to SOAP,
+ * Muon, and Scalable Training", sections 11.3-11.5):
+ *   B <- beta B + G            (momentum_ema: B <- beta B + (1 - beta) G)
+ *   N  = G + beta B            (nesterov; else N = B)
+ *   O  = NS(N): ns_steps quintic Newton-Schulz iterations on
+ *        N / (||N||_F + eps), tall matrices transposed so that the Gram
+ *        matrix is the smaller one; bf16 operands, fp32 accumulation, every
+ *        stored iterate rounded to bf16 (nearest-even); the normalisation
+ *        scale is applied in fp32 inside the first iteration
+ *   W <- (1 - lr wd) W - lr s O,  s = 0.2 sqrt(max(m, n))  (adjust_lr 0)
+ *                                 s = sqrt(max(1, m / n))   (adjust_lr 1)
+ * Matrices of equal (oriented) shape are batched into grouped launches. */
+typedef struct {
+  int64_t rows, cols;   /* m, n */
+  float* W;             /* parameter, updated in place */
+  const float* G;       /* gradient; NULL skips this matrix */
+  float* momentum;      /* momentum buffer B (zero before the first step) */
+} mo_muon_mat;
+
+typedef struct {
+  float lr, weight_decay, momentum;  /* lr >= 0, wd >= 0, 0 <= momentum < 1 */
+  int nesterov;                      /* 1: N = G + beta B (default); 0: N = B */
+  int momentum_ema;                  /* 0: B = beta B + G (default); 1: EMA form */
+  int ns_steps;                      /* 1..64 (5) */
+  float a, b, c;                     /* (3.4445, -4.7750, 2.0315) */
+  float eps;                         /* 1e-7 */
+  int adjust_lr;                     /* 0: 0.2 sqrt(max(m,n)); 1: sqrt(max(1,m/n)) */
+  int32_t* nonfinite;                /* optional device int32[n]: ||N||_F not finite */
+} mo_muon_cfg;
+
+MO_API mo_status muon_step(mo_ctx* ctx, const mo_muon_mat* mats /* host array */, int n,
+                    const mo_muon_cfg* cfg, void* stream);
+
+/* ------------------------------------------------------------------ Newton-Schulz
+ * O_i = NS(in_i) for n matrices of possibly different shapes, with the same
+ * iteration and rounding points as muon_step (section 11.4 of the LLM
+ * Optimizers guide).  in/out/rows/cols are host arrays of device pointers
+ * and sizes; out_i has in_i's shape and receives the bf16 iterate widened to
+ * fp32.  in_i and out_i must not overlap. */
+typedef struct {
+  int ns_steps;         /* 1..64 */
+  float a, b, c;
+  float eps;
+  int32_t* nonfinite;   /* optional device int32[n]: ||in_i||_F not finite */
+} mo_ns_cfg;
+
+MO_API mo_status ns_orthogonalize(mo_ctx* ctx, const float* const* in, float* const* out,
+                           const int64_t* rows, const int64_t* cols, int n, const mo_ns_cfg* cfg,
+                           void* stream);
+
+/* ------------------------------------------------------------------ SOAP
+ * One SOAP step per matrix with a per-step eigenbasis refresh ("Reading
+ * notes on SOAP, Muon, and Beyond", sections 1 and 4; "LLM Optimizers",
+ * section 11.1; "初探优化器（一）", section 6.2), at step t >= 1:
+ *   L <- bs L + (1 - bs) G G^T,   R <- bs R + (1 - bs) G^T G
+ *   Q_L <- qr(L Q_L),             Q_R <- qr(R Q_R)   (one power step + QR,
+ *                                  diag(R) > 0; fp32-accurate)
+ *   M <- b1 M + (1 - b1) G        (original space)
+ *   M' = Q_L^T M Q_R,  G' = Q_L^T G Q_R
+ *   V <- b2 V + (1 - b2) G' * G'
+ *   Dbar = (M' / (1 - b1^t)) / (sqrt(V / (1 - b2^t)) + eps)
+ *   W <- (1 - lr wd) W - lr Q_L Dbar Q_R^T
+ * A side with L == NULL (resp. R == NULL) uses the identity basis; Q_* then
+ * must be NULL too.  Tensor-core products take bf16 operands with fp32
+ * accumulation; L, R, Q_*, M, V stay fp32.  Initial state: L = R = M = V = 0,
+ * Q = I. */
+typedef struct {
+  int64_t rows, cols;   /* m, n */
+  float* W;
+  const float* G;       /* NULL skips this matrix */
+  float* M;             /* first moment, m x n */
+  float* V;             /* second moment in the rotated basis, m x n */
+  float* L;             /* m x m factor, or NULL (identity left basis) */
+  float* QL;            /* m x m basis, or NULL */
+  float* R;             /* n x n factor, or NULL (identity right basis) */
+  float* QR;            /* n x n basis, or NULL */
+} mo_soap_mat;
+
+typedef struct {
+  float lr, beta1, beta2, shampoo_beta, eps, weight_decay;
+  int bias_correction;  /* 1: divide by 1 - beta^t (default) */
+  int32_t* nonfinite;   /* optional device int32[n]: the QR met a non-positive pivot */
+} mo_soap_cfg;
+
+MO_API mo_status soap_step(mo_ctx* ctx, const mo_soap_mat* mats /* host array */, int n,
+                    const mo_soap_cfg* cfg, int64_t step, void* stream);
+
+/* ------------------------------------------------------------------ building block
+ * The batched tensor-core GEMM the steps are built from, exposed for tests
+ * and for callers composing their own variants:
+ *   D_b = alpha s_b^alpha_pow (A_b B_b) + beta s_b^beta_pow C_b,  b < batch
+ * A is M x K stored K-major ([M][K]) or, with a_mn, MN-major ([K][M]); B is
+ * K x N stored K-major ([N][K]) or, with b_mn, MN-major ([K][N]).  A and B
+ * are bf16 (uint16 storage) with row strides that are multiples of 8
+ * elements and 16-byte aligned bases.  C and D are bf16 or fp32 (c_f32,
+ * d_f32); C may be NULL or alias D.  With sym set the product must be
+ * symmetric (M == N): only tiles that touch the upper triangle are computed
+ * and each upper element is also written to its mirror position. */
+typedef struct {
+  const void* A; int64_t lda, strideA; int a_mn;
+  const void* B; int64_t ldb, strideB; int b_mn;
+  int M, N, K, batch, sym;
+  float alpha, beta;
+  const float* scale; int alpha_pow, beta_pow;   /* scale may be NULL */
+  const void* C; int64_t ldc, strideC; int c_f32;
+  void* D; int64_t ldd, strideD; int d_f32;
+} mo_gemm_desc;
+
+MO_API mo_status mo_gemm_bf16(mo_ctx* ctx, const mo_gemm_desc* desc, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MO_H_ */

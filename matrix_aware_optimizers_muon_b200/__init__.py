@@ -1,0 +1,213 @@
+"""Matrix-aware optimizer steps (Muon, SOAP, Newton-Schulz) on NVIDIA B200.
+
+A thin Python binding of the C ABI in ``include/mo.h``: it turns torch
+tensors into device pointers and the current CUDA stream into a handle, and
+allocates the workspace with torch.  Every step of the computation runs in the
+sm_100a kernels of ``libmo.so``; when that library is missing, importing the
+binding's entry points fails.
+"""
+
+import ctypes
+from ctypes import byref, c_int32, c_int64, c_size_t, c_void_p
+
+from . import _lib
+from ._lib import (GemmDesc, MuonCfg, MuonMat, NsCfg, SoapCfg, SoapMat, OP_MUON, OP_NS,
+                   OP_SOAP)
+
+__all__ = ["Context", "MoError", "QUINTIC", "OP_MUON", "OP_SOAP", "OP_NS"]
+
+QUINTIC = (3.4445, -4.7750, 2.0315)
+
+
+class MoError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"mo status {status}: {message}")
+        self.status = status
+
+
+def _ptr(t):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def _check_f32(t, name):
+    import torch
+    if t is None:
+        return
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+
+
+class Context:
+    """One library context on one CUDA device, with a torch-owned workspace."""
+
+    def __init__(self, device=None):
+        import torch
+        self.lib = _lib.load()
+        self.device = torch.cuda.current_device() if device is None else int(device)
+        h = c_void_p()
+        st = self.lib.mo_ctx_create(byref(h), self.device)
+        if st != 0:
+            raise MoError(st, "mo_ctx_create failed")
+        self.handle = h
+        self.workspace = None
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self.lib.mo_ctx_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------ helpers
+    def _stream(self, stream):
+        import torch
+        s = torch.cuda.current_stream(self.device) if stream is None else stream
+        return c_void_p(s.cuda_stream)
+
+    def _check(self, st):
+        if st != 0:
+            raise MoError(st, self.lib.mo_last_error(self.handle).decode())
+
+    def workspace_bytes(self, op, shapes):
+        n = len(shapes)
+        rows = (c_int64 * max(n, 1))(*[int(s[0]) for s in shapes])
+        cols = (c_int64 * max(n, 1))(*[int(s[1]) for s in shapes])
+        mn, full = c_size_t(), c_size_t()
+        self._check(self.lib.mo_workspace_bytes(self.handle, op, rows, cols, n, byref(mn), byref(full)))
+        return mn.value, full.value
+
+    def attach_workspace(self, nbytes, stream=None):
+        """Allocate ``nbytes`` of device memory with torch and attach it."""
+        import torch
+        buf = torch.empty(int(nbytes), dtype=torch.uint8, device=f"cuda:{self.device}")
+        self._check(self.lib.mo_set_workspace(self.handle, c_void_p(buf.data_ptr()), buf.numel(),
+                                              self._stream(stream)))
+        self.workspace = buf
+        return buf
+
+    def reserve(self, op, shapes, full=True, stream=None):
+        """Make sure the attached workspace fits ``op`` on ``shapes``."""
+        mn, fb = self.workspace_bytes(op, shapes)
+        need = fb if full else mn
+        if self.workspace is None or self.workspace.numel() < need:
+            self.attach_workspace(need, stream)
+
+    def device_status(self, stream=None):
+        v = c_int32()
+        st = self.lib.mo_device_status(self.handle, self._stream(stream), byref(v))
+        if st not in (0, _lib.MO_ERR_DEVICE):
+            self._check(st)
+        return v.value
+
+    def profile(self, enable=True):
+        self._check(self.lib.mo_profile_enable(self.handle, int(enable)))
+
+    def profile_read(self):
+        """{kind: (ms, executed_flops, launches)} since the last read."""
+        n = len(_lib.KINDS)
+        ms = (ctypes.c_double * n)()
+        fl = (ctypes.c_double * n)()
+        ln = (c_int64 * n)()
+        self._check(self.lib.mo_profile_read(self.handle, ms, fl, ln, n))
+        return {k: (ms[i], fl[i], ln[i]) for i, k in enumerate(_lib.KINDS)}
+
+    # ------------------------------------------------------------ entry points
+    def muon_step(self, W, G, B, *, lr=0.02, weight_decay=0.01, momentum=0.95, nesterov=True,
+                  momentum_ema=False, ns_steps=5, coeffs=QUINTIC, eps=1e-7,
+                  adjust_lr="match_rms_adamw", nonfinite=None, stream=None, reserve=True):
+        """One Muon step on lists of fp32 CUDA matrices (G entries may be None)."""
+        n = len(W)
+        if not (len(G) == len(B) == n):
+            raise ValueError("W, G and B must have the same length")
+        mats = (MuonMat * max(n, 1))()
+        for i in range(n):
+            for t, nm in ((W[i], "W"), (G[i], "G"), (B[i], "momentum")):
+                _check_f32(t, f"{nm}[{i}]")
+            if W[i].dim() != 2 or (G[i] is not None and G[i].shape != W[i].shape) or B[i].shape != W[i].shape:
+                raise ValueError(f"matrix {i}: W, G and momentum must be 2-D with one shape")
+            mats[i] = MuonMat(W[i].shape[0], W[i].shape[1], _ptr(W[i]), _ptr(G[i]), _ptr(B[i]))
+        if reserve:
+            self.reserve(OP_MUON, [tuple(w.shape) for w in W], stream=stream)
+        modes = {"match_rms_adamw": 0, "original": 1}
+        cfg = MuonCfg(lr, weight_decay, momentum, int(nesterov), int(momentum_ema), ns_steps,
+                      coeffs[0], coeffs[1], coeffs[2], eps, modes[adjust_lr],
+                      _ptr(nonfinite))
+        self._check(self.lib.muon_step(self.handle, mats, n, byref(cfg), self._stream(stream)))
+
+    def ns_orthogonalize(self, inputs, outputs=None, *, ns_steps=5, coeffs=QUINTIC, eps=1e-7,
+                         nonfinite=None, stream=None, reserve=True):
+        """O_i = NS(in_i); returns the list of fp32 outputs."""
+        import torch
+        n = len(inputs)
+        if outputs is None:
+            outputs = [torch.empty_like(x) for x in inputs]
+        ins = (c_void_p * max(n, 1))()
+        outs = (c_void_p * max(n, 1))()
+        rows = (c_int64 * max(n, 1))()
+        cols = (c_int64 * max(n, 1))()
+        for i, (x, y) in enumerate(zip(inputs, outputs)):
+            _check_f32(x, f"in[{i}]")
+            _check_f32(y, f"out[{i}]")
+            if x.dim() != 2 or y.shape != x.shape:
+                raise ValueError(f"matrix {i}: input and output must be 2-D with one shape")
+            ins[i], outs[i] = x.data_ptr(), y.data_ptr()
+            rows[i], cols[i] = x.shape
+        if reserve:
+            self.reserve(OP_NS, [tuple(x.shape) for x in inputs], stream=stream)
+        cfg = NsCfg(ns_steps, coeffs[0], coeffs[1], coeffs[2], eps, _ptr(nonfinite))
+        self._check(self.lib.ns_orthogonalize(self.handle, ins, outs, rows, cols, n, byref(cfg),
+                                              self._stream(stream)))
+        return outputs
+
+    def soap_step(self, mats, step, *, lr=3e-3, beta1=0.95, beta2=0.95, shampoo_beta=None,
+                  eps=1e-8, weight_decay=0.0, bias_correction=True, nonfinite=None, stream=None,
+                  reserve=True):
+        """One SOAP step.  ``mats`` is a list of dicts with keys W, G, M, V and
+        optionally L, QL, R, QR (missing or None: identity basis on that side)."""
+        n = len(mats)
+        arr = (SoapMat * max(n, 1))()
+        for i, d in enumerate(mats):
+            for k in ("W", "G", "M", "V", "L", "QL", "R", "QR"):
+                _check_f32(d.get(k), f"{k}[{i}]")
+            W = d["W"]
+            arr[i] = SoapMat(W.shape[0], W.shape[1], _ptr(W), _ptr(d.get("G")), _ptr(d["M"]),
+                             _ptr(d["V"]), _ptr(d.get("L")), _ptr(d.get("QL")), _ptr(d.get("R")),
+                             _ptr(d.get("QR")))
+        if reserve:
+            self.reserve(OP_SOAP, [tuple(d["W"].shape) for d in mats], stream=stream)
+        sb = beta2 if shampoo_beta is None else shampoo_beta
+        cfg = SoapCfg(lr, beta1, beta2, sb, eps, weight_decay, int(bias_correction), _ptr(nonfinite))
+        self._check(self.lib.soap_step(self.handle, arr, n, byref(cfg), int(step), self._stream(stream)))
+
+    def gemm_bf16(self, A, B, D, *, M, N, K, batch=1, a_mn=False, b_mn=False, sym=False,
+                  alpha=1.0, beta=0.0, C=None, scale=None, alpha_pow=0, beta_pow=0,
+                  lda=None, ldb=None, ldc=None, ldd=None, strideA=None, strideB=None,
+                  strideC=None, strideD=None, stream=None):
+        """Batched bf16 tensor-core GEMM with the fused epilogue (see mo.h)."""
+        import torch
+
+        def ld_of(t):
+            return t.shape[-1]
+
+        def stride_of(t):
+            return t.shape[-1] * t.shape[-2] if t.dim() == 3 else 0
+
+        d = GemmDesc()
+        d.A, d.lda, d.strideA, d.a_mn = A.data_ptr(), lda or ld_of(A), strideA or stride_of(A), int(a_mn)
+        d.B, d.ldb, d.strideB, d.b_mn = B.data_ptr(), ldb or ld_of(B), strideB or stride_of(B), int(b_mn)
+        d.M, d.N, d.K, d.batch, d.sym = M, N, K, batch, int(sym)
+        d.alpha, d.beta = alpha, beta
+        d.scale = None if scale is None else scale.data_ptr()
+        d.alpha_pow, d.beta_pow = alpha_pow, beta_pow
+        if C is not None:
+            d.C, d.ldc, d.strideC = C.data_ptr(), ldc or ld_of(C), strideC or stride_of(C)
+            d.c_f32 = int(C.dtype == torch.float32)
+        d.D, d.ldd, d.strideD = D.data_ptr(), ldd or ld_of(D), strideD or stride_of(D)
+        d.d_f32 = int(D.dtype == torch.float32)
+        if self.workspace is None:
+            self.attach_workspace(4096, stream)
+        self._check(self.lib.mo_gemm_bf16(self.handle, byref(d), self._stream(stream)))

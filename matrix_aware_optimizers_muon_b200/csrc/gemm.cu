@@ -1,0 +1,118 @@
+// Host side of the tcgen05 GEMM: TMA descriptor encoding and launch.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "gemm.cuh"
+#include "profile.h"
+#include "runtime.h"
+
+namespace mo {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void load_encode_fn() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult qres;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) == cudaSuccess &&
+      qres == cudaDriverEntryPointSuccess) {
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+}
+
+// 3-D bf16 tensor map over `batch` matrices of storage rows x cols (row
+// stride ld, matrix stride bstride, both in elements); box = 64 x box_rows.
+bool encode_bf16_3d(CUtensorMap* map, const void* ptr, long long rows, long long cols, long long ld,
+                    long long bstride, int batch, int box_rows) {
+  std::call_once(g_encode_once, load_encode_fn);
+  if (g_encode == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)((batch > 1 ? bstride : rows * ld) * 2)};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int A_MN, int B_MN>
+cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
+  using Cfg = GemmCfg<BN>;
+  CUtensorMap ta, tb;
+  const bool ok_a = A_MN ? encode_bf16_3d(&ta, op.A, op.K, op.M, op.lda, op.strideA, op.batch, 64)
+                         : encode_bf16_3d(&ta, op.A, op.M, op.K, op.lda, op.strideA, op.batch, GEMM_BM);
+  const bool ok_b = B_MN ? encode_bf16_3d(&tb, op.B, op.K, op.N, op.ldb, op.strideB, op.batch, 64)
+                         : encode_bf16_3d(&tb, op.B, op.N, op.K, op.ldb, op.strideB, op.batch, BN);
+  if (!ok_a || !ok_b) return cudaErrorInvalidValue;
+
+  GemmParams p;
+  p.M = op.M; p.N = op.N; p.K = op.K; p.batch = op.batch;
+  p.tiles_m = (op.M + GEMM_BM - 1) / GEMM_BM;
+  p.tiles_n = (op.N + BN - 1) / BN;
+  p.sym = op.sym;
+  p.alpha = op.alpha; p.beta = op.beta; p.scale = op.scale;
+  p.alpha_pow = op.alpha_pow; p.beta_pow = op.beta_pow;
+  p.C = op.C; p.ldc = op.ldc; p.strideC = op.strideC; p.c_f32 = op.c_f32;
+  p.D = op.D; p.ldd = op.ldd; p.strideD = op.strideD; p.d_f32 = op.d_f32;
+  p.status = status;
+
+  auto kern = gemm_bf16_kernel<BN, A_MN, B_MN>;
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = 1;
+  }
+  const long long total = (long long)p.tiles_m * p.tiles_n * p.batch;
+  const int grid = (int)(total < device_sm_count() ? total : device_sm_count());
+  if (grid <= 0) return cudaSuccess;
+  // executed tensor-core flops: computed tiles x 128 x BN x padded K x 2
+  long long tiles = 0;
+  for (int tn = 0; tn < p.tiles_n; ++tn)
+    for (int tm = 0; tm < p.tiles_m; ++tm)
+      if (!(p.sym && tm * GEMM_BM > tn * BN + BN - 1)) ++tiles;
+  const double flops = 2.0 * tiles * p.batch * GEMM_BM * BN * (double)round_up(p.K, GEMM_BK);
+  ProfScope prof(op.kind, stream, flops);
+  kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+cudaError_t launch_gemm(const GemmOp& op, int* status, cudaStream_t stream) {
+  if (op.M <= 0 || op.N <= 0 || op.K <= 0 || op.batch <= 0) return cudaSuccess;
+  // 128-wide N tiles when N is small, 256 otherwise
+  const bool narrow = op.N <= 128;
+  const int sel = (narrow ? 4 : 0) | (op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0);
+  switch (sel) {
+    case 0: return launch_t<256, 0, 0>(op, status, stream);
+    case 1: return launch_t<256, 0, 1>(op, status, stream);
+    case 2: return launch_t<256, 1, 0>(op, status, stream);
+    case 3: return launch_t<256, 1, 1>(op, status, stream);
+    case 4: return launch_t<128, 0, 0>(op, status, stream);
+    case 5: return launch_t<128, 0, 1>(op, status, stream);
+    case 6: return launch_t<128, 1, 0>(op, status, stream);
+    default: return launch_t<128, 1, 1>(op, status, stream);
+  }
+}
+
+}  // namespace mo

@@ -1,0 +1,353 @@
+// Batched bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA, with a fused epilogue  D = alpha_b * (A B) + beta_b * C.
+//
+// One persistent CTA per SM, 6 warps:
+//   warp 0      TMA producer: fills a ring of shared-memory stages
+//   warp 1      MMA issuer: one elected thread issues tcgen05.mma into one
+//               of two TMEM accumulators (so the epilogue of tile i overlaps
+//               the main loop of tile i+1) and commits stage releases
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (warp w reads TMEM
+//               lanes 32*(w%4)..+31 = tile rows), apply alpha/beta/C, store
+//
+// Tiles are 128 x BN (BN = 256 or 128) with BK = 64 (one 128-byte swizzle
+// row of bf16).  A is M x K and B is K x N; each may be stored K-major
+// (K contiguous) or MN-major (M or N contiguous).  With `sym` set the
+// product is known to be symmetric (X X^T, or A A with A symmetric): only
+// tiles that touch the upper triangle are computed, and each upper element
+// is stored at (r, c) and mirrored to (c, r), so both halves are bit-equal.
+#pragma once
+
+#include "ptx.cuh"
+#include <cuda_bf16.h>
+
+namespace mo {
+
+struct GemmParams {
+  int M, N, K;              // per-matrix problem size
+  int batch;                // number of independent matrices
+  int tiles_m, tiles_n;     // tiles per matrix
+  int sym;                  // symmetric product: upper tiles + mirror stores
+  float alpha, beta;        // epilogue coefficients
+  const float* scale;       // optional per-matrix scale s_b (device)
+  int alpha_pow, beta_pow;  // alpha_b = alpha * s_b^alpha_pow, beta_b likewise
+  const void* C;            // optional epilogue input (may alias D)
+  long long ldc, strideC;   // elements
+  int c_f32;                // C is fp32 (else bf16)
+  void* D;                  // output
+  long long ldd, strideD;   // elements
+  int d_f32;                // D is fp32 (else bf16)
+  int* status;              // device status word (timeouts)
+};
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BK = 64;
+constexpr int GEMM_THREADS = 192;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
+  static constexpr int B_BYTES = BN * GEMM_BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int TMEM_COLS = 2 * BN;          // two fp32 accumulators
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+};
+
+__device__ __forceinline__ bool gemm_decode(const GemmParams& p, int BN, int t, int& b, int& tm,
+                                            int& tn) {
+  const int per = p.tiles_m * p.tiles_n;
+  b = t / per;
+  const int u = t - b * per;
+  tn = u / p.tiles_m;          // M fastest: concurrently running CTAs share B columns
+  tm = u - tn * p.tiles_m;
+  if (p.sym && tm * GEMM_BM > tn * BN + BN - 1) return false;   // entirely below diagonal
+  return true;
+}
+
+__device__ __forceinline__ float ipow_scale(const float* s, int b, int pw) {
+  if (s == nullptr || pw == 0) return 1.0f;
+  const float v = s[b];
+  return pw == 1 ? v : v * v;
+}
+
+// Load 32 consecutive C values of row r starting at column c0 (bounded by N).
+__device__ __forceinline__ void load_c32(const GemmParams& p, int b, int r, int c0, float (&c)[32]) {
+  const bool full = c0 + 32 <= p.N;
+  if (p.c_f32) {
+    const float* src = reinterpret_cast<const float*>(p.C) + b * p.strideC + (long long)r * p.ldc + c0;
+    if (full) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 v = reinterpret_cast<const float4*>(src)[i];
+        c[4 * i] = v.x; c[4 * i + 1] = v.y; c[4 * i + 2] = v.z; c[4 * i + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) c[i] = (c0 + i < p.N) ? src[i] : 0.0f;
+    }
+  } else {
+    const __nv_bfloat16* src =
+        reinterpret_cast<const __nv_bfloat16*>(p.C) + b * p.strideC + (long long)r * p.ldc + c0;
+    if (full) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = reinterpret_cast<const uint4*>(src)[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+          c[8 * i + 2 * j] = f.x;
+          c[8 * i + 2 * j + 1] = f.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) c[i] = (c0 + i < p.N) ? __bfloat162float(src[i]) : 0.0f;
+    }
+  }
+}
+
+__device__ __forceinline__ void store_one(const GemmParams& p, int b, int r, int c, float v) {
+  if (p.d_f32) {
+    reinterpret_cast<float*>(p.D)[b * p.strideD + (long long)r * p.ldd + c] = v;
+  } else {
+    reinterpret_cast<__nv_bfloat16*>(p.D)[b * p.strideD + (long long)r * p.ldd + c] =
+        __float2bfloat16_rn(v);
+  }
+}
+
+__device__ __forceinline__ void store_row32(const GemmParams& p, int b, int r, int c0,
+                                            const float (&x)[32]) {
+  if (p.d_f32) {
+    float* dst = reinterpret_cast<float*>(p.D) + b * p.strideD + (long long)r * p.ldd + c0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      reinterpret_cast<float4*>(dst)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+  } else {
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + b * p.strideD + (long long)r * p.ldd + c0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x[8 * i + 2 * j], x[8 * i + 2 * j + 1]);
+        w[j] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+template <int BN, int A_MN, int B_MN>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const GemmParams p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, BN, A_MN, B_MN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* consumed = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *consumed = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int total = p.tiles_m * p.tiles_n * p.batch;
+  const int nk = (p.K + GEMM_BK - 1) / GEMM_BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int b, tm, tn;
+        if (!gemm_decode(p, BN, t, b, tm, tn)) continue;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, DEV_TIMEOUT_EMPTY)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
+          uint8_t* sb = sa + Cfg::A_BYTES;
+          if (!A_MN) {
+            tma_load_3d(sa, &tmA, &full[stage], kb * GEMM_BK, tm * GEMM_BM, b);
+          } else {
+            tma_load_3d(sa, &tmA, &full[stage], tm * GEMM_BM, kb * GEMM_BK, b);
+            tma_load_3d(sa + GEMM_BK * 128, &tmA, &full[stage], tm * GEMM_BM + 64, kb * GEMM_BK, b);
+          }
+          if (!B_MN) {
+            tma_load_3d(sb, &tmB, &full[stage], kb * GEMM_BK, tn * BN, b);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_3d(sb + j * GEMM_BK * 128, &tmB, &full[stage], tn * BN + 64 * j, kb * GEMM_BK, b);
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let every copy already in flight land before the CTA can exit
+        for (int i = *consumed; i < issued; ++i)
+          mbar_wait_drain(&full[i % STAGES], (uint32_t)((i / STAGES) & 1), p.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool any = false, ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int b, tm, tn;
+        if (!gemm_decode(p, BN, t, b, tm, tn)) continue;
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status, DEV_TIMEOUT_ACC_EMPTY)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, DEV_TIMEOUT_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * Cfg::STAGE_BYTES);
+          const uint32_t sb = sa + Cfg::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < GEMM_BK / 16; ++k) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(sa + k * 2048, GEMM_BK * 128, 1024)
+                                     : smem_desc_sw128(sa + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(sb + k * 2048, GEMM_BK * 128, 1024)
+                                     : smem_desc_sw128(sb + k * 32, 16, 1024);
+            tc_mma_f16(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          any = true;
+          tc_commit(&empty[stage]);
+          *consumed = *consumed + 1;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (any) {
+        // every MMA issued by this thread must finish before TMEM is freed
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0, p.status);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int row_in_tile = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      int b, tm, tn;
+      if (!gemm_decode(p, BN, t, b, tm, tn)) continue;
+      // warp-uniform: tcgen05.ld below must be executed by all 32 lanes
+      const bool ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status, DEV_TIMEOUT_ACC_FULL);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int r = tm * GEMM_BM + row_in_tile;
+      const float alpha = p.alpha * ipow_scale(p.scale, b, p.alpha_pow);
+      const float beta = p.beta * ipow_scale(p.scale, b, p.beta_pow);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int cc = 0; cc < BN; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(taddr + cc, v);
+        tmem_ld_wait();
+        const int c0 = tn * BN + cc;
+        if (r < p.M && c0 < p.N) {
+          float x[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = alpha * __uint_as_float(v[i]);
+          if (p.C != nullptr) {
+            float c[32];
+            load_c32(p, b, r, c0, c);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = fmaf(beta, c[i], x[i]);
+          }
+          if (!p.sym) {
+            if (c0 + 32 <= p.N) {
+              store_row32(p, b, r, c0, x);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (c0 + i < p.N) store_one(p, b, r, c0 + i, x[i]);
+            }
+          } else if (c0 + 31 >= r) {
+            // upper part of this row chunk: store it and its mirror image
+            if (c0 >= r && c0 + 32 <= p.N) {
+              store_row32(p, b, r, c0, x);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (c0 + i >= r && c0 + i < p.N) store_one(p, b, r, c0 + i, x[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c0 + i > r && c0 + i < p.N) store_one(p, b, c0 + i, r, x[i]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace mo

@@ -1,0 +1,46 @@
+// Internal host-side interfaces shared by the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mo {
+
+// One batched GEMM D_b = alpha_b * (A_b B_b) + beta_b * C_b on bf16 operands.
+// Operand storage (row-major, element strides):
+//   A: a_mn ? [K rows][M cols] : [M rows][K cols]
+//   B: b_mn ? [K rows][N cols] : [N rows][K cols]
+// Row strides must be multiples of 8 elements and base pointers 16-byte
+// aligned (TMA); C and D may be bf16 or fp32.
+struct GemmOp {
+  const void* A = nullptr;
+  long long lda = 0, strideA = 0;
+  int a_mn = 0;
+  const void* B = nullptr;
+  long long ldb = 0, strideB = 0;
+  int b_mn = 0;
+  int M = 0, N = 0, K = 0, batch = 1;
+  int sym = 0;
+  float alpha = 1.f, beta = 0.f;
+  const float* scale = nullptr;
+  int alpha_pow = 0, beta_pow = 0;
+  const void* C = nullptr;
+  long long ldc = 0, strideC = 0;
+  int c_f32 = 0;
+  void* D = nullptr;
+  long long ldd = 0, strideD = 0;
+  int d_f32 = 0;
+  int kind = 9;          // profiling tag (ProfKind)
+};
+
+// Launch the tcgen05 GEMM.  Returns cudaSuccess or the launch/encode error.
+cudaError_t launch_gemm(const GemmOp& op, int* status, cudaStream_t stream);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+// Round x up to a multiple of a.
+inline long long round_up(long long x, long long a) { return (x + a - 1) / a * a; }
+
+}  // namespace mo

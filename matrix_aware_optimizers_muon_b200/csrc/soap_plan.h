@@ -1,0 +1,26 @@
+// Planning and launch sequence of the SOAP path.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/mo.h"
+
+namespace mo {
+
+struct SoapItem {
+  mo_soap_mat m;
+  int32_t* flag = nullptr;
+};
+
+void soap_workspace(const int64_t* rows, const int64_t* cols, int n, size_t* min_bytes, size_t* full_bytes);
+
+// Enqueue one SOAP step for every item.  Planning errors set *err.
+cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg, int64_t step, char* ws,
+                     size_t ws_bytes, cudaStream_t stream, std::string* err);
+
+}  // namespace mo

@@ -1,0 +1,44 @@
+"""Comparison gates shared by the parity tests (test-side helpers only)."""
+import numpy as np
+
+
+def rel(a, b):
+    """Relative Frobenius error ||a - b|| / ||b||."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
+
+
+def ns_gate(N, O_gpu, O_ref, O_emu, *, tau=1e-2, sub_tol=2e-2, band=(0.6, 1.3), floor=1.25,
+            floor_abs=2e-3, svd=None):
+    """Newton-Schulz parity on the resolved subspace plus a noise-floor gate.
+
+    The iteration multiplies near-null singular directions by up to a^5, so
+    bf16 rounding noise there is amplified whatever the kernel; the check is
+    (1) on the singular subspace with sigma / ||N||_F >= tau: relative error
+        of U_k^T O V_k against the fp64 oracle <= sub_tol and its singular
+        values inside ``band``;
+    (2) on the full matrix: the GPU's error against fp64 is no worse than
+        ``floor`` times the oracle's own bf16-emulation error (+ floor_abs).
+    Returns a dict of the measured numbers (asserts inside).
+    """
+    N = np.asarray(N, dtype=np.float64)
+    tall = N.shape[0] > N.shape[1]
+    if svd is None:
+        U, s, Vt = np.linalg.svd(N, full_matrices=False)
+    else:
+        U, s, Vt = svd
+    k = int(np.sum(s / np.linalg.norm(s) >= tau))
+    Uk, Vk = U[:, :k], Vt[:k].T
+    P = lambda O: Uk.T @ np.asarray(O, dtype=np.float64) @ Vk
+    sub = rel(P(O_gpu), P(O_ref))
+    sv = np.linalg.svd(P(O_gpu), compute_uv=False)
+    full_gpu = rel(O_gpu, O_ref)
+    full_emu = rel(O_emu, O_ref)
+    out = dict(k=k, sub=sub, sv_min=float(sv.min()), sv_max=float(sv.max()), full_gpu=full_gpu,
+               full_emu=full_emu, tall=tall)
+    assert sub <= sub_tol, out
+    assert band[0] <= sv.min() and sv.max() <= band[1], out
+    assert full_gpu <= floor * full_emu + floor_abs, out
+    return out

@@ -152,6 +152,30 @@ MO_API mo_status ns_orthogonalize(mo_ctx* ctx, const float* const* in, float* co
                            const int64_t* rows, const int64_t* cols, int n, const mo_ns_cfg* cfg,
                            void* stream);
 
+/* ------------------------------------------------------------------ no-allocation variant
+ * The pages have no counterpart to this entry point; it serves callers that
+ * cannot allocate device memory when they call it: programs whose GPU
+ * memory belongs to another allocator with nothing spare, runtimes that
+ * forbid allocation after start-up, or plain C hosts with no allocator at
+ * hand.  It computes exactly what ns_orthogonalize computes for ONE matrix,
+ * but its scratch is a fixed device array of MO_STATIC_SCRATCH_BYTES inside
+ * the library (held by every GPU that loads the library until the process
+ * exits) instead of an attached workspace; the caller passes only the input
+ * and output.  It calls no allocator.
+ *  - Shapes whose scratch exceeds the array (about m' x n' > 1024 x 2048
+ *    with m' <= n') are rejected with MO_ERR_UNSUPPORTED and a message.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it: make that first call before any
+ *    stream capture.
+ *  - All calls share the array and leave their contents behind; each call
+ *    clears what must start at zero.  Calls that overlap on the GPU (for
+ *    example on unordered streams) race on it.
+ *  - ctx supplies the device and receives error messages. */
+#define MO_STATIC_SCRATCH_BYTES (16u << 20)
+
+MO_API mo_status ns_orthogonalize_static(mo_ctx* ctx, const float* in, float* out, int64_t rows,
+                                         int64_t cols, const mo_ns_cfg* cfg, void* stream);
+
 /* ------------------------------------------------------------------ SOAP
  * One SOAP step per matrix with a per-step eigenbasis refresh ("Reading
  * notes on SOAP, Muon, and Beyond", sections 1 and 4; "LLM Optimizers",

@@ -78,6 +78,8 @@ SIGNATURES = {
                                  POINTER(c_int64), c_int, POINTER(NsCfg), c_void_p]),
     "soap_step": (c_int, [c_void_p, POINTER(SoapMat), c_int, POINTER(SoapCfg), c_int64, c_void_p]),
     "mo_gemm_bf16": (c_int, [c_void_p, POINTER(GemmDesc), c_void_p]),
+    "ns_orthogonalize_static": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64,
+                                        POINTER(NsCfg), c_void_p]),
     "mo_profile_enable": (c_int, [c_void_p, c_int]),
     "mo_profile_read": (c_int, [c_void_p, POINTER(ctypes.c_double), POINTER(ctypes.c_double),
                                 POINTER(c_int64), c_int]),

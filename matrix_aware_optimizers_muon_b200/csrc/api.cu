@@ -363,3 +363,9 @@ mo_status mo_gemm_bf16(mo_ctx* ctx, const mo_gemm_desc* d, void* stream) {
 }
 
 }  // extern "C"
+
+// Accessors for entry points defined in other translation units.
+namespace mo {
+int ctx_device(const mo_ctx* ctx) { return ctx->device; }
+mo_status ctx_fail(mo_ctx* ctx, mo_status st, const std::string& msg) { return fail(ctx, st, msg); }
+}  // namespace mo

@@ -202,7 +202,7 @@ def run_ours(args, world, rank, local):
 
     peaks, peak_kind = load_peaks()
     ctx = Context(local)
-    Ws, Gs, Bs, shapes = gpt_workload(dev)
+    Ws, Gs, Bs, shapes = gpt_workload(dev, layers=args.layers)
     ctx.reserve(OP_MUON, shapes)
     torch.cuda.synchronize()
     flops_page = sum(page_flops(m, n) for m, n in shapes)
@@ -263,7 +263,8 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded gradients: N(0,1e-3^2) + rank-16 spike at 10x norm; W ~ N(0,0.02^2))",
-        "config": {"workload": WORKLOAD, "matrices": len(shapes), "params": params,
+        "config": {"workload": WORKLOAD if args.layers == 32 else WORKLOAD.replace("32 layers", f"{args.layers} layers"),
+                   "matrices": len(shapes), "params": params,
                    "ns_steps": 5, "coeffs": [3.4445, -4.775, 2.0315],
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs (84 GB) far larger than L2; no flush"},
@@ -485,6 +486,8 @@ def main():
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--layers", type=int, default=32,
+                    help="dense-GPT layers (32 = the benchmark workload; fewer for small profiling cases)")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     if args.impl == "reference":

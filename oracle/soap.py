@@ -22,12 +22,13 @@ with the current basis is the same as the section 11.1 change-of-basis rule
 for the stored first moment.  V is never re-rotated.
 
 ``precision="bf16"`` reproduces the GPU path's declared rounding points:
-every tensor-core operand is rounded to bf16 (ties to even) and products are
-accumulated wide; the QR is exact (the GPU's is fp32-accurate).  With both
-sides present the two-sided products are taken left factor first:
+the factor EMAs and the rotations take bf16 operands (ties to even) with
+wide accumulation; the basis refresh (power step and QR) is fp32-accurate on
+the GPU and exact here.  With both sides present the two-sided products are
+taken left factor first:
 
     s1: Gb = bf16(G);  L = bs L + (1 - bs) Gb Gb^T   (L itself is not rounded)
-    s2: Y = bf16(L) bf16(Q_L);  Q_L = qr(Y)
+    s2: Y = L Q_L (not rounded);  Q_L = qr(Y)
     s4: T = bf16(bf16(Q_L)^T Mb);  M' = T bf16(Q_R)        (Mb = bf16(M))
         T = bf16(bf16(Q_L)^T Gb);  G' = T bf16(Q_R)
     s6: S = bf16(bf16(Q_L) bf16(Dbar));  D = S bf16(Q_R)^T
@@ -67,10 +68,10 @@ def soap_step(W, G, M, V, L=None, QL=None, R=None, QR=None, *, t=1,
     if refresh:
         if left:
             L = bs * L + (1.0 - bs) * (Gb @ Gb.T)
-            QL, _ = qr_positive(r(L) @ r(QL))
+            QL, _ = qr_positive(L @ QL)
         if right:
             R = bs * R + (1.0 - bs) * (Gb.T @ Gb)
-            QR, _ = qr_positive(r(R) @ r(QR))
+            QR, _ = qr_positive(R @ QR)
     # 3. first moment, original space
     M = beta1 * M + (1.0 - beta1) * G
     Mb = r(M)

@@ -40,7 +40,7 @@ def rnd(x):
     quantum = 2.0 ** (e - (_P - 1))     # spacing of bfloat16 values near x
     q = np.rint(xf / quantum) * quantum  # np.rint rounds half to even
     q = np.where(ax == 0, xf, q)        # keep signed zeros
-    q = np.where(np.abs(q) > _MAX, np.sign(q) * np.inf, q)
+    q = np.where(np.abs(q) > _MAX, np.copysign(np.inf, q), q)
     out[finite] = q
     return out
 

@@ -21,20 +21,22 @@ identity the step is AdamW.  Keeping M in the original space and rotating it
 with the current basis is the same as the section 11.1 change-of-basis rule
 for the stored first moment.  V is never re-rotated.
 
-``precision="bf16"`` reproduces the GPU path's declared rounding points:
-the factor EMAs and the rotations take bf16 operands (ties to even) with
-wide accumulation; the basis refresh (power step and QR) is fp32-accurate on
-the GPU and exact here.  With both sides present the two-sided products are
-taken left factor first:
+``precision="bf16"`` reproduces the GPU path's declared rounding points.
+The factor EMAs take bf16 operands; the basis refresh (power step and QR)
+is fp32-accurate on the GPU and exact here; the rotations take each operand
+as two bf16 planes, x ~ h + l with h = bf16(x), l = bf16(x - h), and form
+the product from the three plane products h h' + h l' + l h' with wide
+accumulation (stored intermediates are kept as h + l).  With both sides
+present the two-sided products are taken left factor first:
 
     s1: Gb = bf16(G);  L = bs L + (1 - bs) Gb Gb^T   (L itself is not rounded)
     s2: Y = L Q_L (not rounded);  Q_L = qr(Y)
-    s4: T = bf16(bf16(Q_L)^T Mb);  M' = T bf16(Q_R)        (Mb = bf16(M))
-        T = bf16(bf16(Q_L)^T Gb);  G' = T bf16(Q_R)
-    s6: S = bf16(bf16(Q_L) bf16(Dbar));  D = S bf16(Q_R)^T
-  one-sided: M' = bf16(Q_L)^T Mb,  D = bf16(Q_L) bf16(Dbar)  (left), or
-             M' = Mb bf16(Q_R),    D = bf16(Dbar) bf16(Q_R)^T (right);
-  no side:   M' = M, G' = G, D = Dbar (no rounding: plain AdamW).
+    s4: M' = p(s(p(Q_L^T, M)), Q_R);   G' = p(s(p(Q_L^T, G)), Q_R)
+    s6: D  = p(s(p(Q_L, Dbar)), Q_R^T)
+  where p(A, B) is the three-plane product and s(x) = h + l;
+  one-sided: M' = p(Q_L^T, M), D = p(Q_L, Dbar) (left) or
+             M' = p(M, Q_R),   D = p(Dbar, Q_R^T) (right);
+  no side:   M' = M, G' = G, D = Dbar (plain AdamW).
 """
 
 import numpy as np
@@ -55,7 +57,26 @@ def soap_step(W, G, M, V, L=None, QL=None, R=None, QR=None, *, t=1,
     """
     if precision not in ("fp64", "bf16"):
         raise ValueError(f"unknown precision {precision!r}")
-    r = rnd if precision == "bf16" else (lambda x: x)
+    emu = precision == "bf16"
+    r = rnd if emu else (lambda x: x)
+
+    def split2(x):
+        h = rnd(x)
+        return h, rnd(x - h)
+
+    def prod(A, B):
+        # the three-plane product of the emulated rotations (exact in fp64)
+        if not emu:
+            return A @ B
+        Ah, Al = split2(A)
+        Bh, Bl = split2(B)
+        return Ah @ Bh + Ah @ Bl + Al @ Bh
+
+    def keep(x):
+        if not emu:
+            return x
+        h, l = split2(x)
+        return h + l
     f64 = lambda x: None if x is None else np.asarray(x, dtype=np.float64)
     W, G, M, V = f64(W), f64(G), f64(M), f64(V)
     L, QL, R, QR = f64(L), f64(QL), f64(R), f64(QR)
@@ -74,22 +95,19 @@ def soap_step(W, G, M, V, L=None, QL=None, R=None, QR=None, *, t=1,
             QR, _ = qr_positive(R @ QR)
     # 3. first moment, original space
     M = beta1 * M + (1.0 - beta1) * G
-    Mb = r(M)
-    QLb = r(QL) if left else None
-    QRb = r(QR) if right else None
 
     # 4. rotate into the basis
-    def rotate_in(X, Xb):
+    def rotate_in(X):
         if left and right:
-            return r(QLb.T @ Xb) @ QRb
+            return prod(keep(prod(QL.T, X)), QR)
         if left:
-            return QLb.T @ Xb
+            return prod(QL.T, X)
         if right:
-            return Xb @ QRb
+            return prod(X, QR)
         return X
 
-    Mr = rotate_in(M, Mb)
-    Gr = rotate_in(G, Gb)
+    Mr = rotate_in(M)
+    Gr = rotate_in(G)
     # 5. Adam in the basis
     V = beta2 * V + (1.0 - beta2) * Gr * Gr
     bc1 = 1.0 - beta1 ** t if bias_correction else 1.0
@@ -97,11 +115,11 @@ def soap_step(W, G, M, V, L=None, QL=None, R=None, QR=None, *, t=1,
     Dbar = (Mr / bc1) / (np.sqrt(V / bc2) + eps)
     # 6. rotate back
     if left and right:
-        D = r(QLb @ r(Dbar)) @ QRb.T
+        D = prod(keep(prod(QL, Dbar)), QR.T)
     elif left:
-        D = QLb @ r(Dbar)
+        D = prod(QL, Dbar)
     elif right:
-        D = r(Dbar) @ QRb.T
+        D = prod(Dbar, QR.T)
     else:
         D = Dbar
     # 7. decoupled weight decay and apply

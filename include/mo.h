@@ -213,6 +213,11 @@ typedef struct {
 MO_API mo_status soap_step(mo_ctx* ctx, const mo_soap_mat* mats /* host array */, int n,
                     const mo_soap_cfg* cfg, int64_t step, void* stream);
 
+/* Exact workspace of soap_step for these matrices, sides as given (the
+ * shape-only query mo_workspace_bytes(op = 1) assumes both sides are kept).
+ * Only rows, cols, L and R are read; no pointer is dereferenced. */
+MO_API mo_status mo_soap_workspace_bytes(mo_ctx* ctx, const mo_soap_mat* mats, int n, size_t* bytes);
+
 /* ------------------------------------------------------------------ building block
  * The batched tensor-core GEMM the steps are built from, exposed for tests
  * and for callers composing their own variants:

@@ -178,7 +178,10 @@ class Context:
                              _ptr(d["V"]), _ptr(d.get("L")), _ptr(d.get("QL")), _ptr(d.get("R")),
                              _ptr(d.get("QR")))
         if reserve:
-            self.reserve(OP_SOAP, [tuple(d["W"].shape) for d in mats], stream=stream)
+            need = c_size_t()
+            self._check(self.lib.mo_soap_workspace_bytes(self.handle, arr, n, byref(need)))
+            if self.workspace is None or self.workspace.numel() < need.value:
+                self.attach_workspace(need.value, stream)
         sb = beta2 if shampoo_beta is None else shampoo_beta
         cfg = SoapCfg(lr, beta1, beta2, sb, eps, weight_decay, int(bias_correction), _ptr(nonfinite))
         self._check(self.lib.soap_step(self.handle, arr, n, byref(cfg), int(step), self._stream(stream)))

@@ -78,6 +78,7 @@ SIGNATURES = {
                                  POINTER(c_int64), c_int, POINTER(NsCfg), c_void_p]),
     "soap_step": (c_int, [c_void_p, POINTER(SoapMat), c_int, POINTER(SoapCfg), c_int64, c_void_p]),
     "mo_gemm_bf16": (c_int, [c_void_p, POINTER(GemmDesc), c_void_p]),
+    "mo_soap_workspace_bytes": (c_int, [c_void_p, POINTER(SoapMat), c_int, POINTER(c_size_t)]),
     "ns_orthogonalize_static": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64,
                                         POINTER(NsCfg), c_void_p]),
     "mo_profile_enable": (c_int, [c_void_p, c_int]),

@@ -322,6 +322,21 @@ mo_status soap_step(mo_ctx* ctx, const mo_soap_mat* mats, int n, const mo_soap_c
   return MO_OK;
 }
 
+mo_status mo_soap_workspace_bytes(mo_ctx* ctx, const mo_soap_mat* mats, int n, size_t* bytes) {
+  if (ctx == nullptr || bytes == nullptr) return MO_ERR_INVALID_ARG;
+  if (n < 0 || (n > 0 && mats == nullptr)) return fail(ctx, MO_ERR_INVALID_ARG, "mo_soap_workspace_bytes: bad arguments");
+  std::vector<mo::SoapItem> items;
+  for (int i = 0; i < n; ++i) {
+    if (mats[i].rows <= 0 || mats[i].cols <= 0 || mats[i].rows > (1 << 16) || mats[i].cols > (1 << 20))
+      return fail(ctx, MO_ERR_INVALID_ARG, "mo_soap_workspace_bytes: bad shape at index " + std::to_string(i));
+    mo::SoapItem it;
+    it.m = mats[i];
+    items.push_back(it);
+  }
+  *bytes = mo::soap_workspace_exact(items);
+  return MO_OK;
+}
+
 // ---------------------------------------------------------------- GEMM block
 
 mo_status mo_gemm_bf16(mo_ctx* ctx, const mo_gemm_desc* d, void* stream) {

@@ -23,30 +23,43 @@ void load_encode_fn() {
   }
 }
 
-// 3-D bf16 tensor map over `batch` matrices of storage rows x cols (row
-// stride ld, matrix stride bstride, both in elements); box = 64 x box_rows.
-bool encode_bf16_3d(CUtensorMap* map, const void* ptr, long long rows, long long cols, long long ld,
-                    long long bstride, int batch, int box_rows) {
+// 4-D bf16 tensor map over `planes` x `batch` matrices of storage rows x cols
+// (row stride ld, matrix stride bstride, plane stride pstride, all in
+// elements); box = 64 x box_rows.
+bool encode_bf16_4d(CUtensorMap* map, const void* ptr, long long rows, long long cols, long long ld,
+                    long long bstride, int batch, long long pstride, int planes, int box_rows) {
   std::call_once(g_encode_once, load_encode_fn);
   if (g_encode == nullptr) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
-  cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)((batch > 1 ? bstride : rows * ld) * 2)};
-  cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+  const long long bs = batch > 1 ? bstride : rows * ld;
+  const long long ps = planes > 1 ? pstride : bs * batch;
+  cuuint64_t dims[4] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch, (cuuint64_t)planes};
+  cuuint64_t strides[3] = {(cuuint64_t)(ld * 2), (cuuint64_t)(bs * 2), (cuuint64_t)(ps * 2)};
+  cuuint32_t box[4] = {64u, (cuuint32_t)box_rows, 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+int planes_of(const unsigned char* pat, int nseg) {
+  int m = 0;
+  for (int i = 0; i < nseg; ++i) m = pat[i] > m ? pat[i] : m;
+  return m + 1;
 }
 
 template <int BN, int A_MN, int B_MN>
 cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   using Cfg = GemmCfg<BN>;
   CUtensorMap ta, tb;
-  const bool ok_a = A_MN ? encode_bf16_3d(&ta, op.A, op.K, op.M, op.lda, op.strideA, op.batch, 64)
-                         : encode_bf16_3d(&ta, op.A, op.M, op.K, op.lda, op.strideA, op.batch, GEMM_BM);
-  const bool ok_b = B_MN ? encode_bf16_3d(&tb, op.B, op.K, op.N, op.ldb, op.strideB, op.batch, 64)
-                         : encode_bf16_3d(&tb, op.B, op.N, op.K, op.ldb, op.strideB, op.batch, BN);
+  const int nseg = op.nseg > 1 ? op.nseg : 1;
+  if (nseg > 8 || (nseg > 1 && op.K % (nseg * GEMM_BK) != 0)) return cudaErrorInvalidValue;
+  const long long kseg = op.K / nseg;
+  const int pa = planes_of(op.pat_a, nseg), pb = planes_of(op.pat_b, nseg);
+  const bool ok_a = A_MN ? encode_bf16_4d(&ta, op.A, kseg, op.M, op.lda, op.strideA, op.batch, op.planeA, pa, 64)
+                         : encode_bf16_4d(&ta, op.A, op.M, kseg, op.lda, op.strideA, op.batch, op.planeA, pa, GEMM_BM);
+  const bool ok_b = B_MN ? encode_bf16_4d(&tb, op.B, kseg, op.N, op.ldb, op.strideB, op.batch, op.planeB, pb, 64)
+                         : encode_bf16_4d(&tb, op.B, op.N, kseg, op.ldb, op.strideB, op.batch, op.planeB, pb, BN);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
 
   GemmParams p;
@@ -59,6 +72,15 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   p.C = op.C; p.ldc = op.ldc; p.strideC = op.strideC; p.c_f32 = op.c_f32;
   p.D = op.D; p.ldd = op.ldd; p.strideD = op.strideD; p.d_f32 = op.d_f32;
   p.status = status;
+  p.c_tab = op.c_tab; p.d_tab = op.d_tab; p.e_tab = op.e_tab;
+  p.epi = op.epi;
+  p.adam_b2 = op.adam_b2; p.adam_ibc1 = op.adam_ibc1; p.adam_ibc2 = op.adam_ibc2; p.adam_eps = op.adam_eps;
+  p.lde = op.lde; p.strideE = 0;
+  p.nseg = nseg;
+  p.kseg = (int)kseg;
+  for (int i = 0; i < 8; ++i) { p.pat_a[i] = op.pat_a[i]; p.pat_b[i] = op.pat_b[i]; }
+  p.d_split = op.d_split;
+  p.d_plane = op.d_plane;
 
   auto kern = gemm_bf16_kernel<BN, A_MN, B_MN>;
   static int attr_done[64] = {0};
@@ -69,14 +91,19 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
-  const long long total = (long long)p.tiles_m * p.tiles_n * p.batch;
+  // tiles enumerated per matrix: all, or those touching the upper triangle
+  long long tiles = 0;
+  for (int tn = 0; tn < p.tiles_n; ++tn) {
+    if (!p.sym) { tiles += p.tiles_m; continue; }
+    const int r = (tn * BN + BN - 1) / GEMM_BM + 1;
+    tiles += r < p.tiles_m ? r : p.tiles_m;
+  }
+  p.tiles_per_mat = (int)tiles;
+  const long long total = tiles * p.batch;
+  if (total >= (1ll << 31)) return cudaErrorInvalidValue;
   const int grid = (int)(total < device_sm_count() ? total : device_sm_count());
   if (grid <= 0) return cudaSuccess;
   // executed tensor-core flops: computed tiles x 128 x BN x padded K x 2
-  long long tiles = 0;
-  for (int tn = 0; tn < p.tiles_n; ++tn)
-    for (int tm = 0; tm < p.tiles_m; ++tm)
-      if (!(p.sym && tm * GEMM_BM > tn * BN + BN - 1)) ++tiles;
   const double flops = 2.0 * tiles * p.batch * GEMM_BM * BN * (double)round_up(p.K, GEMM_BK);
   ProfScope prof(op.kind, stream, flops);
   kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);

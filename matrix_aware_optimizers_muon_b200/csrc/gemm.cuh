@@ -25,7 +25,8 @@ namespace mo {
 struct GemmParams {
   int M, N, K;              // per-matrix problem size
   int batch;                // number of independent matrices
-  int tiles_m, tiles_n;     // tiles per matrix
+  int tiles_m, tiles_n;     // tile grid of one matrix
+  int tiles_per_mat;        // tiles enumerated per matrix (fewer when sym)
   int sym;                  // symmetric product: upper tiles + mirror stores
   float alpha, beta;        // epilogue coefficients
   const float* scale;       // optional per-matrix scale s_b (device)
@@ -37,7 +38,26 @@ struct GemmParams {
   long long ldd, strideD;   // elements
   int d_f32;                // D is fp32 (else bf16)
   int* status;              // device status word (timeouts)
+  // optional per-matrix pointer tables (device arrays of `batch` entries);
+  // when set they replace base + b * stride for C, D and E
+  const void* const* c_tab;
+  void* const* d_tab;
+  float* const* e_tab;
+  int epi;                  // EPI_AXPBY or EPI_ADAM
+  // Adam-in-basis epilogue (acc = G'): V = b2 V + (1 - b2) acc^2 (E, fp32,
+  // in place); D = bf16((C * ibc1) / (sqrt(V * ibc2) + eps)) with C = M'
+  float adam_b2, adam_ibc1, adam_ibc2, adam_eps;
+  long long lde, strideE;
+  // plane-stacked K: K = nseg * kseg; segment s multiplies plane pat_a[s] of
+  // A by plane pat_b[s] of B (split-precision products); nseg == 1: plain
+  int nseg, kseg;
+  unsigned char pat_a[8], pat_b[8];
+  // bf16 output as two planes: D = bf16(x), D + d_plane = bf16(x - bf16(x))
+  int d_split;
+  long long d_plane;
 };
+
+enum { EPI_AXPBY = 0, EPI_ADAM = 1 };
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;
@@ -54,15 +74,42 @@ struct GemmCfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
 };
 
+// Tiles of one matrix in column order (M fastest, so the CTAs in flight
+// share B columns in L2).  For a symmetric product only the tiles touching
+// the upper triangle are enumerated: column tn holds rows tm with
+// tm * BM <= tn * BN + BN - 1, so the persistent CTAs get equal shares of
+// computed tiles.
+__device__ __forceinline__ int sym_rows_in_col(const GemmParams& p, int BN, int tn) {
+  const int r = (tn * BN + BN - 1) / GEMM_BM + 1;
+  return r < p.tiles_m ? r : p.tiles_m;
+}
+
 __device__ __forceinline__ bool gemm_decode(const GemmParams& p, int BN, int t, int& b, int& tm,
                                             int& tn) {
-  const int per = p.tiles_m * p.tiles_n;
-  b = t / per;
-  const int u = t - b * per;
-  tn = u / p.tiles_m;          // M fastest: concurrently running CTAs share B columns
-  tm = u - tn * p.tiles_m;
-  if (p.sym && tm * GEMM_BM > tn * BN + BN - 1) return false;   // entirely below diagonal
+  b = t / p.tiles_per_mat;
+  int u = t - b * p.tiles_per_mat;
+  if (!p.sym) {
+    tn = u / p.tiles_m;
+    tm = u - tn * p.tiles_m;
+    return true;
+  }
+  for (tn = 0; tn < p.tiles_n; ++tn) {
+    const int c = sym_rows_in_col(p, BN, tn);
+    if (u < c) break;
+    u -= c;
+  }
+  tm = u;
   return true;
+}
+
+__device__ __forceinline__ const void* c_base(const GemmParams& p, int b) {
+  if (p.c_tab) return p.c_tab[b];
+  return reinterpret_cast<const char*>(p.C) + (size_t)b * p.strideC * (p.c_f32 ? 4 : 2);
+}
+
+__device__ __forceinline__ void* d_base(const GemmParams& p, int b) {
+  if (p.d_tab) return p.d_tab[b];
+  return reinterpret_cast<char*>(p.D) + (size_t)b * p.strideD * (p.d_f32 ? 4 : 2);
 }
 
 __device__ __forceinline__ float ipow_scale(const float* s, int b, int pw) {
@@ -75,7 +122,7 @@ __device__ __forceinline__ float ipow_scale(const float* s, int b, int pw) {
 __device__ __forceinline__ void load_c32(const GemmParams& p, int b, int r, int c0, float (&c)[32]) {
   const bool full = c0 + 32 <= p.N;
   if (p.c_f32) {
-    const float* src = reinterpret_cast<const float*>(p.C) + b * p.strideC + (long long)r * p.ldc + c0;
+    const float* src = reinterpret_cast<const float*>(c_base(p, b)) + (long long)r * p.ldc + c0;
     if (full) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -88,7 +135,7 @@ __device__ __forceinline__ void load_c32(const GemmParams& p, int b, int r, int 
     }
   } else {
     const __nv_bfloat16* src =
-        reinterpret_cast<const __nv_bfloat16*>(p.C) + b * p.strideC + (long long)r * p.ldc + c0;
+        reinterpret_cast<const __nv_bfloat16*>(c_base(p, b)) + (long long)r * p.ldc + c0;
     if (full) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -110,31 +157,38 @@ __device__ __forceinline__ void load_c32(const GemmParams& p, int b, int r, int 
 
 __device__ __forceinline__ void store_one(const GemmParams& p, int b, int r, int c, float v) {
   if (p.d_f32) {
-    reinterpret_cast<float*>(p.D)[b * p.strideD + (long long)r * p.ldd + c] = v;
+    reinterpret_cast<float*>(d_base(p, b))[(long long)r * p.ldd + c] = v;
   } else {
-    reinterpret_cast<__nv_bfloat16*>(p.D)[b * p.strideD + (long long)r * p.ldd + c] =
-        __float2bfloat16_rn(v);
+    __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(d_base(p, b)) + (long long)r * p.ldd + c;
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    *d = h;
+    if (p.d_split) d[p.d_plane] = __float2bfloat16_rn(v - __bfloat162float(h));
   }
 }
 
 __device__ __forceinline__ void store_row32(const GemmParams& p, int b, int r, int c0,
                                             const float (&x)[32]) {
   if (p.d_f32) {
-    float* dst = reinterpret_cast<float*>(p.D) + b * p.strideD + (long long)r * p.ldd + c0;
+    float* dst = reinterpret_cast<float*>(d_base(p, b)) + (long long)r * p.ldd + c0;
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       reinterpret_cast<float4*>(dst)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
   } else {
-    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + b * p.strideD + (long long)r * p.ldd + c0;
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(d_base(p, b)) + (long long)r * p.ldd + c0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      uint32_t w[4];
+      uint32_t w[4], wl[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(x[8 * i + 2 * j], x[8 * i + 2 * j + 1]);
+        const float x0 = x[8 * i + 2 * j], x1 = x[8 * i + 2 * j + 1];
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
         w[j] = *reinterpret_cast<const uint32_t*>(&h);
+        const float2 hf = __bfloat1622float2(h);
+        const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+        wl[j] = *reinterpret_cast<const uint32_t*>(&l);
       }
       reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+      if (p.d_split) reinterpret_cast<uint4*>(dst + p.d_plane)[i] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
     }
   }
 }
@@ -186,7 +240,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int total = p.tiles_m * p.tiles_n * p.batch;
+  const int total = p.tiles_per_mat * p.batch;
   const int nk = (p.K + GEMM_BK - 1) / GEMM_BK;
 
   if (warp == 0) {
@@ -206,18 +260,25 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
           uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
           uint8_t* sb = sa + Cfg::A_BYTES;
+          int kl = kb * GEMM_BK, pa = 0, pb = 0;
+          if (p.nseg > 1) {
+            const int seg = kl / p.kseg;
+            kl -= seg * p.kseg;
+            pa = p.pat_a[seg];
+            pb = p.pat_b[seg];
+          }
           if (!A_MN) {
-            tma_load_3d(sa, &tmA, &full[stage], kb * GEMM_BK, tm * GEMM_BM, b);
+            tma_load_4d(sa, &tmA, &full[stage], kl, tm * GEMM_BM, b, pa);
           } else {
-            tma_load_3d(sa, &tmA, &full[stage], tm * GEMM_BM, kb * GEMM_BK, b);
-            tma_load_3d(sa + GEMM_BK * 128, &tmA, &full[stage], tm * GEMM_BM + 64, kb * GEMM_BK, b);
+            tma_load_4d(sa, &tmA, &full[stage], tm * GEMM_BM, kl, b, pa);
+            tma_load_4d(sa + GEMM_BK * 128, &tmA, &full[stage], tm * GEMM_BM + 64, kl, b, pa);
           }
           if (!B_MN) {
-            tma_load_3d(sb, &tmB, &full[stage], kb * GEMM_BK, tn * BN, b);
+            tma_load_4d(sb, &tmB, &full[stage], kl, tn * BN, b, pb);
           } else {
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j)
-              tma_load_3d(sb + j * GEMM_BK * 128, &tmB, &full[stage], tn * BN + 64 * j, kb * GEMM_BK, b);
+              tma_load_4d(sb + j * GEMM_BK * 128, &tmB, &full[stage], tn * BN + 64 * j, kl, b, pb);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -306,7 +367,22 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           float x[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) x[i] = alpha * __uint_as_float(v[i]);
-          if (p.C != nullptr) {
+          if (p.epi == EPI_ADAM) {
+            // V <- b2 V + (1 - b2) G'^2 ;  Dbar = (M' / bc1) / (sqrt(V / bc2) + eps)
+            float mr[32];
+            load_c32(p, b, r, c0, mr);
+            float* vp = (p.e_tab ? p.e_tab[b] : nullptr) + (long long)r * p.lde + c0;
+            const bool full = c0 + 32 <= p.N;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (full || c0 + i < p.N) {
+                const float g = x[i];
+                const float vn = fmaf(p.adam_b2, vp[i], (1.0f - p.adam_b2) * g * g);
+                vp[i] = vn;
+                x[i] = (mr[i] * p.adam_ibc1) / (sqrtf(vn * p.adam_ibc2) + p.adam_eps);
+              }
+            }
+          } else if (p.C != nullptr || p.c_tab != nullptr) {
             float c[32];
             load_c32(p, b, r, c0, c);
 #pragma unroll

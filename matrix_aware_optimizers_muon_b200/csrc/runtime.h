@@ -32,6 +32,24 @@ struct GemmOp {
   long long ldd = 0, strideD = 0;
   int d_f32 = 0;
   int kind = 9;          // profiling tag (ProfKind)
+  // per-matrix pointer tables in device memory (optional)
+  const void* const* c_tab = nullptr;
+  void* const* d_tab = nullptr;
+  float* const* e_tab = nullptr;
+  long long lde = 0;
+  // epilogue mode: 0 = alpha acc + beta C, 1 = Adam in the rotated basis
+  int epi = 0;
+  float adam_b2 = 0.f, adam_ibc1 = 1.f, adam_ibc2 = 1.f, adam_eps = 0.f;
+  // plane-stacked K (split-precision products): K = nseg * kseg, segment s
+  // uses plane pat_a[s] of A and pat_b[s] of B; planes are planeA/planeB
+  // elements apart.  kseg must be a multiple of 64 when nseg > 1.
+  int nseg = 1;
+  unsigned char pat_a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  unsigned char pat_b[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  long long planeA = 0, planeB = 0;
+  // bf16 D written as two planes (h, l) d_plane elements apart
+  int d_split = 0;
+  long long d_plane = 0;
 };
 
 // Launch the tcgen05 GEMM.  Returns cudaSuccess or the launch/encode error.

@@ -1,0 +1,104 @@
+// Kernels of the SOAP path other than the tensor-core GEMM.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace mo {
+
+constexpr int SOAP_MAXB = 256;   // matrices per launch (pointer tables in kernel params)
+constexpr int QR_B = 128;        // Cholesky diagonal block
+
+// Copy a table of device pointers into device memory (stream ordered).
+void launch_upload_ptrs(void** dst, const void* const* src, int n, cudaStream_t s);
+
+struct SoapPrepArgs {
+  int count;
+  long long rows, cols;            // matrix shape (cols % 4 == 0)
+  float beta1;
+  const float* G[SOAP_MAXB];
+  float* M[SOAP_MAXB];
+  __nv_bfloat16* Gp;               // two planes of G: [2][count][*][ldp]
+  __nv_bfloat16* Mp;               // two planes of M
+  long long ldp, mat_stride, plane_stride;
+};
+// M <- b1 M + (1 - b1) G ; two bf16 planes (h, l) of G and of the new M
+void launch_soap_prep(const SoapPrepArgs& a, cudaStream_t s);
+
+// Split fp32 matrices into bf16 planes x = h + m + l (nearly exact): plane p
+// of matrix b is written to dst + p * plane_stride + b * mat_stride, with row
+// stride ldd; rows >= rows_valid or cols >= cols_valid are written as zero
+// (or as the identity when `pad_identity`), up to rows_pad x cols_pad.
+// Optional: per-column scale (inv_d[b * cols_pad + c]) applied first, and the
+// scaled fp32 value written back to the source.
+struct SplitArgs {
+  int count, rows_valid, cols_valid, rows_pad, cols_pad;
+  const float* src[SOAP_MAXB];     // fp32, row stride lds
+  long long lds;
+  const float* col_scale;          // optional [count][cols_pad]
+  float* write_back;               // optional: scaled fp32, [count][rows_pad][ldw]
+  long long ldw, wb_stride;
+  __nv_bfloat16* dst;
+  long long ldd, mat_stride, plane_stride;
+  int nplanes;                     // 1 (bf16 cast), 2 (h, l) or 3 (h, m, l)
+  int pad_identity;
+};
+void launch_split(const SplitArgs& a, cudaStream_t s);
+
+// inv_d[b][c] = 1 / ||Y[b][:, c]||_2 over rows < rows (fixed summation order)
+void launch_colnorm(const float* Y, long long ld, long long mat_stride, int count, int rows, int cols,
+                    float* inv_d, cudaStream_t s);
+
+// C[b][i][i] += shift for i < n
+void launch_shift_diag(float* C, long long ld, long long mat_stride, int count, int n, float shift,
+                       cudaStream_t s);
+
+struct FlagTable {
+  int32_t* f[SOAP_MAXB];           // per-matrix flag slots (entries may be null)
+};
+
+// Cholesky of the 128 x 128 diagonal block at (k0, k0) of each C[b] (lower
+// factor, fp32, in shared memory) and its inverse -> Dinv[b] (128 x 128,
+// lower).  A non-positive pivot sets *flag[b] = 1 (if given) and the block
+// inverse to NaN.
+void launch_chol_diag(const float* C, long long ld, long long mat_stride, int count, int k0,
+                      float* Dinv, const FlagTable& flags, cudaStream_t s);
+
+// out = in * Dinv^T for 128-wide row blocks: in/out are rows x 128 fp32
+// views (row stride ld); out may alias in.  Optionally writes the three bf16
+// planes of out to planes (+ p * plane_stride + b * mat_stride, row stride
+// 128) and skips the fp32 store.
+struct RowBlockArgs {
+  int count, rows;
+  const float* in; long long ld_in, in_stride;
+  float* out; long long ld_out, out_stride;         // may be null
+  const float* Dinv;                                 // [count][128][128]
+  __nv_bfloat16* planes; long long plane_stride, mat_stride;
+};
+void launch_rowblock_dinv(const RowBlockArgs& a, cudaStream_t s);
+
+// Final basis: Qout[b] (caller fp32 k x k) = Y[b][:k, :k]
+struct CopyOutArgs {
+  int count, k;
+  const float* Y; long long ld, mat_stride;
+  float* dst[SOAP_MAXB];
+};
+void launch_copy_out(const CopyOutArgs& a, cudaStream_t s);
+
+// Adam step with identity bases (both sides) fused with the apply:
+// V <- b2 V + (1-b2) G^2 ; W <- decay W - lr (M / bc1) / (sqrt(V / bc2) + eps)
+struct AdamIdArgs {
+  int count;
+  long long elems;
+  float beta2, ibc1, ibc2, eps, decay, lr;
+  const float* G[SOAP_MAXB];
+  const float* M[SOAP_MAXB];
+  float* V[SOAP_MAXB];
+  float* W[SOAP_MAXB];
+};
+void launch_adam_identity(const AdamIdArgs& a, cudaStream_t s);
+
+// Per-matrix flag reset (the QR pivots report into them)
+void launch_set_flags(const FlagTable& flags, int count, int32_t value, cudaStream_t s);
+
+}  // namespace mo

@@ -19,6 +19,9 @@ struct SoapItem {
 
 void soap_workspace(const int64_t* rows, const int64_t* cols, int n, size_t* min_bytes, size_t* full_bytes);
 
+// Exact workspace for these matrices (sides as given).
+size_t soap_workspace_exact(const std::vector<SoapItem>& items);
+
 // Enqueue one SOAP step for every item.  Planning errors set *err.
 cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg, int64_t step, char* ws,
                      size_t ws_bytes, cudaStream_t stream, std::string* err);

@@ -1,0 +1,142 @@
+"""SOAP parity: the CUDA path through the C ABI against the fp64 oracle and
+its bf16-emulation mode, from the same seeded warm state."""
+import numpy as np
+import pytest
+
+import workloads as wl
+from gates import rel
+from gpu_env import context
+from oracle import soap as osoap
+
+pytestmark = pytest.mark.gpu
+
+HP = dict(lr=3e-3, beta1=0.95, beta2=0.95, eps=1e-8, weight_decay=0.0)
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    return context()
+
+
+def _cuda(a):
+    import torch
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def _np(t):
+    return None if t is None else t.detach().cpu().numpy().astype(np.float64)
+
+
+def warm_state(m, n, left, right, steps, tag, cfg=wl.CFG4_MINI):
+    """Oracle (fp64) steps from zero state; returns the float32 state and the
+    gradient of the next step."""
+    st = wl.SpikeStream(tag, "warm", m * 1000 + n, m, n, cfg)
+    S = dict(W=st.W.astype(np.float64), M=np.zeros((m, n)), V=np.zeros((m, n)),
+             L=np.zeros((m, m)) if left else None, QL=np.eye(m) if left else None,
+             R=np.zeros((n, n)) if right else None, QR=np.eye(n) if right else None)
+    for t in range(1, steps + 1):
+        G = st.next()
+        out = osoap.soap_step(S["W"], G, S["M"], S["V"], S["L"], S["QL"], S["R"], S["QR"], t=t, **HP)
+        S = {k: out[k] for k in S}
+    f32 = {k: (None if v is None else v.astype(np.float32)) for k, v in S.items()}
+    return f32, st.next(), steps + 1
+
+
+def run_gpu(ctx, S, G, t, flags=None):
+    import torch
+    d = {k: _cuda(v) for k, v in S.items()}
+    d["G"] = _cuda(G)
+    ctx.soap_step([d], t, nonfinite=flags, **HP)
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    return {k: _np(v) for k, v in d.items() if k != "G"}
+
+
+def check_step(ctx, m, n, left, right, steps=10, tag="soap"):
+    S, G, t = warm_state(m, n, left, right, steps, tag)
+    out = run_gpu(ctx, S, G, t)
+    args = (S["W"], G, S["M"], S["V"], S["L"], S["QL"], S["R"], S["QR"])
+    ref = osoap.soap_step(*args, t=t, **HP)
+    emu = osoap.soap_step(*args, t=t, precision="bf16", **HP)
+    res = {}
+    res["M"] = rel(out["M"], ref["M"])
+    assert res["M"] <= 1e-6, res                                   # fp32 path
+    for side, fac, q in (("L", "L", "QL"), ("R", "R", "QR")):
+        if S[fac] is None:
+            continue
+        res[fac] = rel(out[fac], emu[fac])
+        assert res[fac] <= 1e-4, res                               # bf16-operand EMA, fp32 state
+        Q = out[q]
+        res[q + "_orth"] = float(np.abs(Q.T @ Q - np.eye(Q.shape[0])).max())
+        assert res[q + "_orth"] <= 1e-4, res
+        res[q] = rel(Q, emu[q])
+        assert res[q] <= 5e-3, res                                 # fp32-accurate refresh
+    res["V"] = rel(out["V"], emu["V"])
+    assert res["V"] <= 1e-2, res
+    decayed = (1 - HP["lr"] * HP["weight_decay"]) * S["W"].astype(np.float64)
+    dW = out["W"] - decayed
+    res["dW_emu"] = rel(dW, emu["dW"])
+    res["dW_fp64"] = rel(dW, ref["dW"])
+    assert res["dW_emu"] <= 1e-2, res
+    assert res["dW_fp64"] <= 2e-2, res                              # bf16-operand path
+    return res
+
+
+@pytest.mark.parametrize("m,n,left,right", [
+    (256, 256, True, True),      # two-sided, square
+    (128, 384, True, True),      # two-sided, wide
+    (256, 896, True, False),     # right side identity (large axis)
+    (160, 96, False, True),      # left side identity
+])
+def test_warm_step_parity(ctx, m, n, left, right):
+    check_step(ctx, m, n, left, right)
+
+
+def test_identity_bases_is_adamw(ctx):
+    rng = wl.rng_of("soap-adamw")
+    m, n = 64, 128
+    S = dict(W=wl.weights(rng, m, n), M=wl.gaussian(rng, (m, n), 1e-3),
+             V=np.abs(wl.gaussian(rng, (m, n), 1e-6)), L=None, QL=None, R=None, QR=None)
+    G = wl.gaussian(rng, (m, n), 1e-3)
+    out = run_gpu(ctx, S, G, 4)
+    ref = osoap.soap_step(S["W"], G, S["M"], S["V"], t=4, **HP)
+    assert rel(out["W"] - S["W"], ref["dW"]) <= 1e-5
+    assert rel(out["V"], ref["V"]) <= 1e-6
+
+
+def test_cold_start_properties(ctx):
+    """Step 1 from zero state: L_1 is ill-conditioned (kappa ~ 1e4), so the
+    basis is compared by its defining properties: orthonormal, and Q^T Y
+    upper triangular with a positive diagonal (Y = L_1 Q_0 = L_1)."""
+    import torch
+    m, n = 256, 896
+    st = wl.SpikeStream("soap-cold", "x", 0, m, n, wl.CFG4_MINI)
+    G = st.next()
+    S = dict(W=st.W, M=np.zeros((m, n), np.float32), V=np.zeros((m, n), np.float32),
+             L=np.zeros((m, m), np.float32), QL=np.eye(m, dtype=np.float32), R=None, QR=None)
+    flags = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    out = run_gpu(ctx, S, G, 1, flags)
+    assert int(flags.item()) == 0
+    Q, L1 = out["QL"], out["L"]
+    assert np.abs(Q.T @ Q - np.eye(m)).max() <= 1e-4
+    R = Q.T @ L1
+    assert np.abs(np.tril(R, -1)).max() <= 1e-4 * np.abs(R).max()
+    assert (np.diag(R) > 0).all()
+    # first Adam step is a sign-like step: |Dbar| ~ 1 entrywise
+    dW = out["W"] - S["W"]
+    ratio = np.linalg.norm(dW) / (HP["lr"] * np.sqrt(m * n))
+    assert 0.9 <= ratio <= 1.0 + 1e-3
+
+
+def test_skip_leaves_state(ctx):
+    m, n = 64, 64
+    rng = wl.rng_of("soap-skip")
+    S = dict(W=wl.weights(rng, m, n), M=np.zeros((m, n), np.float32), V=np.zeros((m, n), np.float32),
+             L=np.zeros((m, m), np.float32), QL=np.eye(m, dtype=np.float32), R=None, QR=None)
+    import torch
+    d = {k: _cuda(v) for k, v in S.items()}
+    d["G"] = None
+    ctx.soap_step([d], 1, **HP)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(_np(d["W"]), S["W"])
+    np.testing.assert_array_equal(_np(d["QL"]), S["QL"])

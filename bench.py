@@ -376,6 +376,93 @@ def heads_gpu(count, dim, dev, cond=1e4):
     return [G[i].contiguous() for i in range(count)]
 
 
+def soap_flops(m, n, left, right):
+    """The SOAP step's count per matrix: factor EMAs 2m^2n / 2n^2m, power
+    steps 2k^3, QR counted as Householder (8/3)k^3 whatever algorithm runs,
+    and the rotations: rotating M and G in and the update back out."""
+    f = 0.0
+    rot = 0.0
+    if left:
+        f += 2.0 * m * m * n + 2.0 * m ** 3 + (8.0 / 3.0) * m ** 3
+        rot += 2.0 * m * m * n
+    if right:
+        f += 2.0 * n * n * m + 2.0 * n ** 3 + (8.0 / 3.0) * n ** 3
+        rot += 2.0 * m * n * n
+    return f + 3.0 * rot, 3.0 * rot
+
+
+def soap_workload(dev, sq=4096, wide=14336, n_sq=4, n_wide=4, rank=32, noise=1e-3, ratio=10.0):
+    """SOAP matrices: n_sq two-sided sq x sq, n_wide sq x wide with the wide
+    side on the identity basis.  Gradients: fixed rank-32 spike at 10x the
+    noise norm plus fresh Gaussian noise every step."""
+    import torch
+    import workloads as wl
+    mats, spikes = [], []
+    for kind, count, n in (("sq", n_sq, sq), ("wide", n_wide, wide)):
+        for i in range(count):
+            g = torch.Generator(device=dev)
+            g.manual_seed(wl.seed_of("bench-cfg4", kind, i))
+            m = sq
+            d = dict(W=torch.randn(m, n, generator=g, device=dev) * 0.02,
+                     G=torch.empty(m, n, device=dev),
+                     M=torch.zeros(m, n, device=dev), V=torch.zeros(m, n, device=dev),
+                     L=torch.zeros(m, m, device=dev), QL=torch.eye(m, device=dev))
+            if kind == "sq":
+                d["R"] = torch.zeros(n, n, device=dev)
+                d["QR"] = torch.eye(n, device=dev)
+            P = torch.randn(m, rank, generator=g, device=dev)
+            Q = torch.randn(n, rank, generator=g, device=dev)
+            mats.append(d)
+            spikes.append((P @ Q.T, g))
+    def fill():
+        for d, (S, g) in zip(mats, spikes):
+            E = torch.randn(d["G"].shape, generator=g, device=dev) * noise
+            d["G"].copy_(E + S * (ratio * E.norm() / S.norm()))
+    return mats, fill
+
+
+def soap_bench(ctx, dev, steps=3, warm=10):
+    import torch
+    mats, fill = soap_workload(dev)
+    fl, rot = 0.0, 0.0
+    for d in mats:
+        f, r = soap_flops(d["W"].shape[0], d["W"].shape[1], "L" in d, "R" in d)
+        fl += f
+        rot += r
+    hp = dict(lr=3e-3, beta1=0.95, beta2=0.95, eps=1e-8, weight_decay=0.0)
+    for t in range(1, warm + 1):
+        fill()
+        ctx.soap_step(mats, t, **hp)
+    torch.cuda.synchronize()
+    ctx.profile(True)
+    ctx.profile_read()
+    total = 0.0
+    for t in range(warm + 1, warm + 1 + steps):
+        fill()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        ctx.soap_step(mats, t, reserve=False, **hp)
+        e.record()
+        torch.cuda.synchronize()
+        total += s.elapsed_time(e)
+    prof = ctx.profile_read()
+    ctx.profile(False)
+    ms = total / steps
+    k = {kk: round(v[0] / steps, 3) for kk, v in prof.items() if v[2]}
+    rot_ms = prof["soap_rot"][0] / steps
+    rot_exec = prof["soap_rot"][1] / steps
+    return {"workload": "soap_step 4 x 4096^2 (two-sided) + 4 x 4096x14336 (left side only), step 11",
+            "ms": round(ms, 3), "TFLOP/s": round(fl / (ms / 1e3) / 1e12, 1),
+            "flops_per_step": fl, "matrices_per_s": round(len(mats) / (ms / 1e3), 1),
+            "kernels_ms_per_step": k,
+            "rotation_gemm": {"ms": round(rot_ms, 3),
+                              "useful_TFLOP/s": round(rot / (rot_ms / 1e3) / 1e12, 1) if rot_ms else None,
+                              "executed_TFLOP/s": round(rot_exec / (rot_ms / 1e3) / 1e12, 1) if rot_ms else None,
+                              "note": "two-plane operands: 3 bf16 MMAs per useful product"},
+            "gpu_launches": int(sum(v[2] for v in prof.values()) / steps)}
+
+
 def extras(ctx, dev, args):
     """The other workloads, measured the same way (short runs)."""
     import torch
@@ -417,6 +504,9 @@ def extras(ctx, dev, args):
                                    "TFLOP/s": round(4096 * page_flops(128, 128) / (ms / 1e3) / 1e12, 2)}
     res["ns_sweep"] = sweep
     del Ht, Ho
+    ctx.workspace = None
+    torch.cuda.empty_cache()
+    res["soap"] = soap_bench(ctx, dev)
     ctx.workspace = None
     torch.cuda.empty_cache()
     return res
@@ -476,6 +566,20 @@ def run_reference(args, world, rank):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_soap_only(args, world, rank, local):
+    """The SOAP step alone (profiling and ncu runs)."""
+    import torch
+    from matrix_aware_optimizers_muon_b200 import Context
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ctx = Context(local)
+    res = soap_bench(ctx, dev, steps=args.steps, warm=max(args.warmup, 1))
+    return {"metric": METRIC, "value": res["TFLOP/s"], "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": {"workload": res["workload"]},
+            "soap": res}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -486,12 +590,16 @@ def main():
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--workload", choices=["muon", "soap"], default="muon",
+                    help="muon: the dense-GPT Muon step (the benchmark line); soap: the SOAP step alone")
     ap.add_argument("--layers", type=int, default=32,
                     help="dense-GPT layers (32 = the benchmark workload; fewer for small profiling cases)")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     if args.impl == "reference":
         out = run_reference(args, world, rank)
+    elif args.workload == "soap":
+        out = run_soap_only(args, world, rank, local)
     else:
         out = run_ours(args, world, rank, local)
     if rank == 0 and out is not None:

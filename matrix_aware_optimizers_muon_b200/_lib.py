@@ -21,7 +21,8 @@ MO_ERR_DEVICE = -5
 OP_MUON, OP_SOAP, OP_NS = 0, 1, 2
 
 # kernel kinds reported by mo_profile_read
-KINDS = ["prep", "norm", "gram", "poly", "update", "apply", "soap_ew", "soap_gemm", "soap_qr", "gemm"]
+KINDS = ["prep", "norm", "gram", "poly", "update", "apply", "soap_ew", "soap_rot", "soap_qr", "gemm",
+         "soap_ema", "qr_chol", "qr_rowblock", "qr_trail"]
 
 
 class MuonMat(ctypes.Structure):

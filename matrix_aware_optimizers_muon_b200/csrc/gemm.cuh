@@ -118,12 +118,12 @@ __device__ __forceinline__ float ipow_scale(const float* s, int b, int pw) {
   return pw == 1 ? v : v * v;
 }
 
-// Load 32 consecutive C values of row r starting at column c0 (bounded by N).
-__device__ __forceinline__ void load_c32(const GemmParams& p, int b, int r, int c0, float (&c)[32]) {
-  const bool full = c0 + 32 <= p.N;
-  if (p.c_f32) {
-    const float* src = reinterpret_cast<const float*>(c_base(p, b)) + (long long)r * p.ldc + c0;
-    if (full) {
+// Load n (<= 32) consecutive values at base + off (fp32 or bf16) into c[0..31];
+// the vector path needs n == 32 and 16-byte aligned rows.
+__device__ __forceinline__ void load_row32(const char* base, int f32, long long off, int n, float (&c)[32]) {
+  if (f32) {
+    const float* src = reinterpret_cast<const float*>(base) + off;
+    if (n == 32) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float4 v = reinterpret_cast<const float4*>(src)[i];
@@ -131,12 +131,11 @@ __device__ __forceinline__ void load_c32(const GemmParams& p, int b, int r, int 
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) c[i] = (c0 + i < p.N) ? src[i] : 0.0f;
+      for (int i = 0; i < 32; ++i) c[i] = i < n ? src[i] : 0.0f;
     }
   } else {
-    const __nv_bfloat16* src =
-        reinterpret_cast<const __nv_bfloat16*>(c_base(p, b)) + (long long)r * p.ldc + c0;
-    if (full) {
+    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(base) + off;
+    if (n == 32) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint4 v = reinterpret_cast<const uint4*>(src)[i];
@@ -150,45 +149,84 @@ __device__ __forceinline__ void load_c32(const GemmParams& p, int b, int r, int 
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) c[i] = (c0 + i < p.N) ? __bfloat162float(src[i]) : 0.0f;
+      for (int i = 0; i < 32; ++i) c[i] = i < n ? __bfloat162float(src[i]) : 0.0f;
     }
   }
 }
 
-__device__ __forceinline__ void store_one(const GemmParams& p, int b, int r, int c, float v) {
+// Store x[lo..hi) at base + off + i (fp32, bf16, or bf16 as two planes).
+__device__ __forceinline__ void store_row(const GemmParams& p, char* base, long long off, int hi, int lo,
+                                          const float (&x)[32]) {
   if (p.d_f32) {
-    reinterpret_cast<float*>(d_base(p, b))[(long long)r * p.ldd + c] = v;
+    float* dst = reinterpret_cast<float*>(base) + off;
+    if (lo == 0 && hi == 32) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<float4*>(dst)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i >= lo && i < hi) dst[i] = x[i];
+    }
+    return;
+  }
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(base) + off;
+  if (lo == 0 && hi == 32) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x[8 * i + 2 * j], x[8 * i + 2 * j + 1]);
+        w[j] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (p.d_split) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float x0 = x[8 * i + 2 * j], x1 = x[8 * i + 2 * j + 1];
+          const float2 hf = __bfloat1622float2(__floats2bfloat162_rn(x0, x1));
+          const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+          w[j] = *reinterpret_cast<const uint32_t*>(&l);
+        }
+        reinterpret_cast<uint4*>(dst + p.d_plane)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
   } else {
-    __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(d_base(p, b)) + (long long)r * p.ldd + c;
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    *d = h;
-    if (p.d_split) d[p.d_plane] = __float2bfloat16_rn(v - __bfloat162float(h));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (i >= lo && i < hi) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(x[i]);
+        dst[i] = h;
+        if (p.d_split) dst[i + p.d_plane] = __float2bfloat16_rn(x[i] - __bfloat162float(h));
+      }
+    }
   }
 }
 
-__device__ __forceinline__ void store_row32(const GemmParams& p, int b, int r, int c0,
-                                            const float (&x)[32]) {
+// Mirror stores of a symmetric product: element (r, c0 + i) also goes to
+// (c0 + i, r) for lo <= i < hi with c0 + i > r.  For fixed i the lanes of a
+// warp hold consecutive rows r, so each store instruction is contiguous.
+__device__ __forceinline__ void store_mirror(const GemmParams& p, char* base, int r, int c0, int lo, int hi,
+                                             const float (&x)[32]) {
   if (p.d_f32) {
-    float* dst = reinterpret_cast<float*>(d_base(p, b)) + (long long)r * p.ldd + c0;
+    float* dst = reinterpret_cast<float*>(base) + r;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      reinterpret_cast<float4*>(dst)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+    for (int i = 0; i < 32; ++i)
+      if (i >= lo && i < hi && c0 + i > r) dst[(long long)(c0 + i) * p.ldd] = x[i];
   } else {
-    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(d_base(p, b)) + (long long)r * p.ldd + c0;
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(base) + r;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t w[4], wl[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float x0 = x[8 * i + 2 * j], x1 = x[8 * i + 2 * j + 1];
-        const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-        w[j] = *reinterpret_cast<const uint32_t*>(&h);
-        const float2 hf = __bfloat1622float2(h);
-        const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
-        wl[j] = *reinterpret_cast<const uint32_t*>(&l);
+    for (int i = 0; i < 32; ++i) {
+      if (i >= lo && i < hi && c0 + i > r) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(x[i]);
+        dst[(long long)(c0 + i) * p.ldd] = h;
+        if (p.d_split) dst[(long long)(c0 + i) * p.ldd + p.d_plane] = __float2bfloat16_rn(x[i] - __bfloat162float(h));
       }
-      reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[0], w[1], w[2], w[3]);
-      if (p.d_split) reinterpret_cast<uint4*>(dst + p.d_plane)[i] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
     }
   }
 }
@@ -344,6 +382,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
+    const bool has_c = p.C != nullptr || p.c_tab != nullptr;
+    const bool adam = p.epi == EPI_ADAM;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -354,8 +394,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int r = tm * GEMM_BM + row_in_tile;
+      const bool row_ok = r < p.M;
       const float alpha = p.alpha * ipow_scale(p.scale, b, p.alpha_pow);
       const float beta = p.beta * ipow_scale(p.scale, b, p.beta_pow);
+      // this matrix's operands, resolved once per tile
+      const char* cbase = has_c ? reinterpret_cast<const char*>(c_base(p, b)) : nullptr;
+      char* dbase = reinterpret_cast<char*>(d_base(p, b));
+      float* vbase = adam ? p.e_tab[b] : nullptr;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
       for (int cc = 0; cc < BN; cc += 32) {
@@ -363,16 +408,16 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tmem_ld32(taddr + cc, v);
         tmem_ld_wait();
         const int c0 = tn * BN + cc;
-        if (r < p.M && c0 < p.N) {
+        if (row_ok && c0 < p.N) {
+          const bool full = c0 + 32 <= p.N;
           float x[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) x[i] = alpha * __uint_as_float(v[i]);
-          if (p.epi == EPI_ADAM) {
+          if (adam) {
             // V <- b2 V + (1 - b2) G'^2 ;  Dbar = (M' / bc1) / (sqrt(V / bc2) + eps)
             float mr[32];
-            load_c32(p, b, r, c0, mr);
-            float* vp = (p.e_tab ? p.e_tab[b] : nullptr) + (long long)r * p.lde + c0;
-            const bool full = c0 + 32 <= p.N;
+            load_row32(cbase, p.c_f32, (long long)r * p.ldc + c0, full ? 32 : p.N - c0, mr);
+            float* vp = vbase + (long long)r * p.lde + c0;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               if (full || c0 + i < p.N) {
@@ -382,32 +427,20 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 x[i] = (mr[i] * p.adam_ibc1) / (sqrtf(vn * p.adam_ibc2) + p.adam_eps);
               }
             }
-          } else if (p.C != nullptr || p.c_tab != nullptr) {
+          } else if (has_c) {
             float c[32];
-            load_c32(p, b, r, c0, c);
+            load_row32(cbase, p.c_f32, (long long)r * p.ldc + c0, full ? 32 : p.N - c0, c);
 #pragma unroll
             for (int i = 0; i < 32; ++i) x[i] = fmaf(beta, c[i], x[i]);
           }
           if (!p.sym) {
-            if (c0 + 32 <= p.N) {
-              store_row32(p, b, r, c0, x);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (c0 + i < p.N) store_one(p, b, r, c0 + i, x[i]);
-            }
+            store_row(p, dbase, (long long)r * p.ldd + c0, full ? 32 : p.N - c0, 0, x);
           } else if (c0 + 31 >= r) {
-            // upper part of this row chunk: store it and its mirror image
-            if (c0 >= r && c0 + 32 <= p.N) {
-              store_row32(p, b, r, c0, x);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (c0 + i >= r && c0 + i < p.N) store_one(p, b, r, c0 + i, x[i]);
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (c0 + i > r && c0 + i < p.N) store_one(p, b, c0 + i, r, x[i]);
+            // upper part of this row chunk: store it, then its mirror image
+            const int lo = c0 >= r ? 0 : r - c0;          // first column with c >= r
+            const int hi = full ? 32 : p.N - c0;
+            store_row(p, dbase, (long long)r * p.ldd + c0, hi, lo, x);
+            store_mirror(p, dbase, r, c0, lo, hi, x);
           }
         }
       }

@@ -20,6 +20,10 @@ enum ProfKind {
   PK_SOAP_GEMM = 7,  // SOAP tensor-core products
   PK_SOAP_QR = 8,    // SOAP QR (Cholesky / triangular kernels)
   PK_GEMM = 9,       // stand-alone mo_gemm_bf16
+  PK_SOAP_EMA = 10,  // SOAP factor EMAs (symmetric products)
+  PK_QR_CHOL = 11,   // QR: diagonal-block Cholesky + inverse
+  PK_QR_ROWBLK = 12, // QR: panel / TRSM row blocks times the block inverse
+  PK_QR_TRAIL = 13,  // QR: tensor-core trailing updates
   PK_COUNT = 16
 };
 

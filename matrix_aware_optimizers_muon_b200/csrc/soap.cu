@@ -185,7 +185,6 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
   // ---------------------------------------------------------------- phase 1
   for (const Group& g : P.groups) {
     const int c = (int)g.items.size();
-    const long long mn = g.m * g.n;
     void** tab = at<void*>(ws, g.tabs);       // [L | R | V | W] pointer tables
     const void* ptrs[SOAP_MAXB];
     for (int k = 0; k < 4; ++k) {
@@ -222,7 +221,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
       op.alpha = 1.f - bs; op.beta = bs;
       op.C = tab; op.c_tab = (const void* const*)(tab + 0 * SOAP_MAXB); op.ldc = g.m; op.c_f32 = 1;
       op.D = tab; op.d_tab = (void* const*)(tab + 0 * SOAP_MAXB); op.ldd = g.m; op.d_f32 = 1;
-      op.kind = PK_SOAP_GEMM;
+      op.kind = PK_SOAP_EMA;
       if ((e = launch_gemm(op, status, s)) != cudaSuccess) return e;
     }
     if (g.right) {         // R <- bs R + (1 - bs) Gb^T Gb
@@ -233,7 +232,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
       op.alpha = 1.f - bs; op.beta = bs;
       op.C = tab; op.c_tab = (const void* const*)(tab + 1 * SOAP_MAXB); op.ldc = g.n; op.c_f32 = 1;
       op.D = tab; op.d_tab = (void* const*)(tab + 1 * SOAP_MAXB); op.ldd = g.n; op.d_f32 = 1;
-      op.kind = PK_SOAP_GEMM;
+      op.kind = PK_SOAP_EMA;
       if ((e = launch_gemm(op, status, s)) != cudaSuccess) return e;
     }
   }
@@ -337,7 +336,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
           float* c22 = C + (k0 + QR_B) * kp + (k0 + QR_B);
           op.C = c22; op.ldc = kp; op.strideC = kk; op.c_f32 = 1;
           op.D = c22; op.ldd = kp; op.strideD = kk; op.d_f32 = 1;
-          op.kind = PK_SOAP_QR;
+          op.kind = PK_QR_TRAIL;
           if ((e = launch_gemm(op, status, s)) != cudaSuccess) return e;
           GemmOp t;         // Y[:, k0+128:] -= Q_j L21^T
           t.A = Qjpl; t.lda = QR_B; t.strideA = kp * QR_B;
@@ -348,7 +347,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
           float* yr = Y + (k0 + QR_B);
           t.C = yr; t.ldc = kp; t.strideC = kk; t.c_f32 = 1;
           t.D = yr; t.ldd = kp; t.strideD = kk; t.d_f32 = 1;
-          t.kind = PK_SOAP_QR;
+          t.kind = PK_QR_TRAIL;
           if ((e = launch_gemm(t, status, s)) != cudaSuccess) return e;
         }
       }

@@ -122,108 +122,127 @@ __global__ void shift_diag_kernel(float* C, long long ld, long long stride, int 
   if (i < n) C[(size_t)b * stride + (long long)i * ld + i] += shift;
 }
 
-// One CTA (1024 threads) per matrix: Cholesky of a 128 x 128 block in shared
-// memory, then the inverse of the lower factor, 8 threads per column.
-__global__ void __launch_bounds__(1024) chol_diag_kernel(const float* C, long long ld, long long stride,
-                                                         int k0, float* Dinv, const FlagTable flags) {
+// One CTA (256 threads) per matrix: Cholesky of the 128 x 128 diagonal block
+// in shared memory, then the inverse of its lower factor.  Thread (ty, tx)
+// of a 16 x 16 grid owns rows i = ty (mod 16) and columns c = tx (mod 16) of
+// the trailing update.
+__global__ void __launch_bounds__(256) chol_diag_kernel(const float* C, long long ld, long long stride,
+                                                        int k0, float* Dinv, const FlagTable flags) {
   extern __shared__ float sm[];
-  float* A = sm;                      // [128][129]
-  float* X = sm + QR_B * (QR_B + 1);  // [128][129]
   constexpr int LDS = QR_B + 1;
+  float* A = sm;                      // [128][129]
+  float* X = sm + QR_B * LDS;         // [128][129]
+  __shared__ float piv_inv;
+  __shared__ int bad;
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;
   const float* src = C + (size_t)b * stride + (long long)k0 * ld + k0;
   for (int e = tid; e < QR_B * QR_B; e += blockDim.x) {
-    const int r = e / QR_B, c = e % QR_B;
+    const int r = e >> 7, c = e & 127;
     A[r * LDS + c] = src[(long long)r * ld + c];
   }
-  __shared__ int bad;
   if (tid == 0) bad = 0;
   __syncthreads();
   for (int j = 0; j < QR_B; ++j) {
     if (tid == 0) {
       const float d = A[j * LDS + j];
       if (!(d > 0.f)) bad = 1;
-      A[j * LDS + j] = sqrtf(d);
+      const float sq = sqrtf(d);
+      A[j * LDS + j] = sq;
+      piv_inv = 1.0f / sq;
     }
     __syncthreads();
-    const float piv = A[j * LDS + j];
-    for (int i = j + 1 + tid; i < QR_B; i += blockDim.x) A[i * LDS + j] /= piv;
+    if (tid > j && tid < QR_B) A[tid * LDS + j] *= piv_inv;
     __syncthreads();
-    // trailing lower update: A[i][c] -= A[i][j] A[c][j] for j < c <= i
-    const int n = QR_B - 1 - j;
-    const int tot = n * (n + 1) / 2;
-    for (int e = tid; e < tot; e += blockDim.x) {
-      // e -> (i, c) with 0 <= c <= i < n (row-major lower triangle)
-      int i = (int)((sqrtf(8.0f * e + 1.0f) - 1.0f) * 0.5f);
-      while ((i + 1) * (i + 2) / 2 <= e) ++i;
-      while (i * (i + 1) / 2 > e) --i;
-      const int c = e - i * (i + 1) / 2;
-      const int ii = i + j + 1, cc = c + j + 1;
-      A[ii * LDS + cc] -= A[ii * LDS + j] * A[cc * LDS + j];
+    // A[i][c] -= L[i][j] L[c][j] for j < c <= i
+    const int i0 = j + 1 + ((ty - (j + 1)) & 15);      // first owned row > j
+    for (int i = i0; i < QR_B; i += 16) {
+      const float lij = A[i * LDS + j];
+      const int c0 = j + 1 + ((tx - (j + 1)) & 15);
+      for (int c = c0; c <= i; c += 16) A[i * LDS + c] = fmaf(-lij, A[c * LDS + j], A[i * LDS + c]);
     }
     __syncthreads();
   }
-  // inverse of the lower factor: X = L^{-1}, row by row; 8 threads per column
-  const int col = tid >> 3, part = tid & 7;
+  // X = L^{-1} by forward substitution, two threads per column (same warp)
+  const int col = tid >> 1, half = tid & 1;
   for (int i = 0; i < QR_B; ++i) {
     float s = 0.f;
-    if (col < i) {
-      for (int p = col + part; p < i; p += 8) s = fmaf(A[i * LDS + p], X[p * LDS + col], s);
-    }
+    if (col < i)
+      for (int p = col + half; p < i; p += 2) s = fmaf(A[i * LDS + p], X[p * LDS + col], s);
     s += __shfl_xor_sync(0xffffffffu, s, 1);
-    s += __shfl_xor_sync(0xffffffffu, s, 2);
-    s += __shfl_xor_sync(0xffffffffu, s, 4);
-    if (part == 0) {
-      float v;
-      if (col < i) v = -s / A[i * LDS + i];
-      else if (col == i) v = 1.0f / A[i * LDS + i];
-      else v = 0.f;
-      X[i * LDS + col] = v;
-    }
-    __syncthreads();
+    const float v = col < i ? -s / A[i * LDS + i] : (col == i ? 1.0f / A[i * LDS + i] : 0.f);
+    if (half == 0) X[i * LDS + col] = v;
+    __syncwarp();
   }
+  __syncthreads();
   const float nanv = __int_as_float(0x7fc00000);
   float* dst = Dinv + (size_t)b * QR_B * QR_B;
   for (int e = tid; e < QR_B * QR_B; e += blockDim.x) {
-    const int r = e / QR_B, c = e % QR_B;
+    const int r = e >> 7, c = e & 127;
     dst[e] = bad ? nanv : X[r * LDS + c];
   }
   if (tid == 0 && bad && flags.f[b] != nullptr) *flags.f[b] = 1;
 }
 
-// out[r][c] = sum_{p <= c} in[r][p] Dinv[c][p]   (in * Dinv^T, Dinv lower)
-// 64 rows per CTA, 256 threads; Dinv^T and the input rows staged in smem.
+// out[r][c] = sum_{p <= c} in[r][p] Dinv[c][p]   (in * Dinv^T, Dinv lower).
+// 64 rows per CTA, 256 threads; thread (ty, tx) computes rows 4 ty .. +3 and
+// columns 8 tx .. +7 from transposed shared copies of the rows and of Dinv.
 __global__ void __launch_bounds__(256) rowblock_kernel(const RowBlockArgs a) {
   extern __shared__ float sm[];
-  float* D = sm;                       // Dinv [128][129]
-  float* R = sm + QR_B * (QR_B + 1);   // rows [64][129]
-  constexpr int LDS = QR_B + 1;
+  constexpr int LDD = QR_B + 4;        // Dt[p][c] = Dinv[c][p]
+  constexpr int LDR = 64 + 4;          // Rt[p][r] = in[r0 + r][p]
+  float* Dt = sm;
+  float* Rt = sm + QR_B * LDD;
   const int b = blockIdx.y;
   const int r0 = blockIdx.x * 64;
   const float* dinv = a.Dinv + (size_t)b * QR_B * QR_B;
-  for (int e = threadIdx.x; e < QR_B * QR_B; e += blockDim.x) D[(e / QR_B) * LDS + e % QR_B] = dinv[e];
+  for (int e = threadIdx.x; e < QR_B * QR_B; e += blockDim.x) {
+    const int c = e >> 7, p = e & 127;
+    Dt[p * LDD + c] = dinv[e];
+  }
   const float* in = a.in + (size_t)b * a.in_stride;
   for (int e = threadIdx.x; e < 64 * QR_B; e += blockDim.x) {
-    const int r = e / QR_B, c = e % QR_B;
-    R[r * LDS + c] = (r0 + r < a.rows) ? in[(long long)(r0 + r) * a.ld_in + c] : 0.f;
+    const int r = e >> 7, p = e & 127;
+    Rt[p * LDR + r] = (r0 + r < a.rows) ? in[(long long)(r0 + r) * a.ld_in + p] : 0.f;
   }
   __syncthreads();
-  // thread -> (row group of 4, column c); 256 threads = 64 columns x 4 ... loop over 128 columns
-  for (int e = threadIdx.x; e < 64 * QR_B; e += blockDim.x) {
-    const int r = e / QR_B, c = e % QR_B;
-    if (r0 + r >= a.rows) continue;
-    float s = 0.f;
-    for (int p = 0; p <= c; ++p) s = fmaf(R[r * LDS + p], D[c * LDS + p], s);
-    const long long row = r0 + r;
-    if (a.out) a.out[(size_t)b * a.out_stride + row * a.ld_out + c] = s;
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
+  const int pmax = 8 * tx + 7;         // Dinv is lower: p <= c
+  for (int p = 0; p <= pmax; ++p) {
+    const float4 rv = *reinterpret_cast<const float4*>(&Rt[p * LDR + 4 * ty]);
+    const float4 d0 = *reinterpret_cast<const float4*>(&Dt[p * LDD + 8 * tx]);
+    const float4 d1 = *reinterpret_cast<const float4*>(&Dt[p * LDD + 8 * tx + 4]);
+    const float rr[4] = {rv.x, rv.y, rv.z, rv.w};
+    const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[i][k] = fmaf(rr[i], dd[k], acc[i][k]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const long long row = r0 + 4 * ty + i;
+    if (row >= a.rows) continue;
+    const int c0 = 8 * tx;
+    if (a.out) {
+      float* o = a.out + (size_t)b * a.out_stride + row * a.ld_out + c0;
+      reinterpret_cast<float4*>(o)[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      reinterpret_cast<float4*>(o)[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+    }
     if (a.planes) {
-      __nv_bfloat16 h, m, l;
-      split3(s, h, m, l);
-      __nv_bfloat16* d = a.planes + (size_t)b * a.mat_stride + row * QR_B + c;
-      d[0] = h;
-      d[a.plane_stride] = m;
-      d[2 * a.plane_stride] = l;
+      __nv_bfloat16* d = a.planes + (size_t)b * a.mat_stride + row * QR_B + c0;
+      union Pack { __nv_bfloat16 h[8]; uint4 u; } hv, mv, lv;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) split3(acc[i][k], hv.h[k], mv.h[k], lv.h[k]);
+      *reinterpret_cast<uint4*>(d) = hv.u;
+      *reinterpret_cast<uint4*>(d + a.plane_stride) = mv.u;
+      *reinterpret_cast<uint4*>(d + 2 * a.plane_stride) = lv.u;
     }
   }
 }
@@ -305,19 +324,19 @@ void launch_shift_diag(float* C, long long ld, long long mat_stride, int count, 
 
 void launch_chol_diag(const float* C, long long ld, long long mat_stride, int count, int k0,
                       float* Dinv, const FlagTable& flags, cudaStream_t s) {
-  ProfScope prof(PK_SOAP_QR, s);
+  ProfScope prof(PK_QR_CHOL, s);
   const int smem = 2 * QR_B * (QR_B + 1) * 4;
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     attr = true;
   }
-  chol_diag_kernel<<<count, 1024, smem, s>>>(C, ld, mat_stride, k0, Dinv, flags);
+  chol_diag_kernel<<<count, 256, smem, s>>>(C, ld, mat_stride, k0, Dinv, flags);
 }
 
 void launch_rowblock_dinv(const RowBlockArgs& a, cudaStream_t s) {
-  ProfScope prof(PK_SOAP_QR, s);
-  const int smem = (QR_B + 64) * (QR_B + 1) * 4;
+  ProfScope prof(PK_QR_ROWBLK, s);
+  const int smem = (QR_B * (QR_B + 4) + QR_B * (64 + 4)) * 4;
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(rowblock_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

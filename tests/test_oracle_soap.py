@@ -152,10 +152,54 @@ def test_first_step_from_zero_state():
                          beta2=0.9)
     np.testing.assert_allclose(out["L"], 0.1 * G @ G.T, atol=1e-14)
     np.testing.assert_allclose(out["R"], 0.1 * G.T @ G, atol=1e-14)
-    # Q_L's columns are the Gram-Schmidt orthonormalisation of L_1's columns
-    Qg, _ = _gram_schmidt(out["L"].tolist())
+    # Q_L's columns are the Gram-Schmidt orthonormalisation of the damped
+    # L_1's columns (damping 1e-5 of the trace, summed here by a Python loop)
+    L1 = out["L"].tolist()
+    d = 1e-5 * sum(L1[i][i] for i in range(m))
+    Qg, _ = _gram_schmidt([[L1[i][j] + (d if i == j else 0.0) for j in range(m)] for i in range(m)])
     np.testing.assert_allclose(out["QL"], Qg, atol=1e-9)
     np.testing.assert_allclose(out["QL"].T @ out["QL"], np.eye(m), atol=1e-12)
+    # without damping the factor's own Gram-Schmidt basis
+    out0 = soap.soap_step(np.zeros((m, n)), G, np.zeros((m, n)), np.zeros((m, n)),
+                          np.zeros((m, m)), np.eye(m), None, None, beta2=0.9, damping=0.0)
+    Qg0, _ = _gram_schmidt(out0["L"].tolist())
+    np.testing.assert_allclose(out0["QL"], Qg0, atol=1e-9)
+
+
+def test_damped_power_step_worked_example():
+    """2 x 2 by hand: L = diag(3, 1), old basis the rotation with cos 0.6 and
+    sin 0.8.  trace(L) = 4, so d = 4e-5 and (L + d I) Q_old has first column
+    (3.00004 * 0.6, 1.00004 * 0.8) = (1.800024, 0.800032); the new basis is
+    that column normalised and its positive-diagonal completion.  The state
+    is chosen so that the EMA leaves L = diag(3, 1): beta2 = 0.5, L_prev =
+    diag(6, 2) - G G^T with G = diag(0, 0) -> L_prev = diag(6, 2)."""
+    L_prev = np.diag([6.0, 2.0])
+    Q_old = np.array([[0.6, -0.8], [0.8, 0.6]])
+    Z = np.zeros((2, 2))
+    out = soap.soap_step(Z, Z, Z, Z, L_prev, Q_old, t=1, beta2=0.5)
+    np.testing.assert_allclose(out["L"], np.diag([3.0, 1.0]), atol=0)
+    r = (1.800024 ** 2 + 0.800032 ** 2) ** 0.5
+    q1 = np.array([1.800024, 0.800032]) / r
+    expect = np.array([[q1[0], -q1[1]], [q1[1], q1[0]]])
+    np.testing.assert_allclose(out["QL"], expect, rtol=0, atol=1e-13)
+    # the undamped step differs at the 1e-5 level, far above the tolerance
+    r0 = (1.8 ** 2 + 0.8 ** 2) ** 0.5
+    assert abs(out["QL"][0, 0] - 1.8 / r0) > 1e-7
+
+
+def test_damping_keeps_an_exact_eigenbasis_and_a_zero_factor():
+    rng = np.random.default_rng(31)
+    m = 7
+    U, _ = np.linalg.qr(rng.standard_normal((m, m)))
+    L = (U * np.array([9.0, 5.0, 3.0, 2.0, 1.0, 0.5, 0.1])) @ U.T
+    Z = np.zeros((m, 3))
+    # shampoo_beta = 1: the factor is L itself; U is kept up to column signs
+    out = soap.soap_step(Z, Z, Z, Z, L, U, None, None, shampoo_beta=1.0)
+    np.testing.assert_allclose(np.abs(np.sum(out["QL"] * U, axis=0)), np.ones(m), atol=1e-12)
+    # a factor that has seen only zero gradients keeps its basis: d = 1 and
+    # the positive-diagonal QR of an orthogonal U is U itself (R = I)
+    out = soap.soap_step(Z, Z, Z, Z, np.zeros((m, m)), U, None, None)
+    np.testing.assert_allclose(out["QL"], U, atol=1e-12)
 
 
 def test_power_iteration_converges_to_eigenbasis():
@@ -204,3 +248,17 @@ def test_bf16_mode_without_rounding_is_fp64(monkeypatch):
         a = soap.soap_step(*args, *sides, t=3, precision="fp64")
         b = soap.soap_step(*args, *sides, t=3, precision="bf16")
         np.testing.assert_allclose(a["W"], b["W"], atol=1e-12)
+
+
+def test_stale_basis_keeps_q_and_updates_factors():
+    """Between refreshes the factors keep accumulating and the basis stays."""
+    rng = np.random.default_rng(30)
+    m, n = 5, 8
+    G = rng.standard_normal((m, n))
+    QL, _ = np.linalg.qr(rng.standard_normal((m, m)))
+    L0 = np.eye(m)
+    out = soap.soap_step(np.zeros((m, n)), G, np.zeros((m, n)), np.zeros((m, n)), L0, QL,
+                         beta2=0.9, basis_refresh=False)
+    np.testing.assert_array_equal(out["QL"], QL)
+    np.testing.assert_allclose(out["L"], 0.9 * L0 + 0.1 * G @ G.T, atol=1e-14)
+    np.testing.assert_allclose(out["Gr"], QL.T @ G, atol=1e-14)

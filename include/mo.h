@@ -97,7 +97,8 @@ MO_API mo_status mo_device_status(mo_ctx* ctx, void* stream, int32_t* status);
  * cast, 1 norm finalize, 2 Gram X X^T, 3 polynomial b A + c A A, 4 update
  * a X + P X, 5 apply / store, 6 SOAP elementwise, 7 SOAP rotations, 8 SOAP
  * power step and QR (other), 9 mo_gemm_bf16, 10 SOAP factor EMAs, 11 QR
- * diagonal Cholesky blocks, 12 QR row-block solves, 13 QR trailing updates. */
+ * diagonal Cholesky blocks, 12 QR row-block solves, 13 QR trailing updates,
+ * 14 fused small-matrix Newton-Schulz / Muon. */
 MO_API mo_status mo_profile_enable(mo_ctx* ctx, int enable);
 MO_API mo_status mo_profile_read(mo_ctx* ctx, double* ms, double* flops, int64_t* launches, int nkinds);
 
@@ -182,8 +183,14 @@ MO_API mo_status ns_orthogonalize_static(mo_ctx* ctx, const float* in, float* ou
  * notes on SOAP, Muon, and Beyond", sections 1 and 4; "LLM Optimizers",
  * section 11.1; "初探优化器（一）", section 6.2), at step t >= 1:
  *   L <- bs L + (1 - bs) G G^T,   R <- bs R + (1 - bs) G^T G
- *   Q_L <- qr(L Q_L),             Q_R <- qr(R Q_R)   (one power step + QR,
- *                                  diag(R) > 0; fp32-accurate)
+ *   Q_L <- qr((L + dL I) Q_L),    Q_R <- qr((R + dR I) Q_R)
+ *                                 (one power step + QR, diag(R) > 0,
+ *                                  fp32-accurate; dL = damping * trace(L),
+ *                                  or 1 when the trace is zero: the damping
+ *                                  of the Shampoo family, "Matrix optimizers:
+ *                                  K-FAC, Shampoo and Muon", Shampoo; it keeps
+ *                                  the eigenvectors and bounds cond by
+ *                                  1 + 1 / damping)
  *   M <- b1 M + (1 - b1) G        (original space)
  *   M' = Q_L^T M Q_R,  G' = Q_L^T G Q_R
  *   V <- b2 V + (1 - b2) G' * G'
@@ -209,6 +216,13 @@ typedef struct {
   float lr, beta1, beta2, shampoo_beta, eps, weight_decay;
   int bias_correction;  /* 1: divide by 1 - beta^t (default) */
   int32_t* nonfinite;   /* optional device int32[n]: the QR met a non-positive pivot */
+  int skip_refresh;     /* 1: update L, R but keep Q_L, Q_R this step (the steps
+                           between refreshes when the basis is refreshed only
+                           every f steps); 0: refresh every step (default) */
+  float damping;        /* relative damping of the power step, in (0, 1e-2]
+                           (1e-5 by default in the binding); with damping
+                           below 1e-6 the fp32 Cholesky QR may meet a
+                           non-positive pivot on singular factors */
 } mo_soap_cfg;
 
 MO_API mo_status soap_step(mo_ctx* ctx, const mo_soap_mat* mats /* host array */, int n,

@@ -165,9 +165,11 @@ class Context:
 
     def soap_step(self, mats, step, *, lr=3e-3, beta1=0.95, beta2=0.95, shampoo_beta=None,
                   eps=1e-8, weight_decay=0.0, bias_correction=True, nonfinite=None, stream=None,
-                  reserve=True):
+                  reserve=True, refresh=True, damping=1e-5):
         """One SOAP step.  ``mats`` is a list of dicts with keys W, G, M, V and
-        optionally L, QL, R, QR (missing or None: identity basis on that side)."""
+        optionally L, QL, R, QR (missing or None: identity basis on that side).
+        ``refresh=False`` keeps the bases this step (factors still update).
+        ``damping``: the power step runs on L + damping * trace(L) I."""
         n = len(mats)
         arr = (SoapMat * max(n, 1))()
         for i, d in enumerate(mats):
@@ -183,7 +185,8 @@ class Context:
             if self.workspace is None or self.workspace.numel() < need.value:
                 self.attach_workspace(need.value, stream)
         sb = beta2 if shampoo_beta is None else shampoo_beta
-        cfg = SoapCfg(lr, beta1, beta2, sb, eps, weight_decay, int(bias_correction), _ptr(nonfinite))
+        cfg = SoapCfg(lr, beta1, beta2, sb, eps, weight_decay, int(bias_correction), _ptr(nonfinite),
+                      0 if refresh else 1, damping)
         self._check(self.lib.soap_step(self.handle, arr, n, byref(cfg), int(step), self._stream(stream)))
 
     def gemm_bf16(self, A, B, D, *, M, N, K, batch=1, a_mn=False, b_mn=False, sym=False,

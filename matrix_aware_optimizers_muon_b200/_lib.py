@@ -22,7 +22,7 @@ OP_MUON, OP_SOAP, OP_NS = 0, 1, 2
 
 # kernel kinds reported by mo_profile_read
 KINDS = ["prep", "norm", "gram", "poly", "update", "apply", "soap_ew", "soap_rot", "soap_qr", "gemm",
-         "soap_ema", "qr_chol", "qr_rowblock", "qr_trail"]
+         "soap_ema", "qr_chol", "qr_rowblock", "qr_trail", "ns_small"]
 
 
 class MuonMat(ctypes.Structure):
@@ -51,7 +51,8 @@ class SoapMat(ctypes.Structure):
 class SoapCfg(ctypes.Structure):
     _fields_ = [("lr", c_float), ("beta1", c_float), ("beta2", c_float),
                 ("shampoo_beta", c_float), ("eps", c_float), ("weight_decay", c_float),
-                ("bias_correction", c_int), ("nonfinite", c_void_p)]
+                ("bias_correction", c_int), ("nonfinite", c_void_p), ("skip_refresh", c_int),
+                ("damping", c_float)]
 
 
 class GemmDesc(ctypes.Structure):

@@ -288,6 +288,8 @@ mo_status soap_step(mo_ctx* ctx, const mo_soap_mat* mats, int n, const mo_soap_c
   auto beta_ok = [](float b) { return b >= 0.f && b < 1.f; };
   if (!beta_ok(cfg->beta1) || !beta_ok(cfg->beta2) || !beta_ok(cfg->shampoo_beta))
     return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: betas must be in [0, 1)");
+  if (!(cfg->damping > 0.f && cfg->damping <= 1e-2f))
+    return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: damping must be in (0, 1e-2]");
   std::vector<mo::SoapItem> items;
   for (int i = 0; i < n; ++i) {
     const mo_soap_mat& m = mats[i];

@@ -12,6 +12,7 @@
 #include <map>
 
 #include "elementwise.cuh"
+#include "ns_small.cuh"
 #include "ns_plan.h"
 #include "profile.h"
 #include "runtime.h"
@@ -88,6 +89,48 @@ cudaError_t ns_run(const std::vector<NsItem>& items, const NsCall& call, char* w
     // launch below covers a contiguous run of one orientation
     std::stable_partition(idx.begin(), idx.end(), [&](int i) { return !is_tall(i); });
     const Layout L = layout_of(s);
+    if (s.mp <= SMALL_MAX_M && s.np <= SMALL_MAX_N) {
+      // small matrices: one fused launch per orientation, no iterate buffers
+      const size_t need = 4 * idx.size() * sizeof(void*);
+      if (need > avail) {
+        *err = "workspace too small for the pointer tables of " + std::to_string(idx.size()) + " matrices";
+        return cudaSuccess;
+      }
+      void** tab = reinterpret_cast<void**>(base);
+      for (int pass = 0; pass < 2; ++pass) {
+        std::vector<const void*> in, mom, out, flg;
+        long long rows = 0, cols = 0;
+        for (int i : idx) {
+          if (is_tall(i) != (pass == 1)) continue;
+          in.push_back(items[i].in); mom.push_back(items[i].mom);
+          out.push_back(items[i].out); flg.push_back(items[i].flag);
+          rows = items[i].rows; cols = items[i].cols;
+        }
+        const int n = (int)in.size();
+        if (n == 0) continue;
+        launch_upload_tables(tab, n, in.data(), mom.data(), out.data(), flg.data(), stream);
+        SmallArgs sa;
+        sa.count = n; sa.rows = (int)rows; sa.cols = (int)cols; sa.tall = pass;
+        sa.mode = call.muon ? 1 : 0;
+        sa.beta = call.beta; sa.nesterov = call.nesterov; sa.ema = call.ema;
+        sa.steps = call.steps; sa.a = call.a; sa.b = call.b; sa.c = call.c; sa.eps = call.eps;
+        const double m = (double)rows, nn = (double)cols;
+        const double scale = call.adjust_lr == 0 ? 0.2 * std::sqrt(std::max(m, nn)) : std::sqrt(std::max(1.0, m / nn));
+        sa.decay = (float)(1.0 - (double)call.lr * (double)call.wd);
+        sa.step = (float)((double)call.lr * scale);
+        sa.in = reinterpret_cast<const float* const*>(tab);
+        sa.mom = call.muon ? reinterpret_cast<float* const*>(tab + n) : nullptr;
+        sa.out = reinterpret_cast<float* const*>(tab + 2 * n);
+        sa.flag = reinterpret_cast<int32_t* const*>(tab + 3 * n);
+        sa.status = status;
+        const int grid = std::min(n, device_sm_count());
+        cudaError_t e = launch_ns_small(sa, grid, stream);
+        if (e != cudaSuccess) return e;
+        // the next launch may reuse the tables only after this one is done
+        // reading them; both run on one stream, so stream order suffices
+      }
+      continue;
+    }
     if (L.total(1) > avail) {
       *err = "workspace too small for a " + std::to_string(s.mp) + " x " + std::to_string(s.np) +
              " matrix (need " + std::to_string(L.total(1) + WS_HEADER) + " bytes)";

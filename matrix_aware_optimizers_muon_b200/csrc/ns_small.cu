@@ -1,0 +1,327 @@
+// Fused Newton-Schulz (and Muon step) for small matrices: m' <= 128 and
+// n' <= 256 after orientation.  One persistent CTA walks over the matrices;
+// for each it keeps X (m' x n'), A = X X^T and P = b A + c A A in shared
+// memory (128-byte-swizzled K-major tiles, zero padded to 128 x 256 / 128 x
+// 128) and the fp32 products in tensor memory, so HBM sees only the inputs
+// and the outputs.  The arithmetic and rounding points are those of the
+// batched path: N = G + beta B (Muon) or the input, Nb = bf16(N),
+// inv = 1 / (||N||_F + eps) applied in fp32 inside iteration 0, every stored
+// iterate rounded to bf16.
+//
+// Warps 0-3: workers, thread t owns row t of the oriented matrix (loads,
+// norms, tcgen05.ld epilogues, stores).  Warp 4: TMEM allocation and the
+// single-thread tcgen05.mma issue.
+#include <cuda_bf16.h>
+
+#include "ns_small.cuh"
+#include "profile.h"
+#include "ptx.cuh"
+
+namespace mo {
+
+namespace {
+
+constexpr int SM_THREADS = 160;
+constexpr int CHUNK = 128 * 128;                 // bytes of one 64-column chunk of 128 rows
+constexpr int X_BYTES = 4 * CHUNK;               // up to 256 columns
+constexpr int A_BYTES = 2 * CHUNK;               // 128 x 128
+constexpr int SMEM_BYTES = X_BYTES + 2 * A_BYTES + 1024 + 256;
+constexpr uint32_t TMEM_COLS = 256;
+
+// byte offset of element (r, c) inside a swizzled chunked tile
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  const int chunk = c >> 6, cc = c & 63;
+  return (uint32_t)(chunk * CHUNK + r * 128 + ((((cc >> 3) ^ (r & 7))) << 4) + ((cc & 7) << 1));
+}
+
+// byte offset of the 16-byte unit holding columns [8u, 8u + 8) of row r
+__device__ __forceinline__ uint32_t swz_unit(int r, int u) {
+  const int chunk = u >> 3, uu = u & 7;
+  return (uint32_t)(chunk * CHUNK + r * 128 + ((uu ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// K-major descriptor of a chunked tile, for the k-th 16-wide K step
+__device__ __forceinline__ uint64_t desc_k(uint32_t base, int k) {
+  return smem_desc_sw128(base + (k >> 2) * CHUNK + (k & 3) * 32, 16, 1024);
+}
+
+// MN-major descriptor (B = X with K = rows, N = columns), k-th 16-row K step
+__device__ __forceinline__ uint64_t desc_mn(uint32_t base, int k) {
+  return smem_desc_sw128(base + k * 2048, CHUNK, 1024);
+}
+
+__device__ __forceinline__ void store_unit(uint8_t* tile, int r, int u, const float (&x)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
+    w[j] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  *reinterpret_cast<uint4*>(tile + swz_unit(r, u)) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ void load_unit(const uint8_t* tile, int r, int u, float (&x)[8]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(tile + swz_unit(r, u));
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+    x[2 * j] = f.x;
+    x[2 * j + 1] = f.y;
+  }
+}
+
+__global__ void __launch_bounds__(SM_THREADS, 1) ns_small_kernel(const SmallArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* X = smem;
+  uint8_t* A = smem + X_BYTES;
+  uint8_t* P = A + A_BYTES;
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(P + A_BYTES);
+  uint64_t* work_bar = mma_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(work_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(tmem_slot + 4);      // [4] warp partials
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
+  const int np = a.tall ? a.rows : a.cols;      // oriented cols (<= 256)
+  const int npad = (np + 63) & ~63;             // K of the Gram, N of the update
+  const uint32_t idesc_g = idesc_bf16_f32(128, 128, 0, 0);
+  const uint32_t idesc_u = idesc_bf16_f32(128, npad, 0, 1);
+
+  if (tid == 0) {
+    mbar_init(mma_bar, 1);
+    mbar_init(work_bar, 128);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sX = smem_u32(X), sA = smem_u32(A), sP = smem_u32(P);
+
+  uint32_t mma_phase = 0, work_phase = 0;
+  uint32_t ncommit = 0;                          // MMA thread: commits issued so far
+  bool ok = true;
+  for (int mat = blockIdx.x; mat < a.count && ok; mat += gridDim.x) {
+    if (warp < 4) {
+      // ---- load: momentum, Nesterov, bf16 cast into X (oriented), norm
+      for (int e = tid; e < X_BYTES / 16; e += 128) reinterpret_cast<uint4*>(X)[e] = make_uint4(0, 0, 0, 0);
+      __syncwarp();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const float* G = a.in[mat];
+      float* B = a.mom ? a.mom[mat] : nullptr;
+      const int total = a.rows * a.cols;
+      float ss = 0.f;
+      for (int e = tid; e < total; e += 128) {
+        const int r = e / a.cols, c = e - r * a.cols;
+        const float g = G[e];
+        float n = g;
+        if (a.mode == 1) {
+          const float bn = a.ema ? fmaf(a.beta, B[e], (1.0f - a.beta) * g) : fmaf(a.beta, B[e], g);
+          B[e] = bn;
+          n = a.nesterov ? fmaf(a.beta, bn, g) : bn;
+        }
+        ss = fmaf(n, n, ss);
+        const int xr = a.tall ? c : r, xc = a.tall ? r : c;
+        *reinterpret_cast<__nv_bfloat16*>(X + swz(xr, xc)) = __float2bfloat16_rn(n);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) red[warp] = ss;
+      fence_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const float norm = sqrtf(((red[0] + red[1]) + red[2]) + red[3]);
+      const float inv = 1.0f / (norm + a.eps);
+      if (tid == 0 && a.flag && a.flag[mat]) *a.flag[mat] = isfinite(norm) ? 0 : 1;
+      tc_fence_before();
+      mbar_arrive(work_bar);                     // X ready
+
+      const int r = tid;                         // this thread's row
+      const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+      for (int it = 0; it < a.steps && ok; ++it) {
+        // ---- A = X X^T (scaled by inv^2 in iteration 0)
+        ok = mbar_wait(mma_bar, mma_phase, abort_flag, a.status, DEV_TIMEOUT_ACC_FULL);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        mma_phase ^= 1u;
+        tc_fence_after();
+        const float ga = it == 0 ? inv * inv : 1.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < 128; cc += 32) {
+          uint32_t v[32];
+          tmem_ld32(trow + cc, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = ga * __uint_as_float(v[8 * u + j]);
+            store_unit(A, r, (cc >> 3) + u, x);
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(work_bar);
+        // ---- P = b A + c A A
+        ok = mbar_wait(mma_bar, mma_phase, abort_flag, a.status, DEV_TIMEOUT_ACC_FULL);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        mma_phase ^= 1u;
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < 128; cc += 32) {
+          uint32_t v[32];
+          tmem_ld32(trow + cc, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float av[8], x[8];
+            load_unit(A, r, (cc >> 3) + u, av);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = fmaf(a.b, av[j], a.c * __uint_as_float(v[8 * u + j]));
+            store_unit(P, r, (cc >> 3) + u, x);
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(work_bar);
+        // ---- X' = a X + P X   (iteration 0: inv (a Nb + P Nb))
+        ok = mbar_wait(mma_bar, mma_phase, abort_flag, a.status, DEV_TIMEOUT_ACC_FULL);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        mma_phase ^= 1u;
+        tc_fence_after();
+        const float s_acc = it == 0 ? inv : 1.0f;
+        const float s_x = it == 0 ? a.a * inv : a.a;
+#pragma unroll 1
+        for (int cc = 0; cc < npad; cc += 32) {
+          uint32_t v[32];
+          tmem_ld32(trow + cc, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float xv[8], x[8];
+            load_unit(X, r, (cc >> 3) + u, xv);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = fmaf(s_x, xv[j], s_acc * __uint_as_float(v[8 * u + j]));
+            store_unit(X, r, (cc >> 3) + u, x);
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(work_bar);
+      }
+      // ---- the last X is O (a failed wait skips the store; every thread
+      // still meets the block barrier below, which ends the loop)
+      if (ok) {
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        float* out = a.out[mat];
+        for (int e = tid; e < total; e += 128) {
+          const int rr = e / a.cols, c = e - rr * a.cols;
+          const int xr = a.tall ? c : rr, xc = a.tall ? rr : c;
+          const float o = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(X + swz(xr, xc)));
+          out[e] = a.mode == 1 ? fmaf(a.decay, out[e], -a.step * o) : o;
+        }
+      }
+    } else if (lane == 0) {
+      // ---- MMA issuer: per iteration Gram, A A, P X
+      for (int it = 0; it < a.steps && ok; ++it) {
+        ok = mbar_wait(work_bar, work_phase, abort_flag, a.status, DEV_TIMEOUT_FULL);
+        if (!ok) break;
+        work_phase ^= 1u;
+        tc_fence_after();
+        for (int k = 0; k < npad / 16; ++k)
+          tc_mma_f16(tmem, desc_k(sX, k), desc_k(sX, k), idesc_g, k != 0);
+        tc_commit(mma_bar);
+        ++ncommit;
+        ok = mbar_wait(work_bar, work_phase, abort_flag, a.status, DEV_TIMEOUT_FULL);
+        if (!ok) break;
+        work_phase ^= 1u;
+        tc_fence_after();
+        for (int k = 0; k < 8; ++k)
+          tc_mma_f16(tmem, desc_k(sA, k), desc_k(sA, k), idesc_g, k != 0);
+        tc_commit(mma_bar);
+        ++ncommit;
+        ok = mbar_wait(work_bar, work_phase, abort_flag, a.status, DEV_TIMEOUT_FULL);
+        if (!ok) break;
+        work_phase ^= 1u;
+        tc_fence_after();
+        for (int k = 0; k < 8; ++k)
+          tc_mma_f16(tmem, desc_k(sP, k), desc_mn(sX, k), idesc_u, k != 0);
+        tc_commit(mma_bar);
+        ++ncommit;
+      }
+      if (ok) {
+        // the workers' last arrival (after the final X) closes this matrix
+        ok = mbar_wait(work_bar, work_phase, abort_flag, a.status, DEV_TIMEOUT_FULL);
+        work_phase ^= 1u;
+      }
+    }
+    ok = __syncthreads_and(ok);
+  }
+  // drain: every MMA issued must finish before TMEM is released
+  if (warp == 4 && lane == 0 && ncommit > 0) {
+    tc_commit(mma_bar);
+    mbar_wait_drain(mma_bar, ncommit & 1u, a.status);
+  }
+  __syncthreads();
+  if (warp == 4) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+constexpr int UPLOAD_N = 960;       // 4 x 960 pointers = 30 KB of kernel parameters
+
+struct TableUpload {
+  int n;
+  const void* p[4][UPLOAD_N];
+};
+
+__global__ void upload_tables_kernel(void** dst, int stride, const TableUpload u) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < u.n)
+    for (int t = 0; t < 4; ++t) dst[t * stride + i] = const_cast<void*>(u.p[t][i]);
+}
+
+}  // namespace
+
+void launch_upload_tables(void** dst, int n, const void* const* in, const void* const* mom,
+                          const void* const* out, const void* const* flag, cudaStream_t s) {
+  for (int first = 0; first < n; first += UPLOAD_N) {
+    TableUpload u;
+    u.n = n - first < UPLOAD_N ? n - first : UPLOAD_N;
+    for (int i = 0; i < u.n; ++i) {
+      u.p[0][i] = in[first + i];
+      u.p[1][i] = mom[first + i];
+      u.p[2][i] = out[first + i];
+      u.p[3][i] = flag[first + i];
+    }
+    upload_tables_kernel<<<(u.n + 127) / 128, 128, 0, s>>>(dst + first, n, u);
+  }
+}
+
+cudaError_t launch_ns_small(const SmallArgs& a, int grid, cudaStream_t s) {
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = 1;
+  }
+  ProfScope prof(PK_SMALL, s, 0.0);
+  ns_small_kernel<<<grid, SM_THREADS, SMEM_BYTES, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace mo

@@ -73,7 +73,7 @@ struct Job {
 struct Bucket {
   long long k, kp;
   std::vector<Job> jobs;
-  size_t y, c, ypl, qpl, ppl, qjpl, dinv, invd;
+  size_t y, c, ypl, qpl, ppl, qjpl, dinv, invd, damp;
 };
 
 struct Plan {
@@ -142,6 +142,7 @@ Plan make_plan(const std::vector<SoapItem>& items) {
     b.qjpl = off; off += al(3 * q * b.kp * QR_B * 2);
     b.dinv = off; off += al(q * QR_B * QR_B * 4);
     b.invd = off; off += al(q * b.kp * 4);
+    b.damp = off; off += al(q * 4);
   }
   P.total = off;
   return P;
@@ -238,7 +239,32 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
   }
 
   // ---------------------------------------------------------------- phase 2
+  if (cfg.skip_refresh) {
+    // keep the bases: only their two bf16 planes are needed for the rotations
+    for (const Group& g : P.groups) {
+      const int c = (int)g.items.size();
+      for (int side = 0; side < 2; ++side) {
+        if ((side == 0 && !g.left) || (side == 1 && !g.right)) continue;
+        const long long k = side == 0 ? g.m : g.n;
+        const long long kpad = side == 0 ? g.mpad : g.npad;
+        SplitArgs sq;
+        sq.count = c; sq.rows_valid = (int)k; sq.cols_valid = (int)k;
+        sq.rows_pad = (int)kpad; sq.cols_pad = (int)kpad;
+        for (int j = 0; j < c; ++j) {
+          const mo_soap_mat& m = items[g.items[j]].m;
+          sq.src[j] = side == 0 ? m.QL : m.QR;
+        }
+        sq.lds = k; sq.col_scale = nullptr; sq.write_back = nullptr; sq.ldw = 0; sq.wb_stride = 0;
+        sq.dst = at<__nv_bfloat16>(ws, side == 0 ? g.qlp : g.qrp);
+        sq.ldd = kpad; sq.mat_stride = kpad * kpad; sq.plane_stride = (long long)c * kpad * kpad;
+        sq.nplanes = 2; sq.pad_identity = 0;
+        launch_split(sq, s);
+      }
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   for (const Bucket& bk : P.buckets) {
+    if (cfg.skip_refresh) break;
     const int q = (int)bk.jobs.size();
     const long long k = bk.k, kp = bk.kp, kk = kp * kp;
     float* Y = at<float>(ws, bk.y);
@@ -252,7 +278,18 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
     FlagTable flags;
     for (int j = 0; j < q; ++j) flags.f[j] = items[bk.jobs[j].item].flag;
 
-    // power step: Y = L Q (planes of L into Ypl, planes of the old Q into Qpl)
+    // power step: Y = (L + d I) Q, d = damping * trace(L) (planes of the
+    // damped L into Ypl, planes of the old Q into Qpl)
+    float* damp = at<float>(ws, bk.damp);
+    {
+      DampArgs da;
+      da.count = q; da.k = (int)k; da.rho = cfg.damping; da.delta = damp;
+      for (int j = 0; j < q; ++j) {
+        const mo_soap_mat& m = items[bk.jobs[j].item].m;
+        da.F[j] = bk.jobs[j].left ? m.L : m.R;
+      }
+      launch_damping(da, s);
+    }
     SplitArgs sa;
     sa.count = q; sa.rows_valid = (int)k; sa.cols_valid = (int)k; sa.rows_pad = (int)kp; sa.cols_pad = (int)kp;
     sa.lds = k; sa.col_scale = nullptr; sa.write_back = nullptr; sa.ldw = 0; sa.wb_stride = 0;
@@ -262,7 +299,9 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
       sa.src[j] = bk.jobs[j].left ? m.L : m.R;
     }
     sa.dst = Ypl;
+    sa.diag_add = damp;
     launch_split(sa, s);
+    sa.diag_add = nullptr;
     for (int j = 0; j < q; ++j) {
       const mo_soap_mat& m = items[bk.jobs[j].item].m;
       sa.src[j] = bk.jobs[j].left ? m.QL : m.QR;
@@ -301,8 +340,11 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
         op.kind = PK_SOAP_QR;
         if ((e = launch_gemm(op, status, s)) != cudaSuccess) return e;
       }
-      // the first pass shifts the Gram matrix (unit diagonal, trace kp) so
-      // that its Cholesky exists at any conditioning
+      // The first pass shifts the Gram matrix (unit diagonal, trace kp) by
+      // 1e-5 of its trace, above its fp32 rounding error.  With the damped
+      // factor, cond(Y) <= 1 + 1 / damping (1e5 at the default), and the
+      // shifted pass leaves a Q whose Gram the two unshifted passes
+      // factor safely (cond(Q) below the fp32 limit of Cholesky QR).
       if (pass == 0) launch_shift_diag(C, kp, kk, q, (int)kp, 1e-5f * (float)kp, s);
       for (int jb = 0; jb < nb; ++jb) {
         const long long k0 = (long long)jb * QR_B;

@@ -81,6 +81,7 @@ __global__ void split_kernel(const SplitArgs a) {
   float x;
   if (r < a.rows_valid && c < a.cols_valid) {
     x = a.src[b][(long long)r * a.lds + c];
+    if (a.diag_add && r == c) x += a.diag_add[b];
     if (a.col_scale) x *= a.col_scale[(size_t)b * a.cols_pad + c];
   } else {
     x = (a.pad_identity && r == c) ? 1.0f : 0.0f;
@@ -100,6 +101,21 @@ __global__ void split_kernel(const SplitArgs a) {
     d[a.plane_stride] = m;
     d[2 * a.plane_stride] = l;
   }
+}
+
+__global__ void __launch_bounds__(256) damping_kernel(const DampArgs a) {
+  __shared__ float part[256];
+  const int b = blockIdx.x;
+  const float* F = a.F[b];
+  float t = 0.f;
+  for (int i = threadIdx.x; i < a.k; i += 256) t += F[(long long)i * a.k + i];
+  part[threadIdx.x] = t;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) a.delta[b] = part[0] != 0.f ? a.rho * part[0] : 1.0f;
 }
 
 __global__ void colnorm_kernel(const float* Y, long long ld, long long stride, int rows, int cols,
@@ -306,6 +322,11 @@ void launch_split(const SplitArgs& a, cudaStream_t s) {
   ProfScope prof(PK_SOAP_QR, s);
   dim3 grid((a.cols_pad + 255) / 256, a.rows_pad, a.count);
   split_kernel<<<grid, 256, 0, s>>>(a);
+}
+
+void launch_damping(const DampArgs& a, cudaStream_t s) {
+  ProfScope prof(PK_SOAP_QR, s);
+  damping_kernel<<<a.count, 256, 0, s>>>(a);
 }
 
 void launch_colnorm(const float* Y, long long ld, long long mat_stride, int count, int rows, int cols,

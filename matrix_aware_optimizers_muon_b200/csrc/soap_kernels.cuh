@@ -42,8 +42,20 @@ struct SplitArgs {
   long long ldd, mat_stride, plane_stride;
   int nplanes;                     // 1 (bf16 cast), 2 (h, l) or 3 (h, m, l)
   int pad_identity;
+  const float* diag_add = nullptr; // optional [count]: added to the valid diagonal first
 };
 void launch_split(const SplitArgs& a, cudaStream_t s);
+
+// Damping of the power step: delta[b] = rho * trace(F[b]) over the k x k
+// factor F[b] (row stride k), or 1 when that trace is zero.  The trace is
+// summed in a fixed order (per-thread strided sums, then a tree).
+struct DampArgs {
+  int count, k;
+  float rho;
+  const float* F[SOAP_MAXB];
+  float* delta;
+};
+void launch_damping(const DampArgs& a, cudaStream_t s);
 
 // inv_d[b][c] = 1 / ||Y[b][:, c]||_2 over rows < rows (fixed summation order)
 void launch_colnorm(const float* Y, long long ld, long long mat_stride, int count, int rows, int cols,

@@ -39,6 +39,7 @@ def ns_gate(N, O_gpu, O_ref, O_emu, *, tau=1e-2, sub_tol=2e-2, band=(0.6, 1.3), 
     out = dict(k=k, sub=sub, sv_min=float(sv.min()), sv_max=float(sv.max()), full_gpu=full_gpu,
                full_emu=full_emu, tall=tall)
     assert sub <= sub_tol, out
-    assert band[0] <= sv.min() and sv.max() <= band[1], out
+    if band is not None:
+        assert band[0] <= sv.min() and sv.max() <= band[1], out
     assert full_gpu <= floor * full_emu + floor_abs, out
     return out

@@ -117,16 +117,20 @@ def test_ns_rejects_overlap_and_nulls(lib):
 
 def test_soap_rejects_bad_arguments(lib):
     h = _ctx(lib)
-    cfg = _lib.SoapCfg(3e-3, 0.95, 0.95, 0.95, 1e-8, 0.0, 1, None)
+    cfg = _lib.SoapCfg(3e-3, 0.95, 0.95, 0.95, 1e-8, 0.0, 1, None, 0, 1e-5)
     good = _lib.SoapMat(8, 8, 16, 16, 16, 16, 16, 16, None, None)
     mats = (_lib.SoapMat * 1)(good)
     assert lib.soap_step(h, mats, 1, ctypes.byref(cfg), 0, None) == _lib.MO_ERR_INVALID_ARG
     half = _lib.SoapMat(8, 8, 16, 16, 16, 16, 16, None, None, None)
     mats = (_lib.SoapMat * 1)(half)
     assert lib.soap_step(h, mats, 1, ctypes.byref(cfg), 1, None) == _lib.MO_ERR_INVALID_ARG
-    bad_cfg = _lib.SoapCfg(3e-3, 1.0, 0.95, 0.95, 1e-8, 0.0, 1, None)
+    bad_cfg = _lib.SoapCfg(3e-3, 1.0, 0.95, 0.95, 1e-8, 0.0, 1, None, 0, 1e-5)
     mats = (_lib.SoapMat * 1)(good)
     assert lib.soap_step(h, mats, 1, ctypes.byref(bad_cfg), 1, None) == _lib.MO_ERR_INVALID_ARG
+    for damping in (0.0, -1e-5, 0.5, float("nan")):
+        bad_cfg = _lib.SoapCfg(3e-3, 0.95, 0.95, 0.95, 1e-8, 0.0, 1, None, 0, damping)
+        assert lib.soap_step(h, mats, 1, ctypes.byref(bad_cfg), 1, None) == _lib.MO_ERR_INVALID_ARG
+        assert b"damping" in lib.mo_last_error(h)
     lib.mo_ctx_destroy(h)
 
 

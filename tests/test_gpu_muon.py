@@ -194,3 +194,90 @@ def test_ns_matches_muon_direction(ctx):
     Wg, _, _ = run_gpu_muon(ctx, [W], [G], [np.zeros_like(G)], momentum=0.0, lr=1.0, weight_decay=0.0)
     s = 0.2 * np.sqrt(160)
     np.testing.assert_allclose(-Wg[0] / s, O, rtol=0, atol=1e-6)
+
+
+@pytest.mark.parametrize("coeffs,steps,band", [
+    ((1.5, -0.5, 0.0), 5, None),            # classical cubic (Lesson 12, Lemma 3 text)
+    ((2.0, -1.5, 0.5), 12, (0.6, 1.3)),     # exact-at-1 variant run 12 times (mer.dev section 4.3)
+    ((3.4445, -4.7750, 2.0315), 3, None),   # fewer quintic steps
+])
+def test_ns_coefficient_variants(ctx, coeffs, steps, band):
+    mats, factors = wl.cfg5_heads(2, 128, tag="variants")
+    rng = wl.rng_of("variants-wide")
+    Gw = wl.gaussian(rng, (96, 320), 1.0)
+    inputs = [mats[0], Gw]
+    outs = ctx.ns_orthogonalize([_cuda(m) for m in inputs], ns_steps=steps, coeffs=coeffs)
+    for x, o in zip(inputs, outs):
+        ref = ons.newton_schulz(x, coeffs, steps)
+        emu = ons.newton_schulz_bf16(x, coeffs, steps)
+        ns_gate(x, _np(o), ref, emu, band=band)
+
+
+# ------------------------------------------------ fused small-matrix kernel
+
+@pytest.mark.parametrize("shapes", [
+    [(64, 200)] * 170 + [(200, 64)] * 130,    # one bucket, both orientations, > 148 per launch
+    [(128, 256), (256, 128), (128, 128)],     # the largest shapes the fused kernel takes
+    [(1, 1), (5, 250), (33, 100), (100, 33), (127, 255)],   # ragged tails
+])
+def test_small_fused_batches(ctx, shapes):
+    rng = wl.rng_of("small-fused", len(shapes), shapes[0])
+    Ws = [wl.weights(rng, m, n) for m, n in shapes]
+    Gs = [wl.gaussian(rng, (m, n), 1e-3) for m, n in shapes]
+    Bs = [wl.gaussian(rng, (m, n), 1e-3) for m, n in shapes]
+    Wg, Bg, flags = run_gpu_muon(ctx, Ws, Gs, Bs)
+    assert (flags == 0).all()
+    pick = sorted(set([0, len(shapes) - 1, len(shapes) // 2, 149 % len(shapes), 171 % len(shapes)]))
+    for i in pick:
+        check_muon(Ws[i], Gs[i], Bs[i], Wg[i], Bg[i])
+    Wr, Br, _ = run_gpu_muon(ctx, Ws, Gs, Bs)
+    for i in pick:
+        np.testing.assert_array_equal(Wr[i], Wg[i])   # bitwise repeatable
+
+
+@pytest.mark.parametrize("kw", [dict(nesterov=False), dict(momentum_ema=True), dict(ns_steps=3),
+                                dict(adjust_lr="original")])
+def test_small_fused_options(ctx, kw):
+    rng = wl.rng_of("small-options", str(kw))
+    shapes = [(96, 160), (160, 96)]
+    Ws = [wl.weights(rng, m, n) for m, n in shapes]
+    Gs = [wl.gaussian(rng, (m, n), 1e-3) for m, n in shapes]
+    Bs = [wl.gaussian(rng, (m, n), 1e-3) for m, n in shapes]
+    Wg, Bg, _ = run_gpu_muon(ctx, Ws, Gs, Bs, **kw)
+    for i in range(2):
+        check_muon(Ws[i], Gs[i], Bs[i], Wg[i], Bg[i], **kw)
+
+
+def test_cuda_graph_replay_matches_eager(ctx):
+    """A Muon step over both paths (batched GEMMs and the fused small-matrix
+    kernel) captured in a CUDA graph gives bitwise the eager result."""
+    import torch
+    rng = wl.rng_of("graph")
+    shapes = [(64, 200), (200, 64), (256, 320), (320, 256)]
+    Ws = [wl.weights(rng, m, n) for m, n in shapes]
+    Gs = [wl.gaussian(rng, (m, n), 1e-3) for m, n in shapes]
+    Bs = [wl.gaussian(rng, (m, n), 1e-3) for m, n in shapes]
+    We, Be, _ = run_gpu_muon(ctx, Ws, Gs, Bs)
+    W = [_cuda(w) for w in Ws]
+    G = [_cuda(g) for g in Gs]
+    B = [_cuda(b) for b in Bs]
+    ctx.reserve(0, shapes)
+    step = lambda: ctx.muon_step(W, G, B, reserve=False)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()                                     # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for w, b, w0, b0 in zip(W, B, Ws, Bs):         # reset the state, then replay once
+        w.copy_(_cuda(w0))
+        b.copy_(_cuda(b0))
+    graph.replay()
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    for i in range(len(shapes)):
+        np.testing.assert_array_equal(_np(W[i]), We[i])
+        np.testing.assert_array_equal(_np(B[i]), Be[i])
+    del graph

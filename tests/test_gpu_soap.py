@@ -42,11 +42,11 @@ def warm_state(m, n, left, right, steps, tag, cfg=wl.CFG4_MINI):
     return f32, st.next(), steps + 1
 
 
-def run_gpu(ctx, S, G, t, flags=None):
+def run_gpu(ctx, S, G, t, flags=None, refresh=True):
     import torch
     d = {k: _cuda(v) for k, v in S.items()}
     d["G"] = _cuda(G)
-    ctx.soap_step([d], t, nonfinite=flags, **HP)
+    ctx.soap_step([d], t, nonfinite=flags, refresh=refresh, **HP)
     torch.cuda.synchronize()
     assert ctx.device_status() == 0
     return {k: _np(v) for k, v in d.items() if k != "G"}
@@ -105,9 +105,10 @@ def test_identity_bases_is_adamw(ctx):
 
 
 def test_cold_start_properties(ctx):
-    """Step 1 from zero state: L_1 is ill-conditioned (kappa ~ 1e4), so the
-    basis is compared by its defining properties: orthonormal, and Q^T Y
-    upper triangular with a positive diagonal (Y = L_1 Q_0 = L_1)."""
+    """Step 1 from zero state: L_1 is ill-conditioned (kappa ~ 1e4); the basis
+    is checked by its defining properties (orthonormal, Q^T Y upper
+    triangular with a positive diagonal, Y = (L_1 + d I) Q_0) and against the
+    damped fp64 power step."""
     import torch
     m, n = 256, 896
     st = wl.SpikeStream("soap-cold", "x", 0, m, n, wl.CFG4_MINI)
@@ -119,9 +120,12 @@ def test_cold_start_properties(ctx):
     assert int(flags.item()) == 0
     Q, L1 = out["QL"], out["L"]
     assert np.abs(Q.T @ Q - np.eye(m)).max() <= 1e-4
-    R = Q.T @ L1
+    Y = L1 + osoap.damping_of(L1, 1e-5) * np.eye(m)
+    R = Q.T @ Y
     assert np.abs(np.tril(R, -1)).max() <= 1e-4 * np.abs(R).max()
     assert (np.diag(R) > 0).all()
+    from oracle.qr import qr_positive
+    assert rel(Q, qr_positive(Y)[0]) <= 5e-3
     # first Adam step is a sign-like step: |Dbar| ~ 1 entrywise
     dW = out["W"] - S["W"]
     ratio = np.linalg.norm(dW) / (HP["lr"] * np.sqrt(m * n))
@@ -140,3 +144,99 @@ def test_skip_leaves_state(ctx):
     torch.cuda.synchronize()
     np.testing.assert_array_equal(_np(d["W"]), S["W"])
     np.testing.assert_array_equal(_np(d["QL"]), S["QL"])
+
+
+@pytest.mark.parametrize("m,n,left,right", [(256, 256, True, True), (256, 896, True, False)])
+def test_stale_basis_step(ctx, m, n, left, right):
+    """A step between two refreshes: factors update, bases are kept."""
+    S, G, t = warm_state(m, n, left, right, 10, "soap-stale")
+    out = run_gpu(ctx, S, G, t, refresh=False)
+    args = (S["W"], G, S["M"], S["V"], S["L"], S["QL"], S["R"], S["QR"])
+    ref = osoap.soap_step(*args, t=t, basis_refresh=False, **HP)
+    emu = osoap.soap_step(*args, t=t, basis_refresh=False, precision="bf16", **HP)
+    np.testing.assert_array_equal(out["QL"], S["QL"])
+    assert rel(out["L"], emu["L"]) <= 1e-4
+    dW = out["W"] - S["W"].astype(np.float64)
+    assert rel(dW, emu["dW"]) <= 1e-2
+    assert rel(dW, ref["dW"]) <= 2e-2
+
+
+def test_cold_start_square_two_sided(ctx):
+    """Steps 1-3 from zero state with both factors square (the factors are
+    nearly singular at step 1: a rank-8 spike over a square Gaussian); each
+    GPU step is checked against the oracle run from the GPU's own state."""
+    import torch
+    m = n = 512
+    st = wl.SpikeStream("soap-cold-sq", "x", 0, m, n, wl.CFG4_MINI)
+    S = dict(W=st.W, M=np.zeros((m, n), np.float32), V=np.zeros((m, n), np.float32),
+             L=np.zeros((m, m), np.float32), QL=np.eye(m, dtype=np.float32),
+             R=np.zeros((n, n), np.float32), QR=np.eye(n, dtype=np.float32))
+    for t in (1, 2, 3):
+        G = st.next()
+        flags = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+        out = run_gpu(ctx, S, G, t, flags)
+        assert int(flags.item()) == 0, t
+        emu = osoap.soap_step(S["W"], G, S["M"], S["V"], S["L"], S["QL"], S["R"], S["QR"], t=t,
+                              precision="bf16", **HP)
+        for q in ("QL", "QR"):
+            Q = out[q]
+            assert np.abs(Q.T @ Q - np.eye(m)).max() <= 1e-4, (t, q)
+            assert rel(Q, emu[q]) <= 5e-3, (t, q, rel(Q, emu[q]))
+        dW = out["W"] - S["W"]
+        if t == 1:
+            # Dbar = M' / |G'| is sign-like at step 1: entries where G' is at
+            # rounding level differ in sign, so only the update's size is
+            # compared.  M' and G' are rotated separately, so where G' is tiny
+            # |Dbar| exceeds 1 in the bf16-operand emulation as well (there by
+            # 0.13 %); the GPU's size is gated against the emulation's.
+            ratio = np.linalg.norm(dW) / (HP["lr"] * np.sqrt(m * n))
+            ratio_emu = np.linalg.norm(emu["dW"]) / (HP["lr"] * np.sqrt(m * n))
+            assert abs(ratio - ratio_emu) <= 2e-3, (ratio, ratio_emu)
+        else:
+            assert rel(dW, emu["dW"]) <= 2e-2, (t, rel(dW, emu["dW"]))
+        S = {k: out[k].astype(np.float32) for k in S}
+
+
+def test_rank_one_and_zero_gradients(ctx):
+    """A rank-one gradient (factor of rank one at step 1) and an all-zero
+    gradient (zero factor: the basis is kept) in one call."""
+    import torch
+    m, n = 256, 384
+    rng = wl.rng_of("soap-rank1")
+    u = rng.standard_normal((m, 1))
+    v = rng.standard_normal((1, n))
+    grads = [(u @ v * 1e-3).astype(np.float32), np.zeros((m, n), np.float32)]
+    states = []
+    for i in range(2):
+        QL, _ = np.linalg.qr(rng.standard_normal((m, m)))
+        states.append(dict(W=wl.weights(rng, m, n), M=np.zeros((m, n), np.float32),
+                           V=np.zeros((m, n), np.float32), L=np.zeros((m, m), np.float32),
+                           QL=QL.astype(np.float32), R=np.zeros((n, n), np.float32),
+                           QR=np.eye(n, dtype=np.float32)))
+    ds = []
+    for S, G in zip(states, grads):
+        d = {k: _cuda(v) for k, v in S.items()}
+        d["G"] = _cuda(G)
+        ds.append(d)
+    flags = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    ctx.soap_step(ds, 1, nonfinite=flags, **HP)
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    assert (flags.cpu().numpy() == 0).all()
+    for S, G, d in zip(states, grads, ds):
+        out = {k: _np(v) for k, v in d.items() if k != "G"}
+        emu = osoap.soap_step(S["W"], G, S["M"], S["V"], S["L"], S["QL"], S["R"], S["QR"], t=1,
+                              precision="bf16", **HP)
+        for q in ("QL", "QR"):
+            assert np.abs(out[q].T @ out[q] - np.eye(out[q].shape[0])).max() <= 1e-4
+            assert rel(out[q], emu[q]) <= 5e-3, (q, rel(out[q], emu[q]))
+        if not G.any():
+            assert np.abs(out["QL"] - S["QL"]).max() <= 1e-5     # zero factor keeps its basis
+            np.testing.assert_array_equal(out["W"], S["W"])      # zero step, no decay
+        else:
+            # the resolved direction: the first left basis vector is +-u / |u|;
+            # the rest of G' is at rounding level, where the sign-like first
+            # Adam step is not determined, so dW is only checked to be finite
+            c = abs(float(out["QL"][:, 0] @ u[:, 0])) / np.linalg.norm(u)
+            assert c >= 1 - 1e-6
+            assert np.isfinite(out["W"]).all()

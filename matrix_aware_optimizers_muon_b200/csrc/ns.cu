@@ -108,12 +108,17 @@ cudaError_t ns_run(const std::vector<NsItem>& items, const NsCall& call, char* w
         }
         const int n = (int)in.size();
         if (n == 0) continue;
+        bool vec = cols % 4 == 0;
+        for (int j = 0; j < n && vec; ++j) {
+          auto al16 = [](const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+          vec = al16(in[j]) && al16(out[j]) && (!call.muon || al16(mom[j]));
+        }
         launch_upload_tables(tab, n, in.data(), mom.data(), out.data(), flg.data(), stream);
         SmallArgs sa;
         sa.count = n; sa.rows = (int)rows; sa.cols = (int)cols; sa.tall = pass;
         sa.mode = call.muon ? 1 : 0;
         sa.beta = call.beta; sa.nesterov = call.nesterov; sa.ema = call.ema;
-        sa.steps = call.steps; sa.a = call.a; sa.b = call.b; sa.c = call.c; sa.eps = call.eps;
+        sa.steps = call.steps; sa.vec = vec ? 1 : 0; sa.a = call.a; sa.b = call.b; sa.c = call.c; sa.eps = call.eps;
         const double m = (double)rows, nn = (double)cols;
         const double scale = call.adjust_lr == 0 ? 0.2 * std::sqrt(std::max(m, nn)) : std::sqrt(std::max(1.0, m / nn));
         sa.decay = (float)(1.0 - (double)call.lr * (double)call.wd);
@@ -123,8 +128,7 @@ cudaError_t ns_run(const std::vector<NsItem>& items, const NsCall& call, char* w
         sa.out = reinterpret_cast<float* const*>(tab + 2 * n);
         sa.flag = reinterpret_cast<int32_t* const*>(tab + 3 * n);
         sa.status = status;
-        const int grid = std::min(n, device_sm_count());
-        cudaError_t e = launch_ns_small(sa, grid, stream);
+        cudaError_t e = launch_ns_small(sa, device_sm_count(), stream);
         if (e != cudaSuccess) return e;
         // the next launch may reuse the tables only after this one is done
         // reading them; both run on one stream, so stream order suffices

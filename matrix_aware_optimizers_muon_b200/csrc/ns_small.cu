@@ -23,10 +23,12 @@ namespace {
 
 constexpr int SM_THREADS = 160;
 constexpr int CHUNK = 128 * 128;                 // bytes of one 64-column chunk of 128 rows
-constexpr int X_BYTES = 4 * CHUNK;               // up to 256 columns
 constexpr int A_BYTES = 2 * CHUNK;               // 128 x 128
-constexpr int SMEM_BYTES = X_BYTES + 2 * A_BYTES + 1024 + 256;
 constexpr uint32_t TMEM_COLS = 256;
+constexpr int VU = 8;                            // float4 accesses in flight per thread
+
+// X holds npad / 64 chunks; with npad <= 128 two CTAs fit on one SM.
+constexpr int smem_bytes(int npad) { return (npad / 64) * CHUNK + 2 * A_BYTES + 1024 + 256; }
 
 // byte offset of element (r, c) inside a swizzled chunked tile
 __device__ __forceinline__ uint32_t swz(int r, int c) {
@@ -75,11 +77,14 @@ __device__ __forceinline__ void load_unit(const uint8_t* tile, int r, int u, flo
   }
 }
 
-__global__ void __launch_bounds__(SM_THREADS, 1) ns_small_kernel(const SmallArgs a) {
+__global__ void __launch_bounds__(SM_THREADS, 2) ns_small_kernel(const SmallArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int np = a.tall ? a.rows : a.cols;      // oriented cols (<= 256)
+  const int npad = (np + 63) & ~63;             // K of the Gram, N of the update
+  const int xbytes = (npad >> 6) * CHUNK;
   uint8_t* X = smem;
-  uint8_t* A = smem + X_BYTES;
+  uint8_t* A = smem + xbytes;
   uint8_t* P = A + A_BYTES;
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(P + A_BYTES);
   uint64_t* work_bar = mma_bar + 1;
@@ -89,8 +94,6 @@ __global__ void __launch_bounds__(SM_THREADS, 1) ns_small_kernel(const SmallArgs
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
-  const int np = a.tall ? a.rows : a.cols;      // oriented cols (<= 256)
-  const int npad = (np + 63) & ~63;             // K of the Gram, N of the update
   const uint32_t idesc_g = idesc_bf16_f32(128, 128, 0, 0);
   const uint32_t idesc_u = idesc_bf16_f32(128, npad, 0, 1);
 
@@ -116,25 +119,75 @@ __global__ void __launch_bounds__(SM_THREADS, 1) ns_small_kernel(const SmallArgs
   for (int mat = blockIdx.x; mat < a.count && ok; mat += gridDim.x) {
     if (warp < 4) {
       // ---- load: momentum, Nesterov, bf16 cast into X (oriented), norm
-      for (int e = tid; e < X_BYTES / 16; e += 128) reinterpret_cast<uint4*>(X)[e] = make_uint4(0, 0, 0, 0);
+      for (int e = tid; e < xbytes / 16; e += 128) reinterpret_cast<uint4*>(X)[e] = make_uint4(0, 0, 0, 0);
       __syncwarp();
       asm volatile("bar.sync 1, 128;" ::: "memory");
       const float* G = a.in[mat];
       float* B = a.mom ? a.mom[mat] : nullptr;
       const int total = a.rows * a.cols;
       float ss = 0.f;
-      for (int e = tid; e < total; e += 128) {
-        const int r = e / a.cols, c = e - r * a.cols;
-        const float g = G[e];
-        float n = g;
-        if (a.mode == 1) {
-          const float bn = a.ema ? fmaf(a.beta, B[e], (1.0f - a.beta) * g) : fmaf(a.beta, B[e], g);
-          B[e] = bn;
-          n = a.nesterov ? fmaf(a.beta, bn, g) : bn;
+      if (a.vec) {
+        // float4 accesses, VU in flight per thread (cols % 4 == 0, 16-byte
+        // aligned matrices): four consecutive columns of one row each
+        const float4* G4 = reinterpret_cast<const float4*>(G);
+        float4* B4 = reinterpret_cast<float4*>(B);
+        const int total4 = total >> 2;
+        for (int e0 = tid; e0 < total4; e0 += 128 * VU) {
+          float4 g[VU], b[VU];
+#pragma unroll
+          for (int u = 0; u < VU; ++u) {
+            const int e = e0 + u * 128;
+            if (e < total4) {
+              g[u] = __ldg(G4 + e);
+              if (a.mode == 1) b[u] = B4[e];
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < VU; ++u) {
+            const int e = e0 + u * 128;
+            if (e >= total4) break;
+            float gv[4] = {g[u].x, g[u].y, g[u].z, g[u].w}, nv[4];
+            float bv[4] = {0.f, 0.f, 0.f, 0.f};
+            if (a.mode == 1) { bv[0] = b[u].x; bv[1] = b[u].y; bv[2] = b[u].z; bv[3] = b[u].w; }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float n = gv[j];
+              if (a.mode == 1) {
+                const float bn = a.ema ? fmaf(a.beta, bv[j], (1.0f - a.beta) * gv[j]) : fmaf(a.beta, bv[j], gv[j]);
+                bv[j] = bn;
+                n = a.nesterov ? fmaf(a.beta, bn, gv[j]) : bn;
+              }
+              nv[j] = n;
+              ss = fmaf(n, n, ss);
+            }
+            if (a.mode == 1) B4[e] = make_float4(bv[0], bv[1], bv[2], bv[3]);
+            const int r = (4 * e) / a.cols, c = 4 * e - r * a.cols;
+            if (!a.tall) {
+              const __nv_bfloat162 lo = __floats2bfloat162_rn(nv[0], nv[1]);
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(nv[2], nv[3]);
+              *reinterpret_cast<uint2*>(X + swz(r, c)) =
+                  make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<__nv_bfloat16*>(X + swz(c + j, r)) = __float2bfloat16_rn(nv[j]);
+            }
+          }
         }
-        ss = fmaf(n, n, ss);
-        const int xr = a.tall ? c : r, xc = a.tall ? r : c;
-        *reinterpret_cast<__nv_bfloat16*>(X + swz(xr, xc)) = __float2bfloat16_rn(n);
+      } else {
+        for (int e = tid; e < total; e += 128) {
+          const int r = e / a.cols, c = e - r * a.cols;
+          const float g = G[e];
+          float n = g;
+          if (a.mode == 1) {
+            const float bn = a.ema ? fmaf(a.beta, B[e], (1.0f - a.beta) * g) : fmaf(a.beta, B[e], g);
+            B[e] = bn;
+            n = a.nesterov ? fmaf(a.beta, bn, g) : bn;
+          }
+          ss = fmaf(n, n, ss);
+          const int xr = a.tall ? c : r, xc = a.tall ? r : c;
+          *reinterpret_cast<__nv_bfloat16*>(X + swz(xr, xc)) = __float2bfloat16_rn(n);
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -224,11 +277,46 @@ __global__ void __launch_bounds__(SM_THREADS, 1) ns_small_kernel(const SmallArgs
       if (ok) {
         asm volatile("bar.sync 1, 128;" ::: "memory");
         float* out = a.out[mat];
-        for (int e = tid; e < total; e += 128) {
-          const int rr = e / a.cols, c = e - rr * a.cols;
-          const int xr = a.tall ? c : rr, xc = a.tall ? rr : c;
-          const float o = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(X + swz(xr, xc)));
-          out[e] = a.mode == 1 ? fmaf(a.decay, out[e], -a.step * o) : o;
+        if (a.vec) {
+          float4* O4 = reinterpret_cast<float4*>(out);
+          const int total4 = total >> 2;
+          for (int e0 = tid; e0 < total4; e0 += 128 * VU) {
+            float4 w[VU];
+            if (a.mode == 1) {
+#pragma unroll
+              for (int u = 0; u < VU; ++u)
+                if (e0 + u * 128 < total4) w[u] = O4[e0 + u * 128];
+            }
+#pragma unroll
+            for (int u = 0; u < VU; ++u) {
+              const int e = e0 + u * 128;
+              if (e >= total4) break;
+              const int r = (4 * e) / a.cols, c = 4 * e - r * a.cols;
+              float o[4];
+              if (!a.tall) {
+                const uint2 v = *reinterpret_cast<const uint2*>(X + swz(r, c));
+                const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+                const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+                o[0] = lo.x; o[1] = lo.y; o[2] = hi.x; o[3] = hi.y;
+              } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  o[j] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(X + swz(c + j, r)));
+              }
+              if (a.mode == 1)
+                O4[e] = make_float4(fmaf(a.decay, w[u].x, -a.step * o[0]), fmaf(a.decay, w[u].y, -a.step * o[1]),
+                                    fmaf(a.decay, w[u].z, -a.step * o[2]), fmaf(a.decay, w[u].w, -a.step * o[3]));
+              else
+                O4[e] = make_float4(o[0], o[1], o[2], o[3]);
+            }
+          }
+        } else {
+          for (int e = tid; e < total; e += 128) {
+            const int rr = e / a.cols, c = e - rr * a.cols;
+            const int xr = a.tall ? c : rr, xc = a.tall ? rr : c;
+            const float o = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(X + swz(xr, xc)));
+            out[e] = a.mode == 1 ? fmaf(a.decay, out[e], -a.step * o) : o;
+          }
         }
       }
     } else if (lane == 0) {
@@ -310,17 +398,25 @@ void launch_upload_tables(void** dst, int n, const void* const* in, const void* 
   }
 }
 
-cudaError_t launch_ns_small(const SmallArgs& a, int grid, cudaStream_t s) {
+cudaError_t launch_ns_small(const SmallArgs& a, int sm_count, cudaStream_t s) {
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem_bytes(SMALL_MAX_N));
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
+  const int np = a.tall ? a.rows : a.cols;
+  const int npad = (np + 63) & ~63;
+  const int smem = smem_bytes(npad);
+  // two CTAs per SM when both fit in shared memory (one's loads and stores
+  // then overlap the other's tensor-core phases)
+  const int per_sm = 2 * (smem + 1024) <= 228 * 1024 ? 2 : 1;
+  const int grid = a.count < per_sm * sm_count ? a.count : per_sm * sm_count;
   ProfScope prof(PK_SMALL, s, 0.0);
-  ns_small_kernel<<<grid, SM_THREADS, SMEM_BYTES, s>>>(a);
+  ns_small_kernel<<<grid, SM_THREADS, smem, s>>>(a);
   return cudaGetLastError();
 }
 

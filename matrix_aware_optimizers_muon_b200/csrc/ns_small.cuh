@@ -17,6 +17,7 @@ struct SmallArgs {
   float beta;
   int nesterov, ema;
   int steps;
+  int vec;                    // 1: cols % 4 == 0 and every matrix 16-byte aligned
   float a, b, c, eps;
   float decay, step;
   const float* const* in;     // device tables of `count` pointers
@@ -31,6 +32,7 @@ struct SmallArgs {
 void launch_upload_tables(void** dst, int n, const void* const* in, const void* const* mom,
                           const void* const* out, const void* const* flag, cudaStream_t s);
 
-cudaError_t launch_ns_small(const SmallArgs& a, int grid, cudaStream_t s);
+// One persistent launch over all matrices (grid: up to two CTAs per SM).
+cudaError_t launch_ns_small(const SmallArgs& a, int sm_count, cudaStream_t s);
 
 }  // namespace mo

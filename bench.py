@@ -116,6 +116,18 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(x, world, device="cpu"):
+    """The largest of each rank's x (every rank gets it): a multi-GPU step
+    takes as long as its slowest replica."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -250,10 +262,7 @@ def run_ours(args, world, rank, local):
     prof = ctx.profile_read()
     ctx.profile(False)
     status = ctx.device_status()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
 
     gemm_ms = sum(prof[k][0] for k in ("gram", "poly", "update"))
     gemm_exec = sum(prof[k][1] for k in ("gram", "poly", "update"))
@@ -487,16 +496,38 @@ def extras(ctx, dev, args):
     # single 256 x 512 Muon step (latency)
     W, G, B = (torch.from_numpy(x).to(dev) for x in wl.cfg1())
     ctx.reserve(0, [(256, 512)])
-    ms = time_steps(lambda: ctx.muon_step([W], [G], [B], reserve=False), 50, 5)
+    call = lambda: ctx.muon_step([W], [G], [B], reserve=False)
+    ms_eager = time_steps(call, 50, 5)
+    graph = capture_graph(call)
+    ms = time_steps(graph.replay, 50, 5)
+    del graph
     res["muon_256x512_us"] = round(ms * 1e3, 1)
+    res["muon_256x512_eager_call_us"] = round(ms_eager * 1e3, 1)
     ctx.workspace = None
     # MoE experts, grouped
     Ws, Gs, Bs, shapes = moe_workload(dev)
     ctx.reserve(0, shapes)
-    ms = time_steps(lambda: ctx.muon_step(Ws, Gs, Bs, reserve=False), 5, 2)
+    call = lambda: ctx.muon_step(Ws, Gs, Bs, reserve=False)
+    ms_eager = time_steps(call, 5, 2)
+    graph = capture_graph(call)
+    ms = time_steps(graph.replay, 5, 2)
+    del graph
+    ctx.profile(True)
+    ctx.profile_read()
+    call()
+    torch.cuda.synchronize()
+    prof = ctx.profile_read()
+    ctx.profile(False)
     fl = sum(page_flops(m, n) for m, n in shapes)
-    res["muon_moe_1536x768x2048"] = {"ms": round(ms, 3), "TFLOP/s": round(fl / (ms / 1e3) / 1e12, 1),
-                                     "matrices_per_s": round(len(shapes) / (ms / 1e3), 1)}
+    gemm = [k for k in ("gram", "poly", "update")]
+    g_ms = sum(prof[k][0] for k in gemm)
+    g_fl = sum(prof[k][1] for k in gemm)
+    res["muon_moe_1536x768x2048"] = {
+        "ms": round(ms, 3), "TFLOP/s": round(fl / (ms / 1e3) / 1e12, 1),
+        "matrices_per_s": round(len(shapes) / (ms / 1e3), 1), "eager_call_ms": round(ms_eager, 3),
+        "kernels_ms": {k: round(v[0], 3) for k, v in prof.items() if v[2]},
+        "gemm_executed_TFLOP/s": round(g_fl / (g_ms / 1e3) / 1e12, 1) if g_ms else None,
+        "note": "ms: CUDA-graph replay of the whole step; kernels_ms from one eager step"}
     del Ws, Gs, Bs
     ctx.workspace = None
     torch.cuda.empty_cache()

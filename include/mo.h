@@ -233,6 +233,61 @@ MO_API mo_status soap_step(mo_ctx* ctx, const mo_soap_mat* mats /* host array */
  * Only rows, cols, L and R are read; no pointer is dereferenced. */
 MO_API mo_status mo_soap_workspace_bytes(mo_ctx* ctx, const mo_soap_mat* mats, int n, size_t* bytes);
 
+/* ------------------------------------------------------------------ SOAP-Muon
+ * SOAP preconditions the Muon momentum with the bases of the previous step,
+ * Newton-Schulz orthogonalises the result and Muon's update applies it; the
+ * factors then take the raw gradient and the bases are refreshed for the
+ * next step ("初探优化器（一）：从SGD到SOAP-Muon", sections 7.1-7.2; the
+ * section's formula was lost, these steps are the plainest reading of its
+ * implementation notes).  At step t >= 1:
+ *   B <- mu B + G,  N = G + mu B (nesterov) or B
+ *   N' = Q_L^T N Q_R,  G' = Q_L^T G Q_R          (bases as passed in)
+ *   V <- b2 V + (1 - b2) G' * G'
+ *   P = Q_L [N' / (sqrt(V / (1 - b2^t)) + eps)] Q_R^T
+ *   O = NS(P)   (quintic Newton-Schulz as in ns_orthogonalize; its Frobenius
+ *                normalisation is the rescaling)
+ *   W <- (1 - lr wd) W - lr s O   (s as in muon_step's adjust_lr)
+ *   L <- bs L + (1 - bs) G G^T,  R likewise;  Q <- qr((F + d I) Q) as in
+ *   soap_step (skipped with skip_refresh)
+ * Sides, layout, alignment and shape rules are those of soap_step (rows and
+ * cols multiples of 8, 16-byte aligned pointers, factor sides <= 16384).
+ * Precision: rotations two-plane bf16, P fp32, NS bf16 operands as in
+ * muon_step, the refresh fp32-accurate.  Initial state: B = V = L = R = 0,
+ * Q = I.  nonfinite[i] is 1 if P was not finite or the QR met a
+ * non-positive pivot. */
+typedef struct {
+  int64_t rows, cols;
+  float* W;
+  const float* G;       /* NULL skips this matrix */
+  float* B;             /* Muon momentum, m x n */
+  float* V;             /* second moment in the rotated basis, m x n */
+  float* L;             /* m x m factor, or NULL (identity left basis) */
+  float* QL;            /* m x m basis, or NULL */
+  float* R;             /* n x n factor, or NULL (identity right basis) */
+  float* QR;            /* n x n basis, or NULL */
+} mo_soap_muon_mat;
+
+typedef struct {
+  float lr, weight_decay, momentum;
+  int nesterov;
+  float beta2;          /* V's beta */
+  float shampoo_beta;   /* factor EMA (0.9 in the records the pages describe) */
+  float eps;            /* Adam epsilon, outside the square root */
+  int bias_correction;  /* 1: V / (1 - b2^t) */
+  int ns_steps; float a, b, c, ns_eps;
+  int adjust_lr;        /* 0: 0.2 sqrt(max(m, n)); 1: sqrt(max(1, m / n)) */
+  float damping;        /* relative damping of the power step, (0, 1e-2] */
+  int32_t* nonfinite;   /* optional device int32[n] */
+  int skip_refresh;     /* 1: keep the bases (factors still update) */
+} mo_soap_muon_cfg;
+
+MO_API mo_status soap_muon_step(mo_ctx* ctx, const mo_soap_muon_mat* mats /* host array */, int n,
+                                const mo_soap_muon_cfg* cfg, int64_t step, void* stream);
+
+/* Exact workspace of soap_muon_step for these matrices (sides as given). */
+MO_API mo_status mo_soap_muon_workspace_bytes(mo_ctx* ctx, const mo_soap_muon_mat* mats, int n,
+                                              size_t* bytes);
+
 /* ------------------------------------------------------------------ building block
  * The batched tensor-core GEMM the steps are built from, exposed for tests
  * and for callers composing their own variants:

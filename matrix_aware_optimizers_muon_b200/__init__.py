@@ -11,8 +11,8 @@ import ctypes
 from ctypes import byref, c_int32, c_int64, c_size_t, c_void_p
 
 from . import _lib
-from ._lib import (GemmDesc, MuonCfg, MuonMat, NsCfg, SoapCfg, SoapMat, OP_MUON, OP_NS,
-                   OP_SOAP)
+from ._lib import (GemmDesc, MuonCfg, MuonMat, NsCfg, SoapCfg, SoapMat, SoapMuonCfg, SoapMuonMat,
+                   OP_MUON, OP_NS, OP_SOAP)
 
 __all__ = ["Context", "MoError", "QUINTIC", "OP_MUON", "OP_SOAP", "OP_NS"]
 
@@ -188,6 +188,33 @@ class Context:
         cfg = SoapCfg(lr, beta1, beta2, sb, eps, weight_decay, int(bias_correction), _ptr(nonfinite),
                       0 if refresh else 1, damping)
         self._check(self.lib.soap_step(self.handle, arr, n, byref(cfg), int(step), self._stream(stream)))
+
+    def soap_muon_step(self, mats, step, *, lr=0.02, weight_decay=0.01, momentum=0.95, nesterov=True,
+                       beta2=0.95, shampoo_beta=0.9, eps=1e-8, bias_correction=True, ns_steps=5,
+                       coeffs=QUINTIC, ns_eps=1e-7, adjust_lr="match_rms_adamw", damping=1e-5,
+                       nonfinite=None, refresh=True, stream=None, reserve=True):
+        """One SOAP-Muon step.  ``mats``: dicts with W, G, B (Muon momentum), V
+        and optionally L, QL, R, QR (missing or None: identity basis)."""
+        n = len(mats)
+        arr = (SoapMuonMat * max(n, 1))()
+        for i, d in enumerate(mats):
+            for k in ("W", "G", "B", "V", "L", "QL", "R", "QR"):
+                _check_f32(d.get(k), f"{k}[{i}]")
+            W = d["W"]
+            arr[i] = SoapMuonMat(W.shape[0], W.shape[1], _ptr(W), _ptr(d.get("G")), _ptr(d["B"]),
+                                 _ptr(d["V"]), _ptr(d.get("L")), _ptr(d.get("QL")), _ptr(d.get("R")),
+                                 _ptr(d.get("QR")))
+        if reserve:
+            need = c_size_t()
+            self._check(self.lib.mo_soap_muon_workspace_bytes(self.handle, arr, n, byref(need)))
+            if self.workspace is None or self.workspace.numel() < need.value:
+                self.attach_workspace(need.value, stream)
+        modes = {"match_rms_adamw": 0, "original": 1}
+        cfg = SoapMuonCfg(lr, weight_decay, momentum, int(nesterov), beta2, shampoo_beta, eps,
+                          int(bias_correction), ns_steps, coeffs[0], coeffs[1], coeffs[2], ns_eps,
+                          modes[adjust_lr], damping, _ptr(nonfinite), 0 if refresh else 1)
+        self._check(self.lib.soap_muon_step(self.handle, arr, n, byref(cfg), int(step),
+                                            self._stream(stream)))
 
     def gemm_bf16(self, A, B, D, *, M, N, K, batch=1, a_mn=False, b_mn=False, sym=False,
                   alpha=1.0, beta=0.0, C=None, scale=None, alpha_pow=0, beta_pow=0,

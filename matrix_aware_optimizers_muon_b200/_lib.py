@@ -55,6 +55,21 @@ class SoapCfg(ctypes.Structure):
                 ("damping", c_float)]
 
 
+class SoapMuonMat(ctypes.Structure):
+    _fields_ = [("rows", c_int64), ("cols", c_int64), ("W", c_void_p), ("G", c_void_p),
+                ("B", c_void_p), ("V", c_void_p), ("L", c_void_p), ("QL", c_void_p),
+                ("R", c_void_p), ("QR", c_void_p)]
+
+
+class SoapMuonCfg(ctypes.Structure):
+    _fields_ = [("lr", c_float), ("weight_decay", c_float), ("momentum", c_float),
+                ("nesterov", c_int), ("beta2", c_float), ("shampoo_beta", c_float),
+                ("eps", c_float), ("bias_correction", c_int), ("ns_steps", c_int),
+                ("a", c_float), ("b", c_float), ("c", c_float), ("ns_eps", c_float),
+                ("adjust_lr", c_int), ("damping", c_float), ("nonfinite", c_void_p),
+                ("skip_refresh", c_int)]
+
+
 class GemmDesc(ctypes.Structure):
     _fields_ = [("A", c_void_p), ("lda", c_int64), ("strideA", c_int64), ("a_mn", c_int),
                 ("B", c_void_p), ("ldb", c_int64), ("strideB", c_int64), ("b_mn", c_int),
@@ -81,6 +96,10 @@ SIGNATURES = {
     "soap_step": (c_int, [c_void_p, POINTER(SoapMat), c_int, POINTER(SoapCfg), c_int64, c_void_p]),
     "mo_gemm_bf16": (c_int, [c_void_p, POINTER(GemmDesc), c_void_p]),
     "mo_soap_workspace_bytes": (c_int, [c_void_p, POINTER(SoapMat), c_int, POINTER(c_size_t)]),
+    "soap_muon_step": (c_int, [c_void_p, POINTER(SoapMuonMat), c_int, POINTER(SoapMuonCfg), c_int64,
+                               c_void_p]),
+    "mo_soap_muon_workspace_bytes": (c_int, [c_void_p, POINTER(SoapMuonMat), c_int,
+                                             POINTER(c_size_t)]),
     "ns_orthogonalize_static": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64,
                                         POINTER(NsCfg), c_void_p]),
     "mo_profile_enable": (c_int, [c_void_p, c_int]),

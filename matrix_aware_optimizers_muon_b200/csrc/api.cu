@@ -275,6 +275,64 @@ mo_status ns_orthogonalize(mo_ctx* ctx, const float* const* in, float* const* ou
 
 // ---------------------------------------------------------------- SOAP
 
+namespace {
+
+// Validation and launch shared by soap_step and soap_muon_step (ext != null;
+// then M is the Muon momentum B).
+mo_status soap_impl(mo_ctx* ctx, const mo_soap_mat* mats, int n, const mo_soap_cfg* cfg, int64_t step,
+                    void* stream, const mo::SoapMuonExt* ext) {
+  const std::string fn = ext ? "soap_muon_step" : "soap_step";
+  if (step < 1) return fail(ctx, MO_ERR_INVALID_ARG, fn + ": step must be >= 1");
+  if (!finite_nonneg(cfg->lr) || !finite_nonneg(cfg->weight_decay) || !finite_nonneg(cfg->eps))
+    return fail(ctx, MO_ERR_INVALID_ARG, fn + ": lr, weight_decay and eps must be finite and >= 0");
+  auto beta_ok = [](float b) { return b >= 0.f && b < 1.f; };
+  if (!beta_ok(cfg->beta1) || !beta_ok(cfg->beta2) || !beta_ok(cfg->shampoo_beta))
+    return fail(ctx, MO_ERR_INVALID_ARG, fn + ": betas must be in [0, 1)");
+  if (!(cfg->damping > 0.f && cfg->damping <= 1e-2f))
+    return fail(ctx, MO_ERR_INVALID_ARG, fn + ": damping must be in (0, 1e-2]");
+  std::vector<mo::SoapItem> items;
+  for (int i = 0; i < n; ++i) {
+    const mo_soap_mat& m = mats[i];
+    if (m.G == nullptr) continue;
+    if (m.rows <= 0 || m.cols <= 0 || m.rows > (1 << 16) || m.cols > (1 << 20))
+      return fail(ctx, MO_ERR_INVALID_ARG, fn + ": bad shape at index " + std::to_string(i));
+    if (m.W == nullptr || m.M == nullptr || m.V == nullptr)
+      return fail(ctx, MO_ERR_INVALID_ARG, fn + ": null W, M or V at index " + std::to_string(i));
+    if ((m.L == nullptr) != (m.QL == nullptr) || (m.R == nullptr) != (m.QR == nullptr))
+      return fail(ctx, MO_ERR_INVALID_ARG, fn + ": a side needs both its factor and its basis (index " + std::to_string(i) + ")");
+    if ((m.L && m.rows > 16384) || (m.R && m.cols > 16384))
+      return fail(ctx, MO_ERR_UNSUPPORTED, fn + ": factor sides above 16384 are not supported; pass NULL for an identity basis");
+    const void* ptrs[8] = {m.W, m.G, m.M, m.V, m.L, m.QL, m.R, m.QR};
+    for (const void* p : ptrs)
+      if (p && !aligned16(p))
+        return fail(ctx, MO_ERR_INVALID_ARG, fn + ": pointers must be 16-byte aligned (index " + std::to_string(i) + ")");
+    if (m.cols % 8 != 0 || m.rows % 8 != 0)
+      return fail(ctx, MO_ERR_UNSUPPORTED, fn + ": rows and cols must be multiples of 8 (index " + std::to_string(i) + ")");
+    mo::SoapItem it;
+    it.m = m;
+    it.flag = cfg->nonfinite ? cfg->nonfinite + i : nullptr;
+    items.push_back(it);
+  }
+  if (items.empty()) return MO_OK;
+  if (ctx->ws == nullptr) return fail(ctx, MO_ERR_NO_WORKSPACE, fn + ": no workspace attached");
+  mo_status st = enter(ctx);
+  if (st != MO_OK) return st;
+  std::string err;
+  cudaError_t e = mo::soap_run(items, *cfg, step, ctx->ws, ctx->ws_bytes, static_cast<cudaStream_t>(stream), &err, ext);
+  if (!err.empty()) return fail(ctx, e == cudaErrorNotSupported ? MO_ERR_UNSUPPORTED : MO_ERR_NO_WORKSPACE, fn + ": " + err);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, fn.c_str());
+  return MO_OK;
+}
+
+mo_soap_mat as_soap_mat(const mo_soap_muon_mat& a) {
+  mo_soap_mat m;
+  m.rows = a.rows; m.cols = a.cols; m.W = a.W; m.G = a.G; m.M = a.B; m.V = a.V;
+  m.L = a.L; m.QL = a.QL; m.R = a.R; m.QR = a.QR;
+  return m;
+}
+
+}  // namespace
+
 mo_status soap_step(mo_ctx* ctx, const mo_soap_mat* mats, int n, const mo_soap_cfg* cfg, int64_t step,
                     void* stream) {
   if (ctx == nullptr) return MO_ERR_INVALID_ARG;
@@ -282,46 +340,35 @@ mo_status soap_step(mo_ctx* ctx, const mo_soap_mat* mats, int n, const mo_soap_c
   ProfBind prof_bind(ctx);
   if (n == 0) return MO_OK;
   if (mats == nullptr || cfg == nullptr) return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: null mats or cfg");
-  if (step < 1) return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: step must be >= 1");
-  if (!finite_nonneg(cfg->lr) || !finite_nonneg(cfg->weight_decay) || !finite_nonneg(cfg->eps))
-    return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: lr, weight_decay and eps must be finite and >= 0");
-  auto beta_ok = [](float b) { return b >= 0.f && b < 1.f; };
-  if (!beta_ok(cfg->beta1) || !beta_ok(cfg->beta2) || !beta_ok(cfg->shampoo_beta))
-    return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: betas must be in [0, 1)");
-  if (!(cfg->damping > 0.f && cfg->damping <= 1e-2f))
-    return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: damping must be in (0, 1e-2]");
-  std::vector<mo::SoapItem> items;
-  for (int i = 0; i < n; ++i) {
-    const mo_soap_mat& m = mats[i];
-    if (m.G == nullptr) continue;
-    if (m.rows <= 0 || m.cols <= 0 || m.rows > (1 << 16) || m.cols > (1 << 20))
-      return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: bad shape at index " + std::to_string(i));
-    if (m.W == nullptr || m.M == nullptr || m.V == nullptr)
-      return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: null W, M or V at index " + std::to_string(i));
-    if ((m.L == nullptr) != (m.QL == nullptr) || (m.R == nullptr) != (m.QR == nullptr))
-      return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: a side needs both its factor and its basis (index " + std::to_string(i) + ")");
-    if ((m.L && m.rows > 16384) || (m.R && m.cols > 16384))
-      return fail(ctx, MO_ERR_UNSUPPORTED, "soap_step: factor sides above 16384 are not supported; pass NULL for an identity basis");
-    const void* ptrs[8] = {m.W, m.G, m.M, m.V, m.L, m.QL, m.R, m.QR};
-    for (const void* p : ptrs)
-      if (p && !aligned16(p))
-        return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: pointers must be 16-byte aligned (index " + std::to_string(i) + ")");
-    if (m.cols % 8 != 0 || m.rows % 8 != 0)
-      return fail(ctx, MO_ERR_UNSUPPORTED, "soap_step: rows and cols must be multiples of 8 (index " + std::to_string(i) + ")");
-    mo::SoapItem it;
-    it.m = m;
-    it.flag = cfg->nonfinite ? cfg->nonfinite + i : nullptr;
-    items.push_back(it);
-  }
-  if (items.empty()) return MO_OK;
-  if (ctx->ws == nullptr) return fail(ctx, MO_ERR_NO_WORKSPACE, "soap_step: no workspace attached");
-  mo_status st = enter(ctx);
+  return soap_impl(ctx, mats, n, cfg, step, stream, nullptr);
+}
+
+mo_status soap_muon_step(mo_ctx* ctx, const mo_soap_muon_mat* mats, int n, const mo_soap_muon_cfg* cfg,
+                         int64_t step, void* stream) {
+  if (ctx == nullptr) return MO_ERR_INVALID_ARG;
+  if (n < 0) return fail(ctx, MO_ERR_INVALID_ARG, "soap_muon_step: n < 0");
+  ProfBind prof_bind(ctx);
+  if (n == 0) return MO_OK;
+  if (mats == nullptr || cfg == nullptr) return fail(ctx, MO_ERR_INVALID_ARG, "soap_muon_step: null mats or cfg");
+  if (!(cfg->momentum >= 0.f && cfg->momentum < 1.f))
+    return fail(ctx, MO_ERR_INVALID_ARG, "soap_muon_step: momentum must be in [0, 1)");
+  if (cfg->adjust_lr != 0 && cfg->adjust_lr != 1)
+    return fail(ctx, MO_ERR_INVALID_ARG, "soap_muon_step: adjust_lr must be 0 or 1");
+  mo_status st = check_ns_coeffs(ctx, cfg->ns_steps, cfg->a, cfg->b, cfg->c, cfg->ns_eps, "soap_muon_step");
   if (st != MO_OK) return st;
-  std::string err;
-  cudaError_t e = mo::soap_run(items, *cfg, step, ctx->ws, ctx->ws_bytes, static_cast<cudaStream_t>(stream), &err);
-  if (!err.empty()) return fail(ctx, e == cudaErrorNotSupported ? MO_ERR_UNSUPPORTED : MO_ERR_NO_WORKSPACE, "soap_step: " + err);
-  if (e != cudaSuccess) return cuda_fail(ctx, e, "soap_step");
-  return MO_OK;
+  std::vector<mo_soap_mat> sm(n);
+  for (int i = 0; i < n; ++i) sm[i] = as_soap_mat(mats[i]);
+  mo_soap_cfg sc;
+  sc.lr = cfg->lr; sc.beta1 = cfg->momentum; sc.beta2 = cfg->beta2; sc.shampoo_beta = cfg->shampoo_beta;
+  sc.eps = cfg->eps; sc.weight_decay = cfg->weight_decay; sc.bias_correction = cfg->bias_correction;
+  sc.nonfinite = cfg->nonfinite; sc.skip_refresh = cfg->skip_refresh; sc.damping = cfg->damping;
+  mo::SoapMuonExt ext;
+  ext.mu = cfg->momentum;
+  ext.nesterov = cfg->nesterov != 0;
+  ext.ns.steps = cfg->ns_steps;
+  ext.ns.a = cfg->a; ext.ns.b = cfg->b; ext.ns.c = cfg->c; ext.ns.eps = cfg->ns_eps;
+  ext.ns.adjust_lr = cfg->adjust_lr;
+  return soap_impl(ctx, sm.data(), n, &sc, step, stream, &ext);
 }
 
 mo_status mo_soap_workspace_bytes(mo_ctx* ctx, const mo_soap_mat* mats, int n, size_t* bytes) {
@@ -336,6 +383,22 @@ mo_status mo_soap_workspace_bytes(mo_ctx* ctx, const mo_soap_mat* mats, int n, s
     items.push_back(it);
   }
   *bytes = mo::soap_workspace_exact(items);
+  return MO_OK;
+}
+
+mo_status mo_soap_muon_workspace_bytes(mo_ctx* ctx, const mo_soap_muon_mat* mats, int n, size_t* bytes) {
+  if (ctx == nullptr || bytes == nullptr) return MO_ERR_INVALID_ARG;
+  if (n < 0 || (n > 0 && mats == nullptr))
+    return fail(ctx, MO_ERR_INVALID_ARG, "mo_soap_muon_workspace_bytes: bad arguments");
+  std::vector<mo::SoapItem> items;
+  for (int i = 0; i < n; ++i) {
+    if (mats[i].rows <= 0 || mats[i].cols <= 0 || mats[i].rows > (1 << 16) || mats[i].cols > (1 << 20))
+      return fail(ctx, MO_ERR_INVALID_ARG, "mo_soap_muon_workspace_bytes: bad shape at index " + std::to_string(i));
+    mo::SoapItem it;
+    it.m = as_soap_mat(mats[i]);
+    items.push_back(it);
+  }
+  *bytes = mo::soap_workspace_exact(items, true);
   return MO_OK;
 }
 

@@ -389,18 +389,33 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       int b, tm, tn;
       if (!gemm_decode(p, BN, t, b, tm, tn)) continue;
-      // warp-uniform: tcgen05.ld below must be executed by all 32 lanes
-      const bool ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status, DEV_TIMEOUT_ACC_FULL);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
       const int r = tm * GEMM_BM + row_in_tile;
       const bool row_ok = r < p.M;
-      const float alpha = p.alpha * ipow_scale(p.scale, b, p.alpha_pow);
-      const float beta = p.beta * ipow_scale(p.scale, b, p.beta_pow);
       // this matrix's operands, resolved once per tile
       const char* cbase = has_c ? reinterpret_cast<const char*>(c_base(p, b)) : nullptr;
       char* dbase = reinterpret_cast<char*>(d_base(p, b));
       float* vbase = adam ? p.e_tab[b] : nullptr;
+      if (row_ok) {
+        // pull this row's epilogue inputs into L2 while the main loop runs,
+        // so that the loads after the accumulator wait do not pay DRAM latency
+        const int n0 = tn * BN;
+        const int nn = p.N - n0 < BN ? p.N - n0 : BN;
+        if (has_c && nn > 0) {
+          const int es = p.c_f32 ? 4 : 2;
+          const char* row = cbase + ((long long)r * p.ldc + n0) * es;
+          for (int off = 0; off < nn * es; off += 128) prefetch_l2(row + off);
+        }
+        if (adam && nn > 0) {
+          const char* row = reinterpret_cast<const char*>(vbase + (long long)r * p.lde + n0);
+          for (int off = 0; off < nn * 4; off += 128) prefetch_l2(row + off);
+        }
+      }
+      // warp-uniform: tcgen05.ld below must be executed by all 32 lanes
+      const bool ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status, DEV_TIMEOUT_ACC_FULL);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const float alpha = p.alpha * ipow_scale(p.scale, b, p.alpha_pow);
+      const float beta = p.beta * ipow_scale(p.scale, b, p.beta_pow);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
       for (int cc = 0; cc < BN; cc += 32) {

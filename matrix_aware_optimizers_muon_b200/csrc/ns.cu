@@ -73,13 +73,15 @@ void ns_workspace(const int64_t* rows, const int64_t* cols, int n, size_t* min_b
 
 cudaError_t ns_run(const std::vector<NsItem>& items, const NsCall& call, char* ws, size_t ws_bytes,
                    cudaStream_t stream, std::string* err) {
+  return ns_run_at(items, call, reinterpret_cast<int*>(ws), ws + WS_HEADER,
+                   ws_bytes > WS_HEADER ? ws_bytes - WS_HEADER : 0, stream, err);
+}
+
+cudaError_t ns_run_at(const std::vector<NsItem>& items, const NsCall& call, int* status, char* base,
+                      size_t avail, cudaStream_t stream, std::string* err) {
   std::map<Shape, std::vector<int>> buckets;
   for (int i = 0; i < (int)items.size(); ++i)
     buckets[oriented(items[i].rows, items[i].cols)].push_back(i);
-
-  int* status = reinterpret_cast<int*>(ws);
-  char* base = ws + WS_HEADER;
-  const size_t avail = ws_bytes > WS_HEADER ? ws_bytes - WS_HEADER : 0;
   auto is_tall = [&](int i) { return items[i].rows > items[i].cols; };
 
   for (auto& kv : buckets) {

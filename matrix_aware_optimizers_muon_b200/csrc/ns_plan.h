@@ -41,4 +41,9 @@ void ns_workspace(const int64_t* rows, const int64_t* cols, int n, size_t* min_b
 cudaError_t ns_run(const std::vector<NsItem>& items, const NsCall& call, char* ws, size_t ws_bytes,
                    cudaStream_t stream, std::string* err);
 
+// The same with the status word and the scratch region given apart (for
+// callers that place the Newton-Schulz scratch inside a larger workspace).
+cudaError_t ns_run_at(const std::vector<NsItem>& items, const NsCall& call, int* status, char* base,
+                      size_t avail, cudaStream_t stream, std::string* err);
+
 }  // namespace mo

@@ -52,12 +52,27 @@ __global__ void soap_prep_kernel(const SoapPrepArgs a) {
     const long long r = i / cols4, q = i - r * cols4;
     const float4 g = __ldcs(reinterpret_cast<const float4*>(G) + i);
     float4 m = reinterpret_cast<const float4*>(M)[i];
+    const size_t off = (size_t)j * a.mat_stride + (size_t)r * a.ldp + 4 * q;
+    if (a.muon) {
+      // Muon momentum (sum form) and the Nesterov numerator
+      m.x = fmaf(a.beta1, m.x, g.x);
+      m.y = fmaf(a.beta1, m.y, g.y);
+      m.z = fmaf(a.beta1, m.z, g.z);
+      m.w = fmaf(a.beta1, m.w, g.w);
+      reinterpret_cast<float4*>(M)[i] = m;
+      float4 nv = m;
+      if (a.nesterov)
+        nv = make_float4(fmaf(a.beta1, m.x, g.x), fmaf(a.beta1, m.y, g.y), fmaf(a.beta1, m.z, g.z),
+                         fmaf(a.beta1, m.w, g.w));
+      store_planes4(a.Gp + off, a.plane_stride, g);
+      store_planes4(a.Mp + off, a.plane_stride, nv);
+      continue;
+    }
     m.x = fmaf(a.beta1, m.x, c * g.x);
     m.y = fmaf(a.beta1, m.y, c * g.y);
     m.z = fmaf(a.beta1, m.z, c * g.z);
     m.w = fmaf(a.beta1, m.w, c * g.w);
     reinterpret_cast<float4*>(M)[i] = m;
-    const size_t off = (size_t)j * a.mat_stride + (size_t)r * a.ldp + 4 * q;
     store_planes4(a.Gp + off, a.plane_stride, g);
     store_planes4(a.Mp + off, a.plane_stride, m);
   }
@@ -281,8 +296,23 @@ __global__ void adam_identity_kernel(const AdamIdArgs a) {
     const float4 g = __ldcs(reinterpret_cast<const float4*>(G) + i);
     const float4 m = __ldcs(reinterpret_cast<const float4*>(M) + i);
     float4 v = reinterpret_cast<const float4*>(V)[i];
-    float4 w = reinterpret_cast<const float4*>(W)[i];
     const float c = 1.0f - a.beta2;
+    if (a.muon) {
+      // SOAP-Muon with identity bases: P = N / (sqrt(V / bc2) + eps)
+      float4 x = m;
+      if (a.nesterov)
+        x = make_float4(fmaf(a.mu, m.x, g.x), fmaf(a.mu, m.y, g.y), fmaf(a.mu, m.z, g.z), fmaf(a.mu, m.w, g.w));
+      float4 pv;
+#define MO_PRE(X)                                                               \
+      v.X = fmaf(a.beta2, v.X, c * g.X * g.X);                                  \
+      pv.X = (x.X * a.ibc1) / (sqrtf(v.X * a.ibc2) + a.eps);
+      MO_PRE(x) MO_PRE(y) MO_PRE(z) MO_PRE(w)
+#undef MO_PRE
+      reinterpret_cast<float4*>(V)[i] = v;
+      reinterpret_cast<float4*>(a.P[j])[i] = pv;
+      continue;
+    }
+    float4 w = reinterpret_cast<const float4*>(W)[i];
 #define MO_ADAM(X)                                                              \
     v.X = fmaf(a.beta2, v.X, c * g.X * g.X);                                    \
     w.X = fmaf(a.decay, w.X, -a.lr * ((m.X * a.ibc1) / (sqrtf(v.X * a.ibc2) + a.eps)));

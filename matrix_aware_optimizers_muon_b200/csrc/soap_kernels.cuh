@@ -15,7 +15,8 @@ void launch_upload_ptrs(void** dst, const void* const* src, int n, cudaStream_t 
 struct SoapPrepArgs {
   int count;
   long long rows, cols;            // matrix shape (cols % 4 == 0)
-  float beta1;
+  float beta1;                     // SOAP: M's beta; SOAP-Muon: the momentum mu
+  int muon = 0, nesterov = 0;      // SOAP-Muon: B <- mu B + G, planes of N = G + mu B (or B)
   const float* G[SOAP_MAXB];
   float* M[SOAP_MAXB];
   __nv_bfloat16* Gp;               // two planes of G: [2][count][*][ldp]
@@ -23,6 +24,7 @@ struct SoapPrepArgs {
   long long ldp, mat_stride, plane_stride;
 };
 // M <- b1 M + (1 - b1) G ; two bf16 planes (h, l) of G and of the new M
+// (SOAP-Muon: of G and of the Nesterov momentum N)
 void launch_soap_prep(const SoapPrepArgs& a, cudaStream_t s);
 
 // Split fp32 matrices into bf16 planes x = h + m + l (nearly exact): plane p
@@ -99,14 +101,19 @@ void launch_copy_out(const CopyOutArgs& a, cudaStream_t s);
 
 // Adam step with identity bases (both sides) fused with the apply:
 // V <- b2 V + (1-b2) G^2 ; W <- decay W - lr (M / bc1) / (sqrt(V / bc2) + eps)
+// SOAP-Muon (muon = 1): M holds the updated momentum B, the numerator is
+// N = G + mu B (Nesterov) or B, and the result Dbar goes to P instead of W.
 struct AdamIdArgs {
   int count;
   long long elems;
   float beta2, ibc1, ibc2, eps, decay, lr;
+  int muon = 0, nesterov = 0;
+  float mu = 0.f;
   const float* G[SOAP_MAXB];
   const float* M[SOAP_MAXB];
   float* V[SOAP_MAXB];
   float* W[SOAP_MAXB];
+  float* P[SOAP_MAXB];
 };
 void launch_adam_identity(const AdamIdArgs& a, cudaStream_t s);
 

@@ -144,3 +144,34 @@ def test_gemm_rejects_misaligned(lib):
     d.sym, d.N = 1, 32
     assert lib.mo_gemm_bf16(h, ctypes.byref(d), None) == _lib.MO_ERR_INVALID_ARG
     lib.mo_ctx_destroy(h)
+
+
+def test_soap_muon_rejects_bad_arguments(lib):
+    h = _ctx(lib)
+    good = _lib.SoapMuonMat(8, 8, 16, 16, 16, 16, 16, 16, None, None)
+    mats = (_lib.SoapMuonMat * 1)(good)
+
+    def cfg(**kw):
+        base = dict(lr=0.02, weight_decay=0.01, momentum=0.95, nesterov=1, beta2=0.95,
+                    shampoo_beta=0.9, eps=1e-8, bias_correction=1, ns_steps=5, a=3.4445,
+                    b=-4.7750, c=2.0315, ns_eps=1e-7, adjust_lr=0, damping=1e-5,
+                    nonfinite=None, skip_refresh=0)
+        base.update(kw)
+        return _lib.SoapMuonCfg(**base)
+
+    for bad in (dict(momentum=1.0), dict(adjust_lr=2), dict(ns_steps=0), dict(damping=0.0),
+                dict(beta2=1.0), dict(lr=float("nan"))):
+        assert lib.soap_muon_step(h, mats, 1, ctypes.byref(cfg(**bad)), 1, None) == _lib.MO_ERR_INVALID_ARG, bad
+        assert lib.mo_last_error(h).startswith(b"soap_muon_step")
+    assert lib.soap_muon_step(h, mats, 1, ctypes.byref(cfg()), 0, None) == _lib.MO_ERR_INVALID_ARG
+    half = _lib.SoapMuonMat(8, 8, 16, 16, 16, 16, 16, None, None, None)
+    mats = (_lib.SoapMuonMat * 1)(half)
+    assert lib.soap_muon_step(h, mats, 1, ctypes.byref(cfg()), 1, None) == _lib.MO_ERR_INVALID_ARG
+    size = ctypes.c_size_t()
+    mats = (_lib.SoapMuonMat * 1)(good)
+    assert lib.mo_soap_muon_workspace_bytes(h, mats, 1, ctypes.byref(size)) == 0
+    plain = ctypes.c_size_t()
+    smats = (_lib.SoapMat * 1)(_lib.SoapMat(8, 8, 16, 16, 16, 16, 16, 16, None, None))
+    assert lib.mo_soap_workspace_bytes(h, smats, 1, ctypes.byref(plain)) == 0
+    assert size.value > plain.value          # P and the Newton-Schulz scratch on top
+    lib.mo_ctx_destroy(h)

@@ -71,7 +71,8 @@ struct GemmCfg {
   static constexpr int STAGES = BN == 256 ? 4 : 6;
   static constexpr int TMEM_COLS = 2 * BN;          // two fp32 accumulators
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr int EPI_BYTES = 4 * 6144;        // per epilogue warp: output block, its transpose, C block
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + EPI_BYTES + 1024;
 };
 
 // Tiles of one matrix in column order (M fastest, so the CTAs in flight
@@ -231,6 +232,48 @@ __device__ __forceinline__ void store_mirror(const GemmParams& p, char* base, in
   }
 }
 
+// Coalesced bf16 stores of one warp's 32 x 32 output block through shared
+// memory: the block (rows of the warp's lanes, columns c0..c0+31) is staged
+// row-major and, for a symmetric product, transposed; then every store
+// instruction writes eight full 64-byte rows.  The staging rows are 64 bytes
+// with their four 16-byte units XOR-swizzled by (row / 2) % 4, which keeps
+// the 16-byte writes, the 2-byte transposed writes and the 16-byte reads
+// free of bank conflicts.  drow = &D[r0][c0]; dmir = &D[c0][r0] or null.
+__device__ __forceinline__ uint32_t stg_off(int row, int unit) {
+  return (uint32_t)(row * 64 + ((unit ^ ((row >> 1) & 3)) << 4));
+}
+
+__device__ __forceinline__ void stage_store32(uint8_t* stg, int lane, const float (&x)[32], __nv_bfloat16* drow,
+                                              __nv_bfloat16* dmir, long long ldd) {
+  uint8_t* srow = stg;
+  uint8_t* scol = stg + 2048;
+  __syncwarp();                       // the previous block's reads are done
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(x[8 * u + 2 * j], x[8 * u + 2 * j + 1]);
+      w[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(srow + stg_off(lane, u)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (dmir) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      *reinterpret_cast<__nv_bfloat16*>(scol + stg_off(i, lane >> 3) + ((lane & 7) << 1)) = __float2bfloat16_rn(x[i]);
+  }
+  __syncwarp();
+  const int u = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int R = 8 * j + (lane >> 2);
+    *reinterpret_cast<uint4*>(drow + (long long)R * ldd + 8 * u) = *reinterpret_cast<const uint4*>(srow + stg_off(R, u));
+    if (dmir)
+      *reinterpret_cast<uint4*>(dmir + (long long)R * ldd + 8 * u) = *reinterpret_cast<const uint4*>(scol + stg_off(R, u));
+  }
+}
+
 template <int BN, int A_MN, int B_MN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -382,6 +425,9 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
+    uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES + q * 6144;
+    uint8_t* stc = stg + 4096;              // staged 32 x 32 block of C
+    const bool plain_bf16 = !p.d_f32 && !p.d_split;
     const bool has_c = p.C != nullptr || p.c_tab != nullptr;
     const bool adam = p.epi == EPI_ADAM;
     int acc = 0;
@@ -417,13 +463,41 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const float alpha = p.alpha * ipow_scale(p.scale, b, p.alpha_pow);
       const float beta = p.beta * ipow_scale(p.scale, b, p.beta_pow);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const int r0 = tm * GEMM_BM + q * 32;     // this warp's first row
+      const int n0 = tn * BN;
+      // a symmetric product skips the 32 x 32 blocks below the diagonal
+      const int cc_begin = p.sym ? (r0 - n0 > 0 ? r0 - n0 : 0) : 0;
+      // bf16 C for full blocks: loaded one block ahead with coalesced
+      // 16-byte loads (eight 64-byte rows per instruction), then transposed
+      // to row-per-lane through shared memory
+      const bool cpre = has_c && !adam && !p.c_f32 && plain_bf16 && n0 + BN <= p.N &&
+                        __all_sync(0xffffffffu, row_ok);
+      const __nv_bfloat16* c16 = reinterpret_cast<const __nv_bfloat16*>(cbase);
+      uint4 cnext[4];
+      auto load_c = [&](int cc) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int R = 8 * j + (lane >> 2);
+          cnext[j] = *reinterpret_cast<const uint4*>(c16 + (long long)(r0 + R) * p.ldc + n0 + cc + 8 * (lane & 3));
+        }
+      };
+      if (cpre && cc_begin < BN) load_c(cc_begin);
 #pragma unroll 1
-      for (int cc = 0; cc < BN; cc += 32) {
+      for (int cc = cc_begin; cc < BN; cc += 32) {
+        uint4 ccur[4];
+        if (cpre) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) ccur[j] = cnext[j];
+          if (cc + 32 < BN) load_c(cc + 32);
+        }
         uint32_t v[32];
         tmem_ld32(taddr + cc, v);
         tmem_ld_wait();
-        const int c0 = tn * BN + cc;
-        if (row_ok && c0 < p.N) {
+        const int c0 = n0 + cc;
+        // warp-uniform: every lane holds a full row segment of plain bf16 output
+        const bool fast = plain_bf16 && __all_sync(0xffffffffu, row_ok && c0 + 32 <= p.N) &&
+                          (!p.sym || c0 >= r0 + 32);
+        if (fast || (row_ok && c0 < p.N)) {
           const bool full = c0 + 32 <= p.N;
           float x[32];
 #pragma unroll
@@ -442,13 +516,34 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 x[i] = (mr[i] * p.adam_ibc1) / (sqrtf(vn * p.adam_ibc2) + p.adam_eps);
               }
             }
+          } else if (cpre) {
+            __syncwarp();                 // the previous block's reads of stc are done
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              *reinterpret_cast<uint4*>(stc + stg_off(8 * j + (lane >> 2), lane & 3)) = ccur[j];
+            __syncwarp();
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint4 w = *reinterpret_cast<const uint4*>(stc + stg_off(lane, u));
+              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ws[j]));
+                x[8 * u + 2 * j] = fmaf(beta, f.x, x[8 * u + 2 * j]);
+                x[8 * u + 2 * j + 1] = fmaf(beta, f.y, x[8 * u + 2 * j + 1]);
+              }
+            }
           } else if (has_c) {
             float c[32];
             load_row32(cbase, p.c_f32, (long long)r * p.ldc + c0, full ? 32 : p.N - c0, c);
 #pragma unroll
             for (int i = 0; i < 32; ++i) x[i] = fmaf(beta, c[i], x[i]);
           }
-          if (!p.sym) {
+          if (fast) {
+            __nv_bfloat16* d16 = reinterpret_cast<__nv_bfloat16*>(dbase);
+            stage_store32(stg, lane, x, d16 + (long long)r0 * p.ldd + c0,
+                          p.sym ? d16 + (long long)c0 * p.ldd + r0 : nullptr, p.ldd);
+          } else if (!p.sym) {
             store_row(p, dbase, (long long)r * p.ldd + c0, full ? 32 : p.N - c0, 0, x);
           } else if (c0 + 31 >= r) {
             // upper part of this row chunk: store it, then its mirror image

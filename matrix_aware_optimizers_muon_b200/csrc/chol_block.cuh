@@ -1,0 +1,155 @@
+// Cholesky factor and its inverse for one 128 x 128 symmetric positive
+// definite block in shared memory, blocked by 32:
+//   for each 32-column block kb:
+//     warp 0 factors the 32 x 32 diagonal block in registers (one row per
+//     lane, pivots and columns exchanged by shuffles);
+//     the rows below solve against it (one row per thread);
+//     every thread updates 4 x 4 tiles of the trailing lower triangle;
+//   then four warps invert the four diagonal 32 x 32 factors (one column per
+//   lane) and the off-diagonal blocks of the inverse follow block row by
+//   block row: X_ij = -X_ii (sum_{j<=k<i} L_ik X_kj).
+// 256 threads; A and X are [128][129] fp32 (row stride 129), T is [32][97]
+// scratch.  A holds the block on entry (lower triangle read) and L on exit
+// (lower triangle); X receives L^{-1} (lower triangle; the upper triangle is
+// not written).  Returns through *bad whether a pivot was not positive
+// (NaN included).
+#pragma once
+
+namespace mo {
+
+constexpr int CB = 128;
+constexpr int CB_LD = CB + 1;
+constexpr int CB_T_LD = 97;
+
+__device__ __forceinline__ void chol128_factor(float* A, float* inv_diag, int* bad) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int kb = 0; kb < 4; ++kb) {
+    const int b0 = 32 * kb;
+    // ---- diagonal block: lane i holds row b0 + i
+    if (warp == 0) {
+      float r[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) r[c] = c <= lane ? A[(b0 + lane) * CB_LD + b0 + c] : 0.f;
+      bool ok = true;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float d = __shfl_sync(0xffffffffu, r[j], j);
+        ok = ok && (d > 0.f);
+        const float sq = sqrtf(d);
+        const float inv = 1.0f / sq;
+        if (lane == j) r[j] = sq;
+        else if (lane > j) r[j] *= inv;
+        if (lane == j) inv_diag[b0 + j] = inv;
+#pragma unroll
+        for (int c = j + 1; c < 32; ++c) {
+          const float lcj = __shfl_sync(0xffffffffu, r[j], c);
+          if (c <= lane) r[c] = fmaf(-r[j], lcj, r[c]);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (c <= lane) A[(b0 + lane) * CB_LD + b0 + c] = r[c];
+      if (lane == 0 && !ok) *bad = 1;
+    }
+    __syncthreads();
+    const int n2 = CB - b0 - 32;                  // rows / columns after this block
+    // ---- panel: rows below solve x L_D^T = a (one row per thread)
+    if (tid < n2) {
+      const int row = b0 + 32 + tid;
+      float a[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) a[c] = A[row * CB_LD + b0 + c];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float acc = a[j];
+#pragma unroll
+        for (int p = 0; p < j; ++p) acc = fmaf(-a[p], A[(b0 + j) * CB_LD + b0 + p], acc);
+        a[j] = acc * inv_diag[b0 + j];
+      }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) A[row * CB_LD + b0 + c] = a[c];
+    }
+    __syncthreads();
+    // ---- trailing update of the lower triangle in 4 x 4 tiles
+    if (n2 > 0) {
+      const int nt = n2 / 4;
+      const int tiles = nt * (nt + 1) / 2;
+      const int base = b0 + 32;
+      for (int t = tid; t < tiles; t += blockDim.x) {
+        // tile (tr, tc) with tc <= tr, enumerated row by row
+        int tr = (int)((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
+        while (tr * (tr + 1) / 2 > t) --tr;
+        while ((tr + 1) * (tr + 2) / 2 <= t) ++tr;
+        const int tc = t - tr * (tr + 1) / 2;
+        const int r0 = base + 4 * tr, c0 = base + 4 * tc;
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+        for (int p = 0; p < 32; ++p) {
+          float lr[4], lc[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            lr[i] = A[(r0 + i) * CB_LD + b0 + p];
+            lc[i] = A[(c0 + i) * CB_LD + b0 + p];
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(lr[i], lc[j], acc[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (c0 + j <= r0 + i) A[(r0 + i) * CB_LD + c0 + j] -= acc[i][j];
+      }
+    }
+    __syncthreads();
+  }
+}
+
+__device__ __forceinline__ void chol128_inverse(const float* A, const float* inv_diag, float* X, float* T) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // ---- diagonal blocks: warp w inverts block w; lane c owns column c
+  if (warp < 4) {
+    const int b0 = 32 * warp;
+    float x[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float acc = i == lane ? 1.0f : 0.f;
+#pragma unroll
+      for (int p = 0; p < i; ++p) acc = fmaf(-A[(b0 + i) * CB_LD + b0 + p], x[p], acc);
+      x[i] = i >= lane ? acc * inv_diag[b0 + i] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) X[(b0 + i) * CB_LD + b0 + lane] = x[i];
+  }
+  __syncthreads();
+  // ---- off-diagonal blocks, block row by block row
+  for (int bi = 1; bi < 4; ++bi) {
+    const int r0 = 32 * bi;
+    // T[:, 32 bj + c] = sum_{bj <= k < bi} L[r0 + :, block k] X[block k, 32 bj + c]
+    const int cols = 32 * bi;
+    for (int e = tid; e < 32 * cols; e += blockDim.x) {
+      const int i = e / cols, c = e - i * cols;     // c: column of X (0 .. 32 bi - 1)
+      const int kstart = c & ~31;                    // X[k][c] is zero for k < block of c
+      float acc = 0.f;
+      for (int k = kstart; k < r0; ++k) acc = fmaf(A[(r0 + i) * CB_LD + k], X[k * CB_LD + c], acc);
+      T[i * CB_T_LD + c] = acc;
+    }
+    __syncthreads();
+    // X[r0 + i, c] = -sum_{p <= i} X[r0 + i, r0 + p] T[p, c]
+    for (int e = tid; e < 32 * cols; e += blockDim.x) {
+      const int i = e / cols, c = e - i * cols;
+      float acc = 0.f;
+      for (int p = 0; p <= i; ++p) acc = fmaf(X[(r0 + i) * CB_LD + r0 + p], T[p * CB_T_LD + c], acc);
+      X[(r0 + i) * CB_LD + c] = -acc;
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace mo

@@ -81,6 +81,7 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   for (int i = 0; i < 8; ++i) { p.pat_a[i] = op.pat_a[i]; p.pat_b[i] = op.pat_b[i]; }
   p.d_split = op.d_split;
   p.d_plane = op.d_plane;
+  p.skip = op.skip;
 
   auto kern = gemm_bf16_kernel<BN, A_MN, B_MN>;
   static int attr_done[64] = {0};

@@ -55,6 +55,9 @@ struct GemmParams {
   // bf16 output as two planes: D = bf16(x), D + d_plane = bf16(x - bf16(x))
   int d_split;
   long long d_plane;
+  // optional per-matrix flags (device): matrices with skip[b] != 0 are left
+  // untouched (every role of the kernel skips their tiles)
+  const int* skip;
 };
 
 enum { EPI_AXPBY = 0, EPI_ADAM = 1 };
@@ -71,7 +74,7 @@ struct GemmCfg {
   static constexpr int STAGES = BN == 256 ? 4 : 6;
   static constexpr int TMEM_COLS = 2 * BN;          // two fp32 accumulators
   static constexpr int BAR_BYTES = 256;
-  static constexpr int EPI_BYTES = 4 * 6144;        // per epilogue warp: output block, its transpose, C block
+  static constexpr int EPI_BYTES = 4 * 8192;        // per epilogue warp: output block (or C), its transpose
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + EPI_BYTES + 1024;
 };
 
@@ -88,6 +91,7 @@ __device__ __forceinline__ int sym_rows_in_col(const GemmParams& p, int BN, int 
 __device__ __forceinline__ bool gemm_decode(const GemmParams& p, int BN, int t, int& b, int& tm,
                                             int& tn) {
   b = t / p.tiles_per_mat;
+  if (p.skip && p.skip[b]) return false;
   int u = t - b * p.tiles_per_mat;
   if (!p.sym) {
     tn = u / p.tiles_m;
@@ -274,6 +278,36 @@ __device__ __forceinline__ void stage_store32(uint8_t* stg, int lane, const floa
   }
 }
 
+// The fp32 version: 128-byte staging rows with the classic 128-byte XOR
+// swizzle (unit ^ row % 8); every store instruction writes four full rows.
+__device__ __forceinline__ uint32_t stg32_off(int row, int unit) {
+  return (uint32_t)(row * 128 + ((unit ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ void stage_store32_f32(uint8_t* stg, int lane, const float (&x)[32], float* drow,
+                                                  float* dmir, long long ldd) {
+  uint8_t* srow = stg;
+  uint8_t* scol = stg + 4096;
+  __syncwarp();                       // earlier reads of the staging rows are done
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    *reinterpret_cast<float4*>(srow + stg32_off(lane, u)) = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+  if (dmir) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      *reinterpret_cast<float*>(scol + stg32_off(i, lane >> 2) + ((lane & 3) << 2)) = x[i];
+  }
+  __syncwarp();
+  const int u = lane & 7;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int R = 4 * j + (lane >> 3);
+    *reinterpret_cast<float4*>(drow + (long long)R * ldd + 4 * u) = *reinterpret_cast<const float4*>(srow + stg32_off(R, u));
+    if (dmir)
+      *reinterpret_cast<float4*>(dmir + (long long)R * ldd + 4 * u) = *reinterpret_cast<const float4*>(scol + stg32_off(R, u));
+  }
+}
+
 template <int BN, int A_MN, int B_MN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -425,9 +459,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
-    uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES + q * 6144;
-    uint8_t* stc = stg + 4096;              // staged 32 x 32 block of C
+    uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES + q * 8192;
+    uint8_t* stc = stg + 4096;              // staged 32 x 32 bf16 block of C
     const bool plain_bf16 = !p.d_f32 && !p.d_split;
+    const bool plain_f32 = p.d_f32 && !p.d_split;
     const bool has_c = p.C != nullptr || p.c_tab != nullptr;
     const bool adam = p.epi == EPI_ADAM;
     int acc = 0;
@@ -482,6 +517,11 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
       };
       if (cpre && cc_begin < BN) load_c(cc_begin);
+      // fp32 C for full blocks: coalesced 16-byte loads issued before the
+      // accumulator read, staged in shared memory (the output's staging rows)
+      const bool cf32 = has_c && !adam && p.c_f32 && !p.d_split && n0 + BN <= p.N &&
+                        __all_sync(0xffffffffu, row_ok);
+      const float* c32 = reinterpret_cast<const float*>(cbase);
 #pragma unroll 1
       for (int cc = cc_begin; cc < BN; cc += 32) {
         uint4 ccur[4];
@@ -490,14 +530,22 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           for (int j = 0; j < 4; ++j) ccur[j] = cnext[j];
           if (cc + 32 < BN) load_c(cc + 32);
         }
+        float4 cf[8];
+        if (cf32) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            cf[j] = *reinterpret_cast<const float4*>(c32 + (long long)(r0 + 4 * j + (lane >> 3)) * p.ldc + n0 + cc +
+                                                     4 * (lane & 7));
+        }
         uint32_t v[32];
         tmem_ld32(taddr + cc, v);
         tmem_ld_wait();
         const int c0 = n0 + cc;
         // warp-uniform: every lane holds a full row segment of plain bf16 output
-        const bool fast = plain_bf16 && __all_sync(0xffffffffu, row_ok && c0 + 32 <= p.N) &&
-                          (!p.sym || c0 >= r0 + 32);
-        if (fast || (row_ok && c0 < p.N)) {
+        const bool blk_full = __all_sync(0xffffffffu, row_ok && c0 + 32 <= p.N) && (!p.sym || c0 >= r0 + 32);
+        const bool fast = plain_bf16 && blk_full;
+        const bool fast32 = plain_f32 && blk_full;
+        if (fast || fast32 || cf32 || (row_ok && c0 < p.N)) {
           const bool full = c0 + 32 <= p.N;
           float x[32];
 #pragma unroll
@@ -515,6 +563,20 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 vp[i] = vn;
                 x[i] = (mr[i] * p.adam_ibc1) / (sqrtf(vn * p.adam_ibc2) + p.adam_eps);
               }
+            }
+          } else if (cf32) {
+            __syncwarp();                 // the previous block's reads of the staging rows are done
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4*>(stg + stg32_off(4 * j + (lane >> 3), lane & 7)) = cf[j];
+            __syncwarp();
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float4 w = *reinterpret_cast<const float4*>(stg + stg32_off(lane, u));
+              x[4 * u] = fmaf(beta, w.x, x[4 * u]);
+              x[4 * u + 1] = fmaf(beta, w.y, x[4 * u + 1]);
+              x[4 * u + 2] = fmaf(beta, w.z, x[4 * u + 2]);
+              x[4 * u + 3] = fmaf(beta, w.w, x[4 * u + 3]);
             }
           } else if (cpre) {
             __syncwarp();                 // the previous block's reads of stc are done
@@ -539,7 +601,11 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 32; ++i) x[i] = fmaf(beta, c[i], x[i]);
           }
-          if (fast) {
+          if (fast32) {
+            float* d32 = reinterpret_cast<float*>(dbase);
+            stage_store32_f32(stg, lane, x, d32 + (long long)r0 * p.ldd + c0,
+                              p.sym ? d32 + (long long)c0 * p.ldd + r0 : nullptr, p.ldd);
+          } else if (fast) {
             __nv_bfloat16* d16 = reinterpret_cast<__nv_bfloat16*>(dbase);
             stage_store32(stg, lane, x, d16 + (long long)r0 * p.ldd + c0,
                           p.sym ? d16 + (long long)c0 * p.ldd + r0 : nullptr, p.ldd);

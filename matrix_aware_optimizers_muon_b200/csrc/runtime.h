@@ -50,6 +50,8 @@ struct GemmOp {
   // bf16 D written as two planes (h, l) d_plane elements apart
   int d_split = 0;
   long long d_plane = 0;
+  // per-matrix skip flags in device memory (optional)
+  const int* skip = nullptr;
 };
 
 // Launch the tcgen05 GEMM.  Returns cudaSuccess or the launch/encode error.

@@ -5,16 +5,22 @@
 //   EMAs:  L <- bs L + (1-bs) Gb Gb^T ; R <- bs R + (1-bs) Gb^T Gb
 //          (symmetric tcgen05 products written into the caller's L / R)
 // Phase 2 (per bucket of equal factor size k, all sides of all matrices):
-//   power: Y = L Q, fp32-accurate (3-plane bf16 split, 6 plane products)
-//   QR:    shifted CholeskyQR3: three passes of
+//   power: Y = (L + d I) Q, d = damping * trace(L), fp32-accurate
+//          (3-plane bf16 split, 6 plane products)
+//   QR:    shifted CholeskyQR3: up to three passes of
 //            column-normalise Y, C = Y^T Y (fp32-accurate), [shift C],
 //            blocked Cholesky C = L L^T with 128-wide diagonal blocks and
-//            Y <- Y L^{-T} (right-looking, tensor-core trailing updates)
+//            Y <- Y L^{-T} (right-looking, tensor-core trailing updates);
+//          the third pass is skipped per matrix when its Gram is already
+//          within 5e-5 of the identity (every warm step)
 //          -> Q (unique QR, diag(R) > 0) into the caller's Q and bf16(Q)
 // Phase 3 (per group): rotations with two-plane bf16 operands (x = h + l,
-//   three bf16 MMAs hh + hl + lh per product), Adam in the rotated basis
+//   three bf16 MMAs lh + hl + hh per product), Adam in the rotated basis
 //   fused into the epilogue of the G' product, rotation back fused with
 //   W <- (1 - lr wd) W - lr D.
+// SOAP-Muon runs phase 1, the rotations with the stored bases (writing the
+// preconditioned momentum P instead of applying), the Muon engine on P, and
+// the refresh last.
 #include <algorithm>
 #include <cmath>
 #include <map>
@@ -34,9 +40,13 @@ constexpr size_t AL = 1024;
 size_t al(size_t x) { return (x + AL - 1) / AL * AL; }
 
 // plane products of the fp32-accurate GEMMs: x = h + m + l, and
-// x y ~ hh + hm + mh + hl + lh + mm  (dropped terms are below 2^-24)
-const unsigned char PAT_A[6] = {0, 0, 1, 0, 2, 1};
-const unsigned char PAT_B[6] = {0, 1, 0, 2, 0, 1};
+// x y ~ hh + hm + mh + hl + lh + mm  (dropped terms are below 2^-24).  The
+// small products are accumulated first and hh last: the tensor core's fp32
+// accumulation loses low-order bits of each addend that is small next to
+// the running sum, so adding the small terms into an accumulator that
+// already holds hh would cost most of their accuracy.
+const unsigned char PAT_A[6] = {1, 2, 0, 1, 0, 0};
+const unsigned char PAT_B[6] = {1, 0, 2, 0, 1, 0};
 
 void set_planes(GemmOp& g, long long planeA, long long planeB) {
   g.nseg = 6;
@@ -45,9 +55,10 @@ void set_planes(GemmOp& g, long long planeA, long long planeB) {
   g.planeB = planeB;
 }
 
-// two-plane products of the rotations: x = h + l, x y ~ hh + hl + lh
+// two-plane products of the rotations: x = h + l, x y ~ lh + hl + hh
+// (small products first, as above)
 void set_planes2(GemmOp& g, long long planeA, long long planeB) {
-  const unsigned char pa[3] = {0, 0, 1}, pb[3] = {0, 1, 0};
+  const unsigned char pa[3] = {1, 0, 0}, pb[3] = {0, 1, 0};
   g.nseg = 3;
   for (int i = 0; i < 3; ++i) { g.pat_a[i] = pa[i]; g.pat_b[i] = pb[i]; }
   g.planeA = planeA;
@@ -73,7 +84,7 @@ struct Job {
 struct Bucket {
   long long k, kp;
   std::vector<Job> jobs;
-  size_t y, c, ypl, qpl, ppl, qjpl, dinv, invd, damp;
+  size_t y, c, ypl, qpl, ppl, qjpl, dinv, invd, damp, qdev, qskip;
 };
 
 struct Plan {
@@ -145,6 +156,8 @@ Plan make_plan(const std::vector<SoapItem>& items, bool with_p = false) {
     b.dinv = off; off += al(q * QR_B * QR_B * 4);
     b.invd = off; off += al(q * b.kp * 4);
     b.damp = off; off += al(q * 4);
+    b.qdev = off; off += al(q * 4);
+    b.qskip = off; off += al(q * 4);
   }
   P.total = off;
   return P;
@@ -396,10 +409,23 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
         // shifted pass leaves a Q whose Gram the two unshifted passes
         // factor safely (cond(Q) below the fp32 limit of Cholesky QR).
         if (pass == 0) launch_shift_diag(C, kp, kk, q, (int)kp, 1e-5f * (float)kp, s);
+        // The last pass only corrects what is left of the previous pass's
+        // rounding.  A basis whose Gram is within 5e-5 of the identity keeps
+        // its (column-normalised) Q and every kernel of the pass skips it:
+        // the tensor core's fp32 accumulation leaves the Gram of an exactly
+        // orthonormal 4096-column basis about 2e-5 off the identity, so the
+        // pass could not lower the error below that floor, and the two-plane
+        // rotations that use the basis resolve 2^-16 = 1.5e-5.  Cold starts
+        // (deviation 1e-2 and more after the shifted pass) run all three.
+        const int* skip = nullptr;
+        if (pass == 2) {
+          launch_identity_check(C, kp, kk, q, (int)kp, 5e-5f, at<int>(ws, bk.qdev), at<int>(ws, bk.qskip), s);
+          skip = at<int>(ws, bk.qskip);
+        }
         for (int jb = 0; jb < nb; ++jb) {
           const long long k0 = (long long)jb * QR_B;
           const long long rem = kp - k0 - QR_B;
-          launch_chol_diag(C, kp, kk, q, (int)k0, Dinv, flags, s);
+          launch_chol_diag(C, kp, kk, q, (int)k0, Dinv, flags, s, skip);
           if (rem > 0) {      // panel L21 = C21 L11^{-T}, kept only as planes
             RowBlockArgs ra;
             ra.count = q; ra.rows = (int)rem;
@@ -407,6 +433,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
             ra.out = nullptr; ra.ld_out = 0; ra.out_stride = 0;
             ra.Dinv = Dinv;
             ra.planes = Ppl; ra.plane_stride = (long long)q * kp * QR_B; ra.mat_stride = kp * QR_B;
+            ra.skip = skip;
             launch_rowblock_dinv(ra, s);
           }
           {                   // Q_j = Y_j L_jj^{-T} (in place) and its planes
@@ -416,6 +443,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
             ra.out = Y + k0; ra.ld_out = kp; ra.out_stride = kk;
             ra.Dinv = Dinv;
             ra.planes = Qjpl; ra.plane_stride = (long long)q * kp * QR_B; ra.mat_stride = kp * QR_B;
+            ra.skip = skip;
             launch_rowblock_dinv(ra, s);
           }
           if (rem > 0) {
@@ -429,6 +457,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
             op.C = c22; op.ldc = kp; op.strideC = kk; op.c_f32 = 1;
             op.D = c22; op.ldd = kp; op.strideD = kk; op.d_f32 = 1;
             op.kind = PK_QR_TRAIL;
+            op.skip = skip;
             if ((e = launch_gemm(op, status, s)) != cudaSuccess) return e;
             GemmOp t;         // Y[:, k0+128:] -= Q_j L21^T
             t.A = Qjpl; t.lda = QR_B; t.strideA = kp * QR_B;
@@ -440,6 +469,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
             t.C = yr; t.ldc = kp; t.strideC = kk; t.c_f32 = 1;
             t.D = yr; t.ldd = kp; t.strideD = kk; t.d_f32 = 1;
             t.kind = PK_QR_TRAIL;
+            t.skip = skip;
             if ((e = launch_gemm(t, status, s)) != cudaSuccess) return e;
           }
         }

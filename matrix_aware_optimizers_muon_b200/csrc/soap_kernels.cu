@@ -1,6 +1,7 @@
 // Elementwise, splitting and small dense kernels of the SOAP path.
 #include "profile.h"
 #include "soap_kernels.cuh"
+#include "chol_block.cuh"
 
 namespace mo {
 
@@ -133,6 +134,33 @@ __global__ void __launch_bounds__(256) damping_kernel(const DampArgs a) {
   if (threadIdx.x == 0) a.delta[b] = part[0] != 0.f ? a.rho * part[0] : 1.0f;
 }
 
+// Largest |C - I| entry per matrix, as the bit pattern of a non-negative
+// float (ordered like the values, so atomicMax on ints is exact); NaN
+// compares above everything.
+__global__ void __launch_bounds__(256) identity_dev_kernel(const float* C, long long ld, long long stride, int k,
+                                                           int* dev) {
+  const int b = blockIdx.y;
+  const float* c = C + (size_t)b * stride;
+  const long long total = (long long)k * k;
+  float m = 0.f;
+  bool nan = false;
+  for (long long e = blockIdx.x * 256LL + threadIdx.x; e < total; e += (long long)gridDim.x * 256) {
+    const long long i = e / k, j = e - i * k;
+    const float d = fabsf(c[i * ld + j] - (i == j ? 1.0f : 0.0f));
+    if (d != d) nan = true;
+    else m = fmaxf(m, d);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  nan = __any_sync(0xffffffffu, nan);
+  if ((threadIdx.x & 31) == 0) atomicMax(dev + b, nan ? 0x7fc00000 : __float_as_int(m));
+}
+
+__global__ void identity_skip_kernel(const int* dev, int count, float tol, int* skip) {
+  const int b = threadIdx.x;
+  if (b < count) skip[b] = dev[b] <= __float_as_int(tol) ? 1 : 0;
+}
+
 __global__ void colnorm_kernel(const float* Y, long long ld, long long stride, int rows, int cols,
                                float* inv_d) {
   const int b = blockIdx.y;
@@ -153,73 +181,44 @@ __global__ void shift_diag_kernel(float* C, long long ld, long long stride, int 
   if (i < n) C[(size_t)b * stride + (long long)i * ld + i] += shift;
 }
 
-// One CTA (256 threads) per matrix: Cholesky of the 128 x 128 diagonal block
-// in shared memory, then the inverse of its lower factor.  Thread (ty, tx)
-// of a 16 x 16 grid owns rows i = ty (mod 16) and columns c = tx (mod 16) of
-// the trailing update.
+// One CTA (256 threads) per matrix: Cholesky of the 128 x 128 diagonal
+// block at (k0, k0) and the inverse of its lower factor (chol_block.cuh).
 __global__ void __launch_bounds__(256) chol_diag_kernel(const float* C, long long ld, long long stride,
-                                                        int k0, float* Dinv, const FlagTable flags) {
+                                                        int k0, float* Dinv, const FlagTable flags,
+                                                        const int* skip) {
+  if (skip && skip[blockIdx.x]) return;
   extern __shared__ float sm[];
-  constexpr int LDS = QR_B + 1;
-  float* A = sm;                      // [128][129]
-  float* X = sm + QR_B * LDS;         // [128][129]
-  __shared__ float piv_inv;
+  float* A = sm;                          // [128][129]
+  float* X = A + CB * CB_LD;              // [128][129]
+  float* T = X + CB * CB_LD;              // [32][97]
+  float* inv_diag = T + 32 * CB_T_LD;     // [128]
   __shared__ int bad;
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
-  const int ty = tid >> 4, tx = tid & 15;
   const float* src = C + (size_t)b * stride + (long long)k0 * ld + k0;
-  for (int e = tid; e < QR_B * QR_B; e += blockDim.x) {
+  for (int e = tid; e < CB * CB; e += blockDim.x) {
     const int r = e >> 7, c = e & 127;
-    A[r * LDS + c] = src[(long long)r * ld + c];
+    A[r * CB_LD + c] = src[(long long)r * ld + c];
   }
   if (tid == 0) bad = 0;
   __syncthreads();
-  for (int j = 0; j < QR_B; ++j) {
-    if (tid == 0) {
-      const float d = A[j * LDS + j];
-      if (!(d > 0.f)) bad = 1;
-      const float sq = sqrtf(d);
-      A[j * LDS + j] = sq;
-      piv_inv = 1.0f / sq;
-    }
-    __syncthreads();
-    if (tid > j && tid < QR_B) A[tid * LDS + j] *= piv_inv;
-    __syncthreads();
-    // A[i][c] -= L[i][j] L[c][j] for j < c <= i
-    const int i0 = j + 1 + ((ty - (j + 1)) & 15);      // first owned row > j
-    for (int i = i0; i < QR_B; i += 16) {
-      const float lij = A[i * LDS + j];
-      const int c0 = j + 1 + ((tx - (j + 1)) & 15);
-      for (int c = c0; c <= i; c += 16) A[i * LDS + c] = fmaf(-lij, A[c * LDS + j], A[i * LDS + c]);
-    }
-    __syncthreads();
-  }
-  // X = L^{-1} by forward substitution, two threads per column (same warp)
-  const int col = tid >> 1, half = tid & 1;
-  for (int i = 0; i < QR_B; ++i) {
-    float s = 0.f;
-    if (col < i)
-      for (int p = col + half; p < i; p += 2) s = fmaf(A[i * LDS + p], X[p * LDS + col], s);
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    const float v = col < i ? -s / A[i * LDS + i] : (col == i ? 1.0f / A[i * LDS + i] : 0.f);
-    if (half == 0) X[i * LDS + col] = v;
-    __syncwarp();
-  }
-  __syncthreads();
+  chol128_factor(A, inv_diag, &bad);
+  chol128_inverse(A, inv_diag, X, T);
   const float nanv = __int_as_float(0x7fc00000);
-  float* dst = Dinv + (size_t)b * QR_B * QR_B;
-  for (int e = tid; e < QR_B * QR_B; e += blockDim.x) {
+  const bool fail = bad != 0;
+  float* dst = Dinv + (size_t)b * CB * CB;
+  for (int e = tid; e < CB * CB; e += blockDim.x) {
     const int r = e >> 7, c = e & 127;
-    dst[e] = bad ? nanv : X[r * LDS + c];
+    dst[e] = fail ? nanv : (c <= r ? X[r * CB_LD + c] : 0.f);
   }
-  if (tid == 0 && bad && flags.f[b] != nullptr) *flags.f[b] = 1;
+  if (tid == 0 && fail && flags.f[b] != nullptr) *flags.f[b] = 1;
 }
 
 // out[r][c] = sum_{p <= c} in[r][p] Dinv[c][p]   (in * Dinv^T, Dinv lower).
 // 64 rows per CTA, 256 threads; thread (ty, tx) computes rows 4 ty .. +3 and
 // columns 8 tx .. +7 from transposed shared copies of the rows and of Dinv.
 __global__ void __launch_bounds__(256) rowblock_kernel(const RowBlockArgs a) {
+  if (a.skip && a.skip[blockIdx.y]) return;
   extern __shared__ float sm[];
   constexpr int LDD = QR_B + 4;        // Dt[p][c] = Dinv[c][p]
   constexpr int LDR = 64 + 4;          // Rt[p][r] = in[r0 + r][p]
@@ -359,6 +358,17 @@ void launch_damping(const DampArgs& a, cudaStream_t s) {
   damping_kernel<<<a.count, 256, 0, s>>>(a);
 }
 
+void launch_identity_check(const float* C, long long ld, long long mat_stride, int count, int k, float tol,
+                           int* dev, int* skip, cudaStream_t s) {
+  ProfScope prof(PK_SOAP_QR, s);
+  cudaMemsetAsync(dev, 0, sizeof(int) * count, s);
+  const long long total = (long long)k * k;
+  long long blocks = (total + 256 * 16 - 1) / (256 * 16);
+  dim3 grid((unsigned)(blocks < 512 ? blocks : 512), count);
+  identity_dev_kernel<<<grid, 256, 0, s>>>(C, ld, mat_stride, k, dev);
+  identity_skip_kernel<<<1, SOAP_MAXB, 0, s>>>(dev, count, tol, skip);
+}
+
 void launch_colnorm(const float* Y, long long ld, long long mat_stride, int count, int rows, int cols,
                     float* inv_d, cudaStream_t s) {
   ProfScope prof(PK_SOAP_QR, s);
@@ -374,15 +384,15 @@ void launch_shift_diag(float* C, long long ld, long long mat_stride, int count, 
 }
 
 void launch_chol_diag(const float* C, long long ld, long long mat_stride, int count, int k0,
-                      float* Dinv, const FlagTable& flags, cudaStream_t s) {
+                      float* Dinv, const FlagTable& flags, cudaStream_t s, const int* skip) {
   ProfScope prof(PK_QR_CHOL, s);
-  const int smem = 2 * QR_B * (QR_B + 1) * 4;
+  const int smem = (2 * CB * CB_LD + 32 * CB_T_LD + CB) * 4;
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     attr = true;
   }
-  chol_diag_kernel<<<count, 256, smem, s>>>(C, ld, mat_stride, k0, Dinv, flags);
+  chol_diag_kernel<<<count, 256, smem, s>>>(C, ld, mat_stride, k0, Dinv, flags, skip);
 }
 
 void launch_rowblock_dinv(const RowBlockArgs& a, cudaStream_t s) {

@@ -76,7 +76,14 @@ struct FlagTable {
 // lower).  A non-positive pivot sets *flag[b] = 1 (if given) and the block
 // inverse to NaN.
 void launch_chol_diag(const float* C, long long ld, long long mat_stride, int count, int k0,
-                      float* Dinv, const FlagTable& flags, cudaStream_t s);
+                      float* Dinv, const FlagTable& flags, cudaStream_t s, const int* skip = nullptr);
+
+// skip[b] = 1 when every entry of the leading k x k block of C[b] (row
+// stride ld) is within tol of the identity, else 0 (NaN never skips).
+// dev is scratch of `count` ints.  One Gram of an already orthonormal basis
+// lets the last CholeskyQR pass be skipped for that matrix.
+void launch_identity_check(const float* C, long long ld, long long mat_stride, int count, int k, float tol,
+                           int* dev, int* skip, cudaStream_t s);
 
 // out = in * Dinv^T for 128-wide row blocks: in/out are rows x 128 fp32
 // views (row stride ld); out may alias in.  Optionally writes the three bf16
@@ -88,6 +95,7 @@ struct RowBlockArgs {
   float* out; long long ld_out, out_stride;         // may be null
   const float* Dinv;                                 // [count][128][128]
   __nv_bfloat16* planes; long long plane_stride, mat_stride;
+  const int* skip = nullptr;                         // per-matrix: leave untouched
 };
 void launch_rowblock_dinv(const RowBlockArgs& a, cudaStream_t s);
 

@@ -184,14 +184,20 @@ def test_cold_start_square_two_sided(ctx):
             assert rel(Q, emu[q]) <= 5e-3, (t, q, rel(Q, emu[q]))
         dW = out["W"] - S["W"]
         if t == 1:
-            # Dbar = M' / |G'| is sign-like at step 1: entries where G' is at
-            # rounding level differ in sign, so only the update's size is
-            # compared.  M' and G' are rotated separately, so where G' is tiny
-            # |Dbar| exceeds 1 in the bf16-operand emulation as well (there by
-            # 0.13 %); the GPU's size is gated against the emulation's.
+            # Dbar = M' / |G'| is sign-like at step 1: where G' is at rounding
+            # level (M' and G' are rotated separately) its entries carry no
+            # information and differ between any two roundings.  So Dbar,
+            # recovered from dW with the GPU's own bases, is compared on the
+            # resolved entries |G'| >= 1e-4 max|G'| (83 % of them here; fp64
+            # and the emulation agree there to 1.5e-4), and the update's
+            # size to 1 %.
+            Dg = out["QL"].T @ (-dW / HP["lr"]) @ out["QR"]
+            mask = np.abs(emu["Gr"]) >= 1e-4 * np.abs(emu["Gr"]).max()
+            assert mask.mean() > 0.5
+            assert rel(Dg[mask], emu["Dbar"][mask]) <= 1e-2, rel(Dg[mask], emu["Dbar"][mask])
             ratio = np.linalg.norm(dW) / (HP["lr"] * np.sqrt(m * n))
             ratio_emu = np.linalg.norm(emu["dW"]) / (HP["lr"] * np.sqrt(m * n))
-            assert abs(ratio - ratio_emu) <= 2e-3, (ratio, ratio_emu)
+            assert abs(ratio - ratio_emu) <= 1e-2, (ratio, ratio_emu)
         else:
             assert rel(dW, emu["dW"]) <= 2e-2, (t, rel(dW, emu["dW"]))
         S = {k: out[k].astype(np.float32) for k in S}

@@ -21,6 +21,30 @@ constexpr int CB = 128;
 constexpr int CB_LD = CB + 1;
 constexpr int CB_T_LD = 97;
 
+// Step J of the warp-level 32 x 32 factorisation (lane i holds row i in
+// r[0..31]); a template so that every register index is a constant.
+template <int J>
+__device__ __forceinline__ void chol32_step(float (&r)[32], int lane, bool& ok, float* inv_diag) {
+  if constexpr (J < 32) {
+    const float d = __shfl_sync(0xffffffffu, r[J], J);
+    ok = ok && (d > 0.f);
+    const float sq = sqrtf(d);
+    const float inv = 1.0f / sq;
+    if (lane == J) {
+      r[J] = sq;
+      inv_diag[J] = inv;
+    } else if (lane > J) {
+      r[J] *= inv;
+    }
+#pragma unroll
+    for (int c = J + 1; c < 32; ++c) {
+      const float lcj = __shfl_sync(0xffffffffu, r[J], c);
+      if (c <= lane) r[c] = fmaf(-r[J], lcj, r[c]);
+    }
+    chol32_step<J + 1>(r, lane, ok, inv_diag);
+  }
+}
+
 __device__ __forceinline__ void chol128_factor(float* A, float* inv_diag, int* bad) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int kb = 0; kb < 4; ++kb) {
@@ -31,21 +55,7 @@ __device__ __forceinline__ void chol128_factor(float* A, float* inv_diag, int* b
 #pragma unroll
       for (int c = 0; c < 32; ++c) r[c] = c <= lane ? A[(b0 + lane) * CB_LD + b0 + c] : 0.f;
       bool ok = true;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float d = __shfl_sync(0xffffffffu, r[j], j);
-        ok = ok && (d > 0.f);
-        const float sq = sqrtf(d);
-        const float inv = 1.0f / sq;
-        if (lane == j) r[j] = sq;
-        else if (lane > j) r[j] *= inv;
-        if (lane == j) inv_diag[b0 + j] = inv;
-#pragma unroll
-        for (int c = j + 1; c < 32; ++c) {
-          const float lcj = __shfl_sync(0xffffffffu, r[j], c);
-          if (c <= lane) r[c] = fmaf(-r[j], lcj, r[c]);
-        }
-      }
+      chol32_step<0>(r, lane, ok, inv_diag + b0);
 #pragma unroll
       for (int c = 0; c < 32; ++c)
         if (c <= lane) A[(b0 + lane) * CB_LD + b0 + c] = r[c];

@@ -488,6 +488,85 @@ def soap_bench(ctx, dev, steps=3, warm=10):
             "gpu_launches": int(sum(v[2] for v in prof.values()) / steps)}
 
 
+def soap_muon_bench(ctx, dev, steps=3, warm=10):
+    """SOAP-Muon on the SOAP workload (the same matrices, sides and gradient
+    stream): SOAP's refresh and rotations plus Newton-Schulz on every matrix."""
+    import torch
+    mats, fill = soap_workload(dev)
+    for d in mats:
+        d["B"] = d.pop("M")
+    fl = 0.0
+    for d in mats:
+        m, n = d["W"].shape
+        f, _ = soap_flops(m, n, "L" in d, "R" in d)
+        fl += f + page_flops(m, n)
+    hp = dict(lr=0.02, weight_decay=0.01, momentum=0.95, beta2=0.95, shampoo_beta=0.9, eps=1e-8)
+    for t in range(1, warm + 1):
+        fill()
+        ctx.soap_muon_step(mats, t, **hp)
+    torch.cuda.synchronize()
+    ctx.profile(True)
+    ctx.profile_read()
+    total = 0.0
+    for t in range(warm + 1, warm + 1 + steps):
+        fill()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        ctx.soap_muon_step(mats, t, reserve=False, **hp)
+        e.record()
+        torch.cuda.synchronize()
+        total += s.elapsed_time(e)
+    prof = ctx.profile_read()
+    ctx.profile(False)
+    ms = total / steps
+    return {"workload": "soap_muon_step on the SOAP matrices (4 x 4096^2 two-sided, 4 x 4096x14336 left side), step 11",
+            "ms": round(ms, 3), "TFLOP/s": round(fl / (ms / 1e3) / 1e12, 1), "flops_per_step": fl,
+            "matrices_per_s": round(len(mats) / (ms / 1e3), 1),
+            "kernels_ms_per_step": {kk: round(v[0] / steps, 3) for kk, v in prof.items() if v[2]},
+            "gpu_launches": int(sum(v[2] for v in prof.values()) / steps),
+            "note": "flops: the SOAP count plus the Newton-Schulz page count of each matrix"}
+
+
+def fwht_last(x):
+    """Unnormalised Walsh-Hadamard transform along the last axis (power of 2)."""
+    import torch
+    n = x.shape[-1]
+    y = x.reshape(-1, n)
+    h = 1
+    while h < n:
+        y = y.view(y.shape[0], n // (2 * h), 2, h)
+        y = torch.stack((y[:, :, 0, :] + y[:, :, 1, :], y[:, :, 0, :] - y[:, :, 1, :]), dim=2)
+        h *= 2
+    return y.reshape(x.shape)
+
+
+def quintic_map(t, steps=5, coeffs=(3.4445, -4.7750, 2.0315)):
+    a, b, c = coeffs
+    for _ in range(steps):
+        t = a * t + b * t ** 3 + c * t ** 5
+    return t
+
+
+def sv_spread(O, d):
+    """Singular-value spread of the NS output of a dyadic known-SVD input
+    G = H diag(d) H / n: H O H / n is diagonal in exact arithmetic with
+    entries sign(d) phi^5(|d| / ||d||); its diagonal gives the output's
+    singular values on the input's own singular vectors."""
+    import numpy as np
+    import torch
+    n = O.shape[0]
+    D = fwht_last(fwht_last(O.double()).T.contiguous()) / n
+    diag = torch.diagonal(D).abs().cpu().numpy()
+    off = float((torch.linalg.matrix_norm(D) ** 2 - (torch.diagonal(D) ** 2).sum()).clamp(min=0).sqrt())
+    exact = quintic_map(np.abs(d) / (np.linalg.norm(d) + 1e-7))
+    q = [0, 5, 50, 95, 100]
+    return {"gpu_percentiles_0_5_50_95_100": [round(float(v), 4) for v in np.percentile(diag, q)],
+            "exact_percentiles_0_5_50_95_100": [round(float(v), 4) for v in np.percentile(exact, q)],
+            "max_abs_dev_from_exact": round(float(np.abs(diag - exact).max()), 5),
+            "offdiag_rel": round(off / float(np.linalg.norm(diag)), 6)}
+
+
 def extras(ctx, dev, args):
     """The other workloads, measured the same way (short runs)."""
     import torch
@@ -540,6 +619,9 @@ def extras(ctx, dev, args):
         reps = 10 if n <= 4096 else 3
         ms = time_steps(lambda: ctx.ns_orthogonalize([Gt], [out], reserve=False), reps, 2)
         sweep[str(n)] = {"ms": round(ms, 3), "TFLOP/s": round(page_flops(n, n) / (ms / 1e3) / 1e12, 1)}
+        ctx.workspace = None
+        d = wl.dyadic_spectrum(wl.rng_of("cfg5", n), n, 1e4)
+        sweep[str(n)]["sv_spread"] = sv_spread(out, d)
         del Gt, out
         ctx.workspace = None
         torch.cuda.empty_cache()
@@ -570,6 +652,9 @@ def extras(ctx, dev, args):
     ctx.workspace = None
     torch.cuda.empty_cache()
     res["soap"] = soap_bench(ctx, dev)
+    ctx.workspace = None
+    torch.cuda.empty_cache()
+    res["soap_muon"] = soap_muon_bench(ctx, dev)
     ctx.workspace = None
     torch.cuda.empty_cache()
     return res

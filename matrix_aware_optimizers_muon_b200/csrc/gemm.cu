@@ -1,6 +1,7 @@
 // Host side of the tcgen05 GEMM: TMA descriptor encoding and launch.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "gemm.cuh"
@@ -48,9 +49,10 @@ int planes_of(const unsigned char* pat, int nseg) {
   return m + 1;
 }
 
-template <int BN, int A_MN, int B_MN>
+template <int BN, int A_MN, int B_MN, bool PAIR = false>
 cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, PAIR>;
+  constexpr int BM_T = PAIR ? 2 * GEMM_BM : GEMM_BM;
   CUtensorMap ta, tb;
   const int nseg = op.nseg > 1 ? op.nseg : 1;
   if (nseg > 8 || (nseg > 1 && op.K % (nseg * GEMM_BK) != 0)) return cudaErrorInvalidValue;
@@ -59,12 +61,14 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   const bool ok_a = A_MN ? encode_bf16_4d(&ta, op.A, kseg, op.M, op.lda, op.strideA, op.batch, op.planeA, pa, 64)
                          : encode_bf16_4d(&ta, op.A, op.M, kseg, op.lda, op.strideA, op.batch, op.planeA, pa, GEMM_BM);
   const bool ok_b = B_MN ? encode_bf16_4d(&tb, op.B, kseg, op.N, op.ldb, op.strideB, op.batch, op.planeB, pb, 64)
-                         : encode_bf16_4d(&tb, op.B, op.N, kseg, op.ldb, op.strideB, op.batch, op.planeB, pb, BN);
+                         : encode_bf16_4d(&tb, op.B, op.N, kseg, op.ldb, op.strideB, op.batch, op.planeB, pb,
+                                          Cfg::BN_LOCAL);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
 
   GemmParams p;
   p.M = op.M; p.N = op.N; p.K = op.K; p.batch = op.batch;
-  p.tiles_m = (op.M + GEMM_BM - 1) / GEMM_BM;
+  p.bm = BM_T;
+  p.tiles_m = (op.M + BM_T - 1) / BM_T;
   p.tiles_n = (op.N + BN - 1) / BN;
   p.sym = op.sym;
   p.alpha = op.alpha; p.beta = op.beta; p.scale = op.scale;
@@ -83,7 +87,7 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   p.d_plane = op.d_plane;
   p.skip = op.skip;
 
-  auto kern = gemm_bf16_kernel<BN, A_MN, B_MN>;
+  auto kern = gemm_bf16_kernel<BN, A_MN, B_MN, PAIR>;
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -96,19 +100,37 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   long long tiles = 0;
   for (int tn = 0; tn < p.tiles_n; ++tn) {
     if (!p.sym) { tiles += p.tiles_m; continue; }
-    const int r = (tn * BN + BN - 1) / GEMM_BM + 1;
+    const int r = (tn * BN + BN - 1) / BM_T + 1;
     tiles += r < p.tiles_m ? r : p.tiles_m;
   }
   p.tiles_per_mat = (int)tiles;
   const long long total = tiles * p.batch;
   if (total >= (1ll << 31)) return cudaErrorInvalidValue;
-  const int grid = (int)(total < device_sm_count() ? total : device_sm_count());
+  // one CTA per SM; a pair per two SMs
+  const long long units = PAIR ? device_sm_count() / 2 : device_sm_count();
+  const int grid = (int)((total < units ? total : units) * (PAIR ? 2 : 1));
   if (grid <= 0) return cudaSuccess;
   // executed tensor-core flops: computed tiles x 128 x BN x padded K x 2
-  const double flops = 2.0 * tiles * p.batch * GEMM_BM * BN * (double)round_up(p.K, GEMM_BK);
+  const double flops = 2.0 * tiles * p.batch * BM_T * BN * (double)round_up(p.K, GEMM_BK);
   ProfScope prof(op.kind, stream, flops);
-  kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
-  return cudaGetLastError();
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(GEMM_THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+  } else {
+    kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
+    return cudaGetLastError();
+  }
 }
 
 }  // namespace
@@ -126,10 +148,31 @@ int device_sm_count() {
   return cache[dev];
 }
 
+namespace {
+// CTA pairs (256 x 256 tiles over two SMs) for products with more than 128
+// rows and N > 128; MO_GEMM_PAIR=0 in the environment selects single-CTA
+// 128 x 256 tiles everywhere.
+bool pairs_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("MO_GEMM_PAIR");
+    return v == nullptr || v[0] != '0';
+  }();
+  return on;
+}
+}  // namespace
+
 cudaError_t launch_gemm(const GemmOp& op, int* status, cudaStream_t stream) {
   if (op.M <= 0 || op.N <= 0 || op.K <= 0 || op.batch <= 0) return cudaSuccess;
   // 128-wide N tiles when N is small, 256 otherwise
   const bool narrow = op.N <= 128;
+  if (!narrow && op.M > GEMM_BM && pairs_enabled()) {
+    switch ((op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0)) {
+      case 0: return launch_t<256, 0, 0, true>(op, status, stream);
+      case 1: return launch_t<256, 0, 1, true>(op, status, stream);
+      case 2: return launch_t<256, 1, 0, true>(op, status, stream);
+      default: return launch_t<256, 1, 1, true>(op, status, stream);
+    }
+  }
   const int sel = (narrow ? 4 : 0) | (op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0);
   switch (sel) {
     case 0: return launch_t<256, 0, 0>(op, status, stream);

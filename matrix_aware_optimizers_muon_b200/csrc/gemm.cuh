@@ -25,6 +25,7 @@ namespace mo {
 struct GemmParams {
   int M, N, K;              // per-matrix problem size
   int batch;                // number of independent matrices
+  int bm;                   // rows of a tile: 128, or 256 for a CTA pair
   int tiles_m, tiles_n;     // tile grid of one matrix
   int tiles_per_mat;        // tiles enumerated per matrix (fewer when sym)
   int sym;                  // symmetric product: upper tiles + mirror stores
@@ -66,12 +67,16 @@ constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;
 constexpr int GEMM_THREADS = 192;
 
-template <int BN>
+// PAIR: a cluster of two CTAs computes a 256 x BN tile with cta_group::2
+// MMAs; each CTA stages its 128 rows of A and BN/2 rows (columns of the
+// product) of B, so a stage is 32 KB instead of 48 KB per SM.
+template <int BN, bool PAIR = false>
 struct GemmCfg {
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
-  static constexpr int B_BYTES = BN * GEMM_BK * 2;
+  static constexpr int BN_LOCAL = PAIR ? BN / 2 : BN;
+  static constexpr int B_BYTES = BN_LOCAL * GEMM_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = PAIR ? 6 : (BN == 256 ? 4 : 6);
   static constexpr int TMEM_COLS = 2 * BN;          // two fp32 accumulators
   static constexpr int BAR_BYTES = 256;
   static constexpr int EPI_BYTES = 4 * 8192;        // per epilogue warp: output block (or C), its transpose
@@ -84,7 +89,7 @@ struct GemmCfg {
 // tm * BM <= tn * BN + BN - 1, so the persistent CTAs get equal shares of
 // computed tiles.
 __device__ __forceinline__ int sym_rows_in_col(const GemmParams& p, int BN, int tn) {
-  const int r = (tn * BN + BN - 1) / GEMM_BM + 1;
+  const int r = (tn * BN + BN - 1) / p.bm + 1;
   return r < p.tiles_m ? r : p.tiles_m;
 }
 
@@ -308,13 +313,15 @@ __device__ __forceinline__ void stage_store32_f32(uint8_t* stg, int lane, const 
   }
 }
 
-template <int BN, int A_MN, int B_MN>
+template <int BN, int A_MN, int B_MN, bool PAIR = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const GemmParams p) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, PAIR>;
   constexpr int STAGES = Cfg::STAGES;
-  constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, BN, A_MN, B_MN);
+  constexpr int BM_T = PAIR ? 2 * GEMM_BM : GEMM_BM;     // rows per tile
+  constexpr int BN_L = Cfg::BN_LOCAL;                     // B rows staged by this CTA
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM_T, BN, A_MN, B_MN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -329,6 +336,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // a pair: rank 0 issues the MMAs; both CTAs load and run the epilogue
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -337,7 +348,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 128);
+      mbar_init(&acc_empty[a], PAIR ? 256 : 128);   // the epilogue threads of every CTA of the tile
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -346,9 +357,15 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
+  if constexpr (PAIR) cluster_sync_all();       // the peer's barriers exist before any remote arrival
   if (warp == 1) {
-    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -364,15 +381,23 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = unit; t < total && ok; t += units) {
         int b, tm, tn;
         if (!gemm_decode(p, BN, t, b, tm, tn)) continue;
+        const int arow = tm * BM_T + (int)rank * GEMM_BM;      // this CTA's rows of A
+        const int bcol = tn * BN + (int)rank * BN_L;           // this CTA's rows of B (columns of D)
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, DEV_TIMEOUT_EMPTY)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          // a pair counts both CTAs' bytes on the even CTA's barrier
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], PAIR ? 2 * Cfg::STAGE_BYTES : Cfg::STAGE_BYTES);
+          const uint32_t full_cl = PAIR ? mapa_shared(&full[stage], 0) : 0u;
+          auto load = [&](void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+            if constexpr (PAIR) tma_load_4d_pair(dst, map, full_cl, c0, c1, c2, c3);
+            else tma_load_4d(dst, map, &full[stage], c0, c1, c2, c3);
+          };
           uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
           uint8_t* sb = sa + Cfg::A_BYTES;
           int kl = kb * GEMM_BK, pa = 0, pb = 0;
@@ -383,17 +408,16 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             pb = p.pat_b[seg];
           }
           if (!A_MN) {
-            tma_load_4d(sa, &tmA, &full[stage], kl, tm * GEMM_BM, b, pa);
+            load(sa, &tmA, kl, arow, b, pa);
           } else {
-            tma_load_4d(sa, &tmA, &full[stage], tm * GEMM_BM, kl, b, pa);
-            tma_load_4d(sa + GEMM_BK * 128, &tmA, &full[stage], tm * GEMM_BM + 64, kl, b, pa);
+            load(sa, &tmA, arow, kl, b, pa);
+            load(sa + GEMM_BK * 128, &tmA, arow + 64, kl, b, pa);
           }
           if (!B_MN) {
-            tma_load_4d(sb, &tmB, &full[stage], kl, tn * BN, b, pb);
+            load(sb, &tmB, kl, bcol, b, pb);
           } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_4d(sb + j * GEMM_BK * 128, &tmB, &full[stage], tn * BN + 64 * j, kl, b, pb);
+            for (int j = 0; j < BN_L / 64; ++j) load(sb + j * GEMM_BK * 128, &tmB, bcol + 64 * j, kl, b, pb);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -402,19 +426,20 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
         }
       }
-      if (!ok) {
+      if (!ok && rank == 0) {
         // let every copy already in flight land before the CTA can exit
+        // (a pair's copies are counted on the even CTA's barriers)
         for (int i = *consumed; i < issued; ++i)
           mbar_wait_drain(&full[i % STAGES], (uint32_t)((i / STAGES) & 1), p.status);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool any = false, ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = unit; t < total && ok; t += units) {
         int b, tm, tn;
         if (!gemm_decode(p, BN, t, b, tm, tn)) continue;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status, DEV_TIMEOUT_ACC_EMPTY)) break;
@@ -434,10 +459,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                      : smem_desc_sw128(sa + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? smem_desc_sw128(sb + k * 2048, GEMM_BK * 128, 1024)
                                      : smem_desc_sw128(sb + k * 32, 16, 1024);
-            tc_mma_f16(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+            if constexpr (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+            else tc_mma_f16(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
           }
           any = true;
-          tc_commit(&empty[stage]);
+          if constexpr (PAIR) tc_commit_pair(&empty[stage], 3);     // frees the stage in both CTAs
+          else tc_commit(&empty[stage]);
           *consumed = *consumed + 1;
           if (++stage == STAGES) {
             stage = 0;
@@ -445,13 +472,15 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
         }
         if (!ok) break;
-        tc_commit(&acc_full[acc]);
+        if constexpr (PAIR) tc_commit_pair(&acc_full[acc], 3);     // both CTAs' epilogues
+        else tc_commit(&acc_full[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       if (any) {
         // every MMA issued by this thread must finish before TMEM is freed
-        tc_commit(drain);
+        if constexpr (PAIR) tc_commit_pair(drain, 1);
+        else tc_commit(drain);
         mbar_wait_drain(drain, 0, p.status);
       }
     }
@@ -467,10 +496,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const bool adam = p.epi == EPI_ADAM;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    // a pair's epilogue threads release the accumulator on the even CTA's barrier
+    const uint32_t acc_empty_cl0 = PAIR ? mapa_shared(&acc_empty[0], 0) : 0u;
+    const uint32_t acc_empty_cl1 = PAIR ? mapa_shared(&acc_empty[1], 0) : 0u;
+    for (int t = unit; t < total; t += units) {
       int b, tm, tn;
       if (!gemm_decode(p, BN, t, b, tm, tn)) continue;
-      const int r = tm * GEMM_BM + row_in_tile;
+      const int r = tm * BM_T + (int)rank * GEMM_BM + row_in_tile;
       const bool row_ok = r < p.M;
       // this matrix's operands, resolved once per tile
       const char* cbase = has_c ? reinterpret_cast<const char*>(c_base(p, b)) : nullptr;
@@ -498,7 +530,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const float alpha = p.alpha * ipow_scale(p.scale, b, p.alpha_pow);
       const float beta = p.beta * ipow_scale(p.scale, b, p.beta_pow);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      const int r0 = tm * GEMM_BM + q * 32;     // this warp's first row
+      const int r0 = tm * BM_T + (int)rank * GEMM_BM + q * 32;     // this warp's first row
       const int n0 = tn * BN;
       // a symmetric product skips the 32 x 32 blocks below the diagonal
       const int cc_begin = p.sym ? (r0 - n0 > 0 ? r0 - n0 : 0) : 0;
@@ -621,17 +653,22 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[acc]);
+      if constexpr (PAIR) mbar_arrive_cluster(acc ? acc_empty_cl1 : acc_empty_cl0);
+      else mbar_arrive(&acc_empty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
   }
 
   __syncthreads();
+  // a pair: the peer's epilogue has read its accumulators and the even CTA's
+  // MMAs (which read the peer's shared memory) have drained
+  if constexpr (PAIR) cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+    else tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
 }
 

@@ -9,6 +9,8 @@
 //  apply     W <- (1 - lr wd) W - lr s O with O the bf16 Newton-Schulz
 //            output (un-oriented), or out = O for the plain orthogonaliser.
 #include "elementwise.cuh"
+#include "runtime.h"
+#include "ptx.cuh"
 #include "profile.h"
 
 namespace mo {
@@ -24,6 +26,8 @@ __device__ __forceinline__ float momentum_update(float g, float b, float beta, i
 __global__ void __launch_bounds__(EW_THREADS) prep_kernel(const EwTable t, const PrepArgs a) {
   __shared__ __align__(16) __nv_bfloat16 xs[EW_TILE][LDS];
   __shared__ float red[EW_THREADS / 32];
+  pdl_wait();
+  pdl_trigger();
 
   const int T = a.tiles_r * a.tiles_c;
   const int j = blockIdx.x / T;
@@ -133,6 +137,8 @@ __global__ void __launch_bounds__(EW_THREADS) prep_kernel(const EwTable t, const
 }
 
 __global__ void finalize_kernel(const EwTable t, const FinalizeArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= a.count) return;
@@ -150,6 +156,8 @@ __global__ void finalize_kernel(const EwTable t, const FinalizeArgs a) {
 
 __global__ void __launch_bounds__(EW_THREADS) apply_kernel(const EwTable t, const ApplyArgs a) {
   __shared__ __align__(16) __nv_bfloat16 xs[EW_TILE][LDS];
+  pdl_wait();
+  pdl_trigger();
 
   const int T = a.tiles_r * a.tiles_c;
   const int j = blockIdx.x / T;
@@ -220,20 +228,20 @@ __global__ void __launch_bounds__(EW_THREADS) apply_kernel(const EwTable t, cons
 void launch_prep(const EwTable& t, const PrepArgs& a, cudaStream_t s) {
   const long long blocks = (long long)a.count * a.tiles_r * a.tiles_c;
   ProfScope prof(PK_PREP, s);
-  if (blocks > 0) prep_kernel<<<(unsigned)blocks, EW_THREADS, 0, s>>>(t, a);
+  if (blocks > 0) launch_pdl(prep_kernel, dim3((unsigned)blocks), dim3(EW_THREADS), 0, s, false, t, a);
 }
 
 void launch_finalize(const EwTable& t, const FinalizeArgs& a, cudaStream_t s) {
   const int warps_per_block = 4;
   const int blocks = (a.count + warps_per_block - 1) / warps_per_block;
   ProfScope prof(PK_NORM, s);
-  if (blocks > 0) finalize_kernel<<<blocks, 32 * warps_per_block, 0, s>>>(t, a);
+  if (blocks > 0) launch_pdl(finalize_kernel, dim3(blocks), dim3(32 * warps_per_block), 0, s, false, t, a);
 }
 
 void launch_apply(const EwTable& t, const ApplyArgs& a, cudaStream_t s) {
   const long long blocks = (long long)a.count * a.tiles_r * a.tiles_c;
   ProfScope prof(PK_APPLY, s);
-  if (blocks > 0) apply_kernel<<<(unsigned)blocks, EW_THREADS, 0, s>>>(t, a);
+  if (blocks > 0) launch_pdl(apply_kernel, dim3((unsigned)blocks), dim3(EW_THREADS), 0, s, false, t, a);
 }
 
 }  // namespace mo

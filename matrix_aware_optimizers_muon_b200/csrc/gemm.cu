@@ -113,24 +113,7 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   // executed tensor-core flops: computed tiles x 128 x BN x padded K x 2
   const double flops = 2.0 * tiles * p.batch * BM_T * BN * (double)round_up(p.K, GEMM_BK);
   ProfScope prof(op.kind, stream, flops);
-  if constexpr (PAIR) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(GEMM_THREADS);
-    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
-  } else {
-    kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
-    return cudaGetLastError();
-  }
+  return launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), Cfg::SMEM_BYTES, stream, PAIR, ta, tb, p);
 }
 
 }  // namespace

@@ -371,6 +371,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the prologue above touched no global memory: from here on the previous
+  // kernel's results are needed
+  pdl_wait();
+  pdl_trigger();
 
   const int total = p.tiles_per_mat * p.batch;
   const int nk = (p.K + GEMM_BK - 1) / GEMM_BK;

@@ -16,6 +16,7 @@
 #include "ns_small.cuh"
 #include "profile.h"
 #include "ptx.cuh"
+#include "runtime.h"
 
 namespace mo {
 
@@ -111,6 +112,8 @@ __global__ void __launch_bounds__(SM_THREADS, 2) ns_small_kernel(const SmallArgs
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();                         // the prologue touched no global memory
+  pdl_trigger();
   const uint32_t sX = smem_u32(X), sA = smem_u32(A), sP = smem_u32(P);
 
   uint32_t mma_phase = 0, work_phase = 0;
@@ -376,6 +379,8 @@ struct TableUpload {
 };
 
 __global__ void upload_tables_kernel(void** dst, int stride, const TableUpload u) {
+  pdl_wait();                         // the previous launch may still read the tables
+  pdl_trigger();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < u.n)
     for (int t = 0; t < 4; ++t) dst[t * stride + i] = const_cast<void*>(u.p[t][i]);
@@ -394,7 +399,7 @@ void launch_upload_tables(void** dst, int n, const void* const* in, const void* 
       u.p[2][i] = out[first + i];
       u.p[3][i] = flag[first + i];
     }
-    upload_tables_kernel<<<(u.n + 127) / 128, 128, 0, s>>>(dst + first, n, u);
+    launch_pdl(upload_tables_kernel, dim3((u.n + 127) / 128), dim3(128), 0, s, false, dst + first, n, u);
   }
 }
 
@@ -416,8 +421,7 @@ cudaError_t launch_ns_small(const SmallArgs& a, int sm_count, cudaStream_t s) {
   const int per_sm = 2 * (smem + 1024) <= 228 * 1024 ? 2 : 1;
   const int grid = a.count < per_sm * sm_count ? a.count : per_sm * sm_count;
   ProfScope prof(PK_SMALL, s, 0.0);
-  ns_small_kernel<<<grid, SM_THREADS, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(ns_small_kernel, dim3(grid), dim3(SM_THREADS), (size_t)smem, s, false, a);
 }
 
 }  // namespace mo

@@ -132,6 +132,17 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// ---------------------------------------------------------------- dependent launches
+// Kernels launched with programmatic stream serialization may start before
+// the previous kernel of the stream has finished.  Every such kernel calls
+// pdl_wait() before its first access to global memory (it returns once the
+// previous grid has completed and its writes are visible), then
+// pdl_trigger() to let the next kernel begin its own prologue.
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- CTA pairs
 // (a cluster of two CTAs sharing tcgen05 MMAs with cta_group::2)
 

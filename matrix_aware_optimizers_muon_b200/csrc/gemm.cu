@@ -146,8 +146,12 @@ bool pairs_enabled() {
 
 cudaError_t launch_gemm(const GemmOp& op, int* status, cudaStream_t stream) {
   if (op.M <= 0 || op.N <= 0 || op.K <= 0 || op.batch <= 0) return cudaSuccess;
-  // 128-wide N tiles when N is small, 256 otherwise
-  const bool narrow = op.N <= 128;
+  // 128-wide N tiles when N is small, or when the product has too few
+  // 128 x 256 tiles to occupy a quarter of the SMs (short launches are bound
+  // by the per-tile epilogue, which narrower tiles spread over more SMs);
+  // 256 otherwise
+  const long long wide_tiles = (long long)((op.M + GEMM_BM - 1) / GEMM_BM) * ((op.N + 255) / 256) * op.batch;
+  const bool narrow = op.N <= 128 || wide_tiles * 4 < device_sm_count();
   if (!narrow && op.M > GEMM_BM && pairs_enabled()) {
     switch ((op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0)) {
       case 0: return launch_t<256, 0, 0, true>(op, status, stream);

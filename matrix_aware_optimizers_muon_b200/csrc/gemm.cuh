@@ -283,6 +283,45 @@ __device__ __forceinline__ void stage_store32(uint8_t* stg, int lane, const floa
   }
 }
 
+// A 32 x 32 block on the diagonal of a symmetric product: each element
+// takes the value computed above the diagonal (its own for c >= r, its
+// mirror's for c < r), so both halves are bit-equal, with the same coalesced
+// row stores.
+__device__ __forceinline__ void stage_store32_diag(uint8_t* stg, int lane, const float (&x)[32], __nv_bfloat16* drow,
+                                                   long long ldd) {
+  uint8_t* srow = stg;
+  uint8_t* scol = stg + 2048;
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(x[8 * u + 2 * j], x[8 * u + 2 * j + 1]);
+      w[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(srow + stg_off(lane, u)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    *reinterpret_cast<__nv_bfloat16*>(scol + stg_off(i, lane >> 3) + ((lane & 7) << 1)) = __float2bfloat16_rn(x[i]);
+  __syncwarp();
+  const int u = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int R = 8 * j + (lane >> 2);
+    uint4 a = *reinterpret_cast<const uint4*>(srow + stg_off(R, u));
+    const uint4 m = *reinterpret_cast<const uint4*>(scol + stg_off(R, u));
+    // columns 8u .. 8u + 7 of row R: below the diagonal (c < R) from the mirror
+    uint16_t* pa = reinterpret_cast<uint16_t*>(&a);
+    const uint16_t* pm = reinterpret_cast<const uint16_t*>(&m);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (8 * u + e < R) pa[e] = pm[e];
+    *reinterpret_cast<uint4*>(drow + (long long)R * ldd + 8 * u) = a;
+  }
+}
+
 // The fp32 version: 128-byte staging rows with the classic 128-byte XOR
 // swizzle (unit ^ row % 8); every store instruction writes four full rows.
 __device__ __forceinline__ uint32_t stg32_off(int row, int unit) {
@@ -310,6 +349,32 @@ __device__ __forceinline__ void stage_store32_f32(uint8_t* stg, int lane, const 
     *reinterpret_cast<float4*>(drow + (long long)R * ldd + 4 * u) = *reinterpret_cast<const float4*>(srow + stg32_off(R, u));
     if (dmir)
       *reinterpret_cast<float4*>(dmir + (long long)R * ldd + 4 * u) = *reinterpret_cast<const float4*>(scol + stg32_off(R, u));
+  }
+}
+
+__device__ __forceinline__ void stage_store32_f32_diag(uint8_t* stg, int lane, const float (&x)[32], float* drow,
+                                                       long long ldd) {
+  uint8_t* srow = stg;
+  uint8_t* scol = stg + 4096;
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    *reinterpret_cast<float4*>(srow + stg32_off(lane, u)) = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    *reinterpret_cast<float*>(scol + stg32_off(i, lane >> 2) + ((lane & 3) << 2)) = x[i];
+  __syncwarp();
+  const int u = lane & 7;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int R = 4 * j + (lane >> 3);
+    float4 a = *reinterpret_cast<const float4*>(srow + stg32_off(R, u));
+    const float4 m = *reinterpret_cast<const float4*>(scol + stg32_off(R, u));
+    if (4 * u + 0 < R) a.x = m.x;
+    if (4 * u + 1 < R) a.y = m.y;
+    if (4 * u + 2 < R) a.z = m.z;
+    if (4 * u + 3 < R) a.w = m.w;
+    *reinterpret_cast<float4*>(drow + (long long)R * ldd + 4 * u) = a;
   }
 }
 
@@ -578,10 +643,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tmem_ld_wait();
         const int c0 = n0 + cc;
         // warp-uniform: every lane holds a full row segment of plain bf16 output
-        const bool blk_full = __all_sync(0xffffffffu, row_ok && c0 + 32 <= p.N) && (!p.sym || c0 >= r0 + 32);
+        const bool all_in = __all_sync(0xffffffffu, row_ok && c0 + 32 <= p.N);
+        const bool blk_full = all_in && (!p.sym || c0 >= r0 + 32);
         const bool fast = plain_bf16 && blk_full;
         const bool fast32 = plain_f32 && blk_full;
-        if (fast || fast32 || cf32 || (row_ok && c0 < p.N)) {
+        const bool diag = p.sym && all_in && c0 == r0 && (plain_bf16 || plain_f32);
+        if (fast || fast32 || diag || cf32 || (row_ok && c0 < p.N)) {
           const bool full = c0 + 32 <= p.N;
           float x[32];
 #pragma unroll
@@ -637,7 +704,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 32; ++i) x[i] = fmaf(beta, c[i], x[i]);
           }
-          if (fast32) {
+          if (diag) {
+            if (plain_f32)
+              stage_store32_f32_diag(stg, lane, x, reinterpret_cast<float*>(dbase) + (long long)r0 * p.ldd + c0, p.ldd);
+            else
+              stage_store32_diag(stg, lane, x, reinterpret_cast<__nv_bfloat16*>(dbase) + (long long)r0 * p.ldd + c0,
+                                 p.ldd);
+          } else if (fast32) {
             float* d32 = reinterpret_cast<float*>(dbase);
             stage_store32_f32(stg, lane, x, d32 + (long long)r0 * p.ldd + c0,
                               p.sym ? d32 + (long long)c0 * p.ldd + r0 : nullptr, p.ldd);

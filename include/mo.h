@@ -29,6 +29,15 @@
  *  - Kernels never wait without a bound: a wait that exceeds two seconds
  *    records a code in the context's device status word, read back with
  *    mo_device_status().
+ *  - The step calls neither allocate nor synchronise, so with the workspace
+ *    attached beforehand a sequence of them can be captured into a CUDA
+ *    graph and replayed.  The library's kernels let their successors start
+ *    their prologue early (programmatic stream serialization); kernels of
+ *    the caller on the same stream are ordered as usual.
+ *  - Environment: MO_GEMM_PAIR=0 makes every tensor-core product use one CTA
+ *    per tile (by default products with more than 128 rows run on pairs of
+ *    CTAs, 256-row tiles); the results are identical up to fp32 rounding of
+ *    the accumulation order.
  *  - One context per host thread.
  */
 #ifndef MO_H_

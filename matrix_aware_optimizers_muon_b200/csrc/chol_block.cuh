@@ -138,25 +138,57 @@ __device__ __forceinline__ void chol128_inverse(const float* A, const float* inv
     for (int i = 0; i < 32; ++i) X[(b0 + i) * CB_LD + b0 + lane] = x[i];
   }
   __syncthreads();
-  // ---- off-diagonal blocks, block row by block row
+  // ---- off-diagonal blocks, block row by block row, in 4 x 4 register tiles
   for (int bi = 1; bi < 4; ++bi) {
     const int r0 = 32 * bi;
-    // T[:, 32 bj + c] = sum_{bj <= k < bi} L[r0 + :, block k] X[block k, 32 bj + c]
-    const int cols = 32 * bi;
-    for (int e = tid; e < 32 * cols; e += blockDim.x) {
-      const int i = e / cols, c = e - i * cols;     // c: column of X (0 .. 32 bi - 1)
-      const int kstart = c & ~31;                    // X[k][c] is zero for k < block of c
-      float acc = 0.f;
-      for (int k = kstart; k < r0; ++k) acc = fmaf(A[(r0 + i) * CB_LD + k], X[k * CB_LD + c], acc);
-      T[i * CB_T_LD + c] = acc;
+    const int cols = 32 * bi;                       // columns 0 .. 32 bi - 1 of X
+    const int tiles = 8 * (cols / 4);               // 4 x 4 tiles of the 32 x cols block
+    // T[i][c] = sum_{block(c) <= k < r0} L[r0 + i][k] X[k][c]  (X[k][c] = 0 above
+    // the diagonal block of column c)
+    for (int t = tid; t < tiles; t += blockDim.x) {
+      const int ti = t / (cols / 4), tc = t - ti * (cols / 4);
+      const int i0 = 4 * ti, c0 = 4 * tc;
+      const int kstart = c0 & ~31;
+      float acc[4][4] = {};
+      for (int k = kstart; k < r0; ++k) {
+        float a[4], x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          a[u] = A[(r0 + i0 + u) * CB_LD + k];
+          x[u] = X[k * CB_LD + c0 + u];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], x[v], acc[u][v]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) T[(i0 + u) * CB_T_LD + c0 + v] = acc[u][v];
     }
     __syncthreads();
-    // X[r0 + i, c] = -sum_{p <= i} X[r0 + i, r0 + p] T[p, c]
-    for (int e = tid; e < 32 * cols; e += blockDim.x) {
-      const int i = e / cols, c = e - i * cols;
-      float acc = 0.f;
-      for (int p = 0; p <= i; ++p) acc = fmaf(X[(r0 + i) * CB_LD + r0 + p], T[p * CB_T_LD + c], acc);
-      X[(r0 + i) * CB_LD + c] = -acc;
+    // X[r0 + i][c] = -sum_{p <= i} X[r0 + i][r0 + p] T[p][c]
+    for (int t = tid; t < tiles; t += blockDim.x) {
+      const int ti = t / (cols / 4), tc = t - ti * (cols / 4);
+      const int i0 = 4 * ti, c0 = 4 * tc;
+      float acc[4][4] = {};
+      for (int p = 0; p < i0 + 4; ++p) {
+        float xr[4], tv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          xr[u] = p <= i0 + u ? X[(r0 + i0 + u) * CB_LD + r0 + p] : 0.f;
+          tv[u] = T[p * CB_T_LD + c0 + u];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(xr[u], tv[v], acc[u][v]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) X[(r0 + i0 + u) * CB_LD + c0 + v] = -acc[u][v];
     }
     __syncthreads();
   }

@@ -3,6 +3,8 @@
 
 #include <cstdlib>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "gemm.cuh"
 #include "profile.h"
@@ -88,14 +90,8 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   p.skip = op.skip;
 
   auto kern = gemm_bf16_kernel<BN, A_MN, B_MN, PAIR>;
-  static int attr_done[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = 1;
-  }
+  cudaError_t ea = ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES);
+  if (ea != cudaSuccess) return ea;
   // tiles enumerated per matrix: all, or those touching the upper triangle
   long long tiles = 0;
   for (int tn = 0; tn < p.tiles_n; ++tn) {
@@ -117,6 +113,19 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
 }
 
 }  // namespace
+
+cudaError_t ensure_smem_attr(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<int, const void*>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({dev, func})) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert({dev, func});
+  return e;
+}
 
 int device_sm_count() {
   static int cache[64] = {0};

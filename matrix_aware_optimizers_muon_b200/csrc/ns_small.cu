@@ -404,15 +404,8 @@ void launch_upload_tables(void** dst, int n, const void* const* in, const void* 
 }
 
 cudaError_t launch_ns_small(const SmallArgs& a, int sm_count, cudaStream_t s) {
-  static int attr_done[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem_bytes(SMALL_MAX_N));
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = 1;
-  }
+  cudaError_t ea = ensure_smem_attr(reinterpret_cast<const void*>(ns_small_kernel), smem_bytes(SMALL_MAX_N));
+  if (ea != cudaSuccess) return ea;
   const int np = a.tall ? a.rows : a.cols;
   const int npad = (np + 63) & ~63;
   const int smem = smem_bytes(npad);

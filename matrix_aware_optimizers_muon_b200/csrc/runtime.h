@@ -8,6 +8,10 @@
 
 namespace mo {
 
+// Allow `bytes` of dynamic shared memory for kernel `func` on the current
+// device: set once per (device, kernel), thread-safe.
+cudaError_t ensure_smem_attr(const void* func, int bytes);
+
 // Launch `kern` with programmatic stream serialization (and, with cluster2,
 // clusters of two CTAs): it may start while the previous kernel of the
 // stream runs, so it must call pdl_wait() before touching global memory.

@@ -1,6 +1,7 @@
 // Elementwise, splitting and small dense kernels of the SOAP path.
 #include "profile.h"
 #include "soap_kernels.cuh"
+#include "runtime.h"
 #include "chol_block.cuh"
 
 namespace mo {
@@ -387,22 +388,16 @@ void launch_chol_diag(const float* C, long long ld, long long mat_stride, int co
                       float* Dinv, const FlagTable& flags, cudaStream_t s, const int* skip) {
   ProfScope prof(PK_QR_CHOL, s);
   const int smem = (2 * CB * CB_LD + 32 * CB_T_LD + CB) * 4;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    attr = true;
-  }
+  // a refused attribute makes the launch below fail; the caller's
+  // cudaGetLastError() reports it
+  (void)ensure_smem_attr(reinterpret_cast<const void*>(chol_diag_kernel), smem);
   chol_diag_kernel<<<count, 256, smem, s>>>(C, ld, mat_stride, k0, Dinv, flags, skip);
 }
 
 void launch_rowblock_dinv(const RowBlockArgs& a, cudaStream_t s) {
   ProfScope prof(PK_QR_ROWBLK, s);
   const int smem = (QR_B * (QR_B + 4) + QR_B * (64 + 4)) * 4;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(rowblock_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    attr = true;
-  }
+  (void)ensure_smem_attr(reinterpret_cast<const void*>(rowblock_kernel), smem);
   dim3 grid((a.rows + 63) / 64, a.count);
   rowblock_kernel<<<grid, 256, smem, s>>>(a);
 }

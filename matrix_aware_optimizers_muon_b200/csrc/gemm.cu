@@ -2,6 +2,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -45,6 +46,24 @@ bool encode_bf16_4d(CUtensorMap* map, const void* ptr, long long rows, long long
   return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor map over `batch` matrices rows x cols (row stride ld,
+// matrix stride bstride, elements) read in 32 x 32 boxes with the 64-byte
+// swizzle (the epilogue's C blocks).
+bool encode_bf16_c(CUtensorMap* map, const void* ptr, long long rows, long long cols, long long ld,
+                   long long bstride, int batch) {
+  std::call_once(g_encode_once, load_encode_fn);
+  if (g_encode == nullptr) return false;
+  const long long bs = batch > 1 ? bstride : rows * ld;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)(bs * 2)};
+  cuuint32_t box[3] = {32u, 32u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int planes_of(const unsigned char* pat, int nseg) {
   int m = 0;
   for (int i = 0; i < nseg; ++i) m = pat[i] > m ? pat[i] : m;
@@ -55,7 +74,8 @@ template <int BN, int A_MN, int B_MN, bool PAIR = false>
 cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   using Cfg = GemmCfg<BN, PAIR>;
   constexpr int BM_T = PAIR ? 2 * GEMM_BM : GEMM_BM;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
+  std::memset(&tc, 0, sizeof(tc));
   const int nseg = op.nseg > 1 ? op.nseg : 1;
   if (nseg > 8 || (nseg > 1 && op.K % (nseg * GEMM_BK) != 0)) return cudaErrorInvalidValue;
   const long long kseg = op.K / nseg;
@@ -88,6 +108,14 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   p.d_split = op.d_split;
   p.d_plane = op.d_plane;
   p.skip = op.skip;
+  // a strided bf16 C of the plain epilogue is read by TMA
+  p.c_tma = 0;
+  if (op.C != nullptr && op.c_tab == nullptr && !op.c_f32 && op.epi == 0 && !op.d_f32 && !op.d_split &&
+      (op.batch == 1 || op.strideC % 8 == 0) && op.ldc % 8 == 0 &&
+      (reinterpret_cast<uintptr_t>(op.C) & 15) == 0) {
+    if (!encode_bf16_c(&tc, op.C, op.M, op.N, op.ldc, op.strideC, op.batch)) return cudaErrorInvalidValue;
+    p.c_tma = 1;
+  }
 
   auto kern = gemm_bf16_kernel<BN, A_MN, B_MN, PAIR>;
   cudaError_t ea = ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES);
@@ -109,7 +137,7 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   // executed tensor-core flops: computed tiles x 128 x BN x padded K x 2
   const double flops = 2.0 * tiles * p.batch * BM_T * BN * (double)round_up(p.K, GEMM_BK);
   ProfScope prof(op.kind, stream, flops);
-  return launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), Cfg::SMEM_BYTES, stream, PAIR, ta, tb, p);
+  return launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), Cfg::SMEM_BYTES, stream, PAIR, ta, tb, tc, p);
 }
 
 }  // namespace

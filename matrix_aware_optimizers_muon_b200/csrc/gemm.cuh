@@ -59,6 +59,8 @@ struct GemmParams {
   // optional per-matrix flags (device): matrices with skip[b] != 0 are left
   // untouched (every role of the kernel skips their tiles)
   const int* skip;
+  // bf16 C read by TMA (tensor map tmC, 32 x 32 boxes, 64-byte swizzle)
+  int c_tma;
 };
 
 enum { EPI_AXPBY = 0, EPI_ADAM = 1 };
@@ -78,7 +80,7 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = PAIR ? 6 : (BN == 256 ? 4 : 6);
   static constexpr int TMEM_COLS = 2 * BN;          // two fp32 accumulators
-  static constexpr int BAR_BYTES = 256;
+  static constexpr int BAR_BYTES = 1024;            // mbarriers; keeps the epilogue stage 1 KB aligned
   static constexpr int EPI_BYTES = 4 * 8192;        // per epilogue warp: output block (or C), its transpose
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + EPI_BYTES + 1024;
 };
@@ -381,7 +383,7 @@ __device__ __forceinline__ void stage_store32_f32_diag(uint8_t* stg, int lane, c
 template <int BN, int A_MN, int B_MN, bool PAIR = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const GemmParams p) {
+                 const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   using Cfg = GemmCfg<BN, PAIR>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int BM_T = PAIR ? 2 * GEMM_BM : GEMM_BM;     // rows per tile
@@ -395,7 +397,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* cbar = drain + 1;                 // [4 warps][2]: C blocks read by TMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* consumed = abort_flag + 1;
 
@@ -416,6 +419,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(&acc_empty[a], PAIR ? 256 : 128);   // the epilogue threads of every CTA of the tile
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&cbar[i], 1);
     *abort_flag = 0;
     *consumed = 0;
     fence_barrier_init();
@@ -559,6 +563,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int row_in_tile = q * 32 + lane;
     uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES + q * 8192;
     uint8_t* stc = stg + 4096;              // staged 32 x 32 bf16 block of C
+    // two 2 KB buffers (at stg + 4096 and + 6144, 1 KB aligned) for C blocks
+    // that TMA writes in the 64-byte-swizzled layout stg_off() reads
+    uint8_t* cbuf0 = stg + 4096;           // buffer bi at cbuf0 + 2048 bi
+    uint64_t* cb = cbar + 2 * q;
+    uint32_t cph = 0u;                      // bit bi: phase of buffer bi
+    uint32_t cpend = 0u;                    // bit bi: a copy into buffer bi is in flight
     const bool plain_bf16 = !p.d_f32 && !p.d_split;
     const bool plain_f32 = p.d_f32 && !p.d_split;
     const bool has_c = p.C != nullptr || p.c_tab != nullptr;
@@ -592,6 +602,23 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           for (int off = 0; off < nn * 4; off += 128) prefetch_l2(row + off);
         }
       }
+      // bf16 C of full blocks comes by TMA, the first two 32-column blocks
+      // requested now so that they arrive while the main loop runs
+      const int r0 = tm * BM_T + (int)rank * GEMM_BM + q * 32;     // this warp's first row
+      const int n0 = tn * BN;
+      // a symmetric product skips the 32 x 32 blocks below the diagonal
+      const int cc_begin = p.sym ? (r0 - n0 > 0 ? r0 - n0 : 0) : 0;
+      const bool ctma = p.c_tma && !adam && plain_bf16 && n0 + BN <= p.N && __all_sync(0xffffffffu, row_ok);
+      auto issue_c = [&](int bi, int cc) {
+        mbar_arrive_expect_tx(&cb[bi], 32 * 32 * 2);
+        tma_load_3d(cbuf0 + 2048 * bi, &tmC, &cb[bi], n0 + cc, r0, b);
+        cpend |= 1u << bi;
+      };
+      if (ctma && lane == 0) {
+        fence_proxy_async_smem();              // earlier reads of the buffers come first
+        if (cc_begin < BN) issue_c(0, cc_begin);
+        if (cc_begin + 32 < BN) issue_c(1, cc_begin + 32);
+      }
       // warp-uniform: tcgen05.ld below must be executed by all 32 lanes
       const bool ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status, DEV_TIMEOUT_ACC_FULL);
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -599,14 +626,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const float alpha = p.alpha * ipow_scale(p.scale, b, p.alpha_pow);
       const float beta = p.beta * ipow_scale(p.scale, b, p.beta_pow);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      const int r0 = tm * BM_T + (int)rank * GEMM_BM + q * 32;     // this warp's first row
-      const int n0 = tn * BN;
-      // a symmetric product skips the 32 x 32 blocks below the diagonal
-      const int cc_begin = p.sym ? (r0 - n0 > 0 ? r0 - n0 : 0) : 0;
-      // bf16 C for full blocks: loaded one block ahead with coalesced
-      // 16-byte loads (eight 64-byte rows per instruction), then transposed
-      // to row-per-lane through shared memory
-      const bool cpre = has_c && !adam && !p.c_f32 && plain_bf16 && n0 + BN <= p.N &&
+      // otherwise bf16 C of full blocks (pointer tables): loaded one block
+      // ahead with coalesced 16-byte loads (eight 64-byte rows per
+      // instruction), then transposed to row-per-lane through shared memory
+      const bool cpre = !ctma && has_c && !adam && !p.c_f32 && plain_bf16 && n0 + BN <= p.N &&
                         __all_sync(0xffffffffu, row_ok);
       const __nv_bfloat16* c16 = reinterpret_cast<const __nv_bfloat16*>(cbase);
       uint4 cnext[4];
@@ -623,8 +646,9 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const bool cf32 = has_c && !adam && p.c_f32 && !p.d_split && n0 + BN <= p.N &&
                         __all_sync(0xffffffffu, row_ok);
       const float* c32 = reinterpret_cast<const float*>(cbase);
+      int kk = 0;                                // 32-column blocks done in this tile
 #pragma unroll 1
-      for (int cc = cc_begin; cc < BN; cc += 32) {
+      for (int cc = cc_begin; cc < BN; cc += 32, ++kk) {
         uint4 ccur[4];
         if (cpre) {
 #pragma unroll
@@ -681,6 +705,27 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
               x[4 * u + 2] = fmaf(beta, w.z, x[4 * u + 2]);
               x[4 * u + 3] = fmaf(beta, w.w, x[4 * u + 3]);
             }
+          } else if (ctma) {
+            const int bi = kk & 1;
+            mbar_wait(&cb[bi], (cph >> bi) & 1u, abort_flag, p.status, DEV_TIMEOUT_ACC_FULL);
+            cph ^= 1u << bi;
+            cpend &= ~(1u << bi);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint4 w = *reinterpret_cast<const uint4*>(cbuf0 + 2048 * bi + stg_off(lane, u));
+              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ws[j]));
+                x[8 * u + 2 * j] = fmaf(beta, f.x, x[8 * u + 2 * j]);
+                x[8 * u + 2 * j + 1] = fmaf(beta, f.y, x[8 * u + 2 * j + 1]);
+              }
+            }
+            __syncwarp();                 // every lane has read the buffer
+            if (lane == 0) {
+              fence_proxy_async_smem();
+              if (cc + 64 < BN) issue_c(bi, cc + 64);
+            }
           } else if (cpre) {
             __syncwarp();                 // the previous block's reads of stc are done
 #pragma unroll
@@ -735,6 +780,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    // C blocks requested for a tile that was abandoned must land before exit
+    if (lane == 0)
+      for (int bi = 0; bi < 2; ++bi)
+        if ((cpend >> bi) & 1u) mbar_wait_drain(&cb[bi], (cph >> bi) & 1u, p.status);
   }
 
   __syncthreads();

@@ -132,6 +132,12 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Order this thread's earlier generic-proxy accesses of shared memory before
+// later async-proxy (TMA, tcgen05) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- dependent launches
 // Kernels launched with programmatic stream serialization may start before
 // the previous kernel of the stream has finished.  Every such kernel calls

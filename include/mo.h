@@ -59,7 +59,7 @@ extern "C" {
 typedef enum {
   MO_OK = 0,
   MO_ERR_INVALID_ARG = -1,   /* null pointer, bad size or hyperparameter */
-  MO_ERR_UNSUPPORTED = -2,   /* valid request this build cannot run */
+  MO_ERR_UNSUPPORTED = -2,   /* valid request the library does not support */
   MO_ERR_NO_WORKSPACE = -3,  /* no workspace attached, or too small */
   MO_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
   MO_ERR_DEVICE = -5         /* the device status word reports a timeout */

@@ -34,10 +34,10 @@
  *    graph and replayed.  The library's kernels let their successors start
  *    their prologue early (programmatic stream serialization); kernels of
  *    the caller on the same stream are ordered as usual.
- *  - Environment: MO_GEMM_PAIR=0 makes every tensor-core product use one CTA
- *    per tile (by default products with more than 128 rows run on pairs of
- *    CTAs, 256-row tiles); the results are identical up to fp32 rounding of
- *    the accumulation order.
+ *  - Environment: MO_GEMM_PAIR=1 runs tensor-core products with more than
+ *    128 rows on pairs of CTAs (256-row tiles) instead of one CTA per
+ *    128-row tile; the results are identical up to fp32 rounding of the
+ *    accumulation order.
  *  - One context per host thread.
  */
 #ifndef MO_H_

@@ -49,7 +49,7 @@ CASES = [
     (128, 520, 72, 1, 1, 1),
     (96, 96, 256, 5, 0, 1),
     (1, 64, 64, 2, 0, 0),
-    # more than 128 rows and N > 128: 256-row tiles on CTA pairs
+    # more than 128 rows and N > 128 (256-row tiles when CTA pairs are on)
     (300, 264, 200, 2, 1, 1),
     (640, 768, 512, 3, 0, 1),
     (520, 1000, 136, 1, 1, 0),

@@ -1,7 +1,7 @@
-"""The single-CTA tiles of the tensor-core GEMM, which CTA pairs replace by
-default for products with more than 128 rows: the GEMM unit tests and the
-Muon parity tests rerun in a child process with MO_GEMM_PAIR=0 (the switch is
-read once per process)."""
+"""The CTA-pair tiles of the tensor-core GEMM (256-row tiles over two SMs,
+enabled with MO_GEMM_PAIR=1): the GEMM unit tests and Muon / SOAP parity
+tests rerun in a child process with the switch set (it is read once per
+process)."""
 import os
 import subprocess
 import sys
@@ -13,8 +13,8 @@ pytestmark = pytest.mark.gpu
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
-def test_single_cta_tiles():
-    env = dict(os.environ, MO_GEMM_PAIR="0")
+def test_cta_pair_tiles():
+    env = dict(os.environ, MO_GEMM_PAIR="1")
     cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
            os.path.join(HERE, "test_gpu_gemm.py"),
            os.path.join(HERE, "test_gpu_muon.py") + "::test_dense_gpt_mini_buckets",

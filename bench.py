@@ -94,7 +94,7 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, mx, reasons = [], [], set()
+        sm, mx, pw, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
@@ -106,14 +106,21 @@ class ClockSampler:
                     mx.append(float(parts[2]))
                 except ValueError:
                     continue
+                try:
+                    pw.append(float(parts[3]))
+                except ValueError:
+                    pass
                 for nm, v in zip(names, parts[5:9]):
                     if v.lower().startswith("active"):
                         reasons.add(nm)
         os.unlink(self.path)
         if not sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+               "samples": len(sm)}
+        if pw:
+            out["power_w"] = statistics.median(pw)
+        return out
 
 
 def max_over_ranks(x, world, device="cpu"):
@@ -732,6 +739,81 @@ def run_soap_only(args, world, rank, local):
             "soap": res}
 
 
+def gemm_vs_cublas(args, local):
+    """The Newton-Schulz products of the dense-GPT 4096 x 14336 bucket (and a
+    square 8192^3 product) through this library's GEMM and through cuBLAS
+    (torch.bmm / torch.matmul) on the same bf16 operands.  Each phase runs
+    back to back for --seconds after a 1 s warm-up, so both sides are timed
+    at the clock the 1 kW power cap settles them at; the SM clock and board
+    power are sampled per phase.  --once runs each product once on a batch
+    of 3 (a small case for counter captures)."""
+    import torch
+    from matrix_aware_optimizers_muon_b200 import Context
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ctx = Context(local)
+    gen = torch.Generator(device=dev).manual_seed(5)
+    bt = 3 if args.once else 96
+    m, n = 4096, 14336
+    X = (torch.randn(bt, m, n, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+    P = (torch.randn(bt, m, m, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+    P = ((P + P.mT) * 0.5).contiguous()
+    Y = torch.empty_like(X)
+    A = torch.empty(bt, m, m, device=dev, dtype=torch.bfloat16)
+    s8 = 8192
+    A8 = (torch.randn(s8, s8, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+    B8 = (torch.randn(s8, s8, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+    D8 = torch.empty(s8, s8, device=dev, dtype=torch.bfloat16)
+    f_prod = 2.0 * m * m * n * bt                   # Gram or update, full product
+    ops = [
+        ("update aX + PX", "ours", f_prod,
+         lambda: ctx.gemm_bf16(P, X, Y, M=m, N=n, K=m, batch=bt, b_mn=True, alpha=1.0, beta=3.4445, C=X)),
+        ("update aX + PX", "cublas", f_prod, lambda: torch.bmm(P, X, out=Y)),
+        ("Gram X X^T", "ours (symmetric)", f_prod,
+         lambda: ctx.gemm_bf16(X, X, A, M=m, N=m, K=n, batch=bt, sym=True)),
+        ("Gram X X^T", "ours (full)", f_prod, lambda: ctx.gemm_bf16(X, X, A, M=m, N=m, K=n, batch=bt)),
+        ("Gram X X^T", "cublas", f_prod, lambda: torch.bmm(X, X.mT, out=A)),
+        ("8192^3", "ours", 2.0 * s8 ** 3, lambda: ctx.gemm_bf16(A8, B8, D8, M=s8, N=s8, K=s8, b_mn=True)),
+        ("8192^3", "cublas", 2.0 * s8 ** 3, lambda: torch.matmul(A8, B8, out=D8)),
+    ]
+    torch.cuda.synchronize()
+    if args.once:
+        for _, _, _, fn in ops:
+            fn()
+        torch.cuda.synchronize()
+        return {"workload": "gemm-vs-cublas once (batch 3)", "device_status": ctx.device_status()}
+    rows = []
+    for _rep in range(2):
+        for prod, impl, flops, fn in ops:
+            t0 = time.time()
+            while time.time() - t0 < 1.0:
+                for _ in range(4):
+                    fn()
+                torch.cuda.synchronize()
+            clk = ClockSampler(local)
+            clk.start()
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 0
+            t0 = time.time()
+            ev0.record()
+            while time.time() - t0 < args.seconds:
+                for _ in range(4):
+                    fn()
+                reps += 4
+                torch.cuda.synchronize()
+            ev1.record()
+            torch.cuda.synchronize()
+            c = clk.stop() or {}
+            ms = ev0.elapsed_time(ev1) / reps
+            tf = flops / (ms * 1e-3) / 1e12
+            rows.append({"product": prod, "impl": impl, "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                         "sm_mhz": c.get("sm_mhz"), "power_w": c.get("power_w"),
+                         "TFLOP/s per GHz": round(tf / c["sm_mhz"] * 1e3, 1) if c.get("sm_mhz") else None,
+                         "reasons": c.get("reasons")})
+    return {"workload": f"gemm-vs-cublas sustained, batch {bt} of 4096 x 14336 (flops: full products)",
+            "phases": rows, "device_status": ctx.device_status()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -742,8 +824,11 @@ def main():
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--workload", choices=["muon", "soap"], default="muon",
-                    help="muon: the dense-GPT Muon step (the benchmark line); soap: the SOAP step alone")
+    ap.add_argument("--workload", choices=["muon", "soap", "gemm-vs-cublas"], default="muon",
+                    help="muon: the dense-GPT Muon step (the benchmark line); soap: the SOAP step alone; "
+                         "gemm-vs-cublas: the NS products against cuBLAS at the sustained clock")
+    ap.add_argument("--seconds", type=float, default=3.0, help="gemm-vs-cublas: timed seconds per phase")
+    ap.add_argument("--once", action="store_true", help="gemm-vs-cublas: each product once, batch 3")
     ap.add_argument("--layers", type=int, default=32,
                     help="dense-GPT layers (32 = the benchmark workload; fewer for small profiling cases)")
     args = ap.parse_args()
@@ -752,6 +837,8 @@ def main():
         out = run_reference(args, world, rank)
     elif args.workload == "soap":
         out = run_soap_only(args, world, rank, local)
+    elif args.workload == "gemm-vs-cublas":
+        out = gemm_vs_cublas(args, local)
     else:
         out = run_ours(args, world, rank, local)
     if rank == 0 and out is not None:

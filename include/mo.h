@@ -307,7 +307,11 @@ MO_API mo_status mo_soap_muon_workspace_bytes(mo_ctx* ctx, const mo_soap_muon_ma
  * elements and 16-byte aligned bases.  C and D are bf16 or fp32 (c_f32,
  * d_f32); C may be NULL or alias D.  With sym set the product must be
  * symmetric (M == N): only tiles that touch the upper triangle are computed
- * and each upper element is also written to its mirror position. */
+ * and each upper element is also written to its mirror position.  band sets
+ * the order in which the persistent CTAs take tiles: 0 lets the library
+ * choose (column order, or bands of row tiles when A overflows L2); n > 0
+ * forces bands of n row tiles, each band taken column by column.  The order
+ * changes no result.  band < 0 is MO_ERR_INVALID_ARG. */
 typedef struct {
   const void* A; int64_t lda, strideA; int a_mn;
   const void* B; int64_t ldb, strideB; int b_mn;
@@ -316,6 +320,7 @@ typedef struct {
   const float* scale; int alpha_pow, beta_pow;   /* scale may be NULL */
   const void* C; int64_t ldc, strideC; int c_f32;
   void* D; int64_t ldd, strideD; int d_f32;
+  int band;
 } mo_gemm_desc;
 
 MO_API mo_status mo_gemm_bf16(mo_ctx* ctx, const mo_gemm_desc* desc, void* stream);

@@ -219,7 +219,7 @@ class Context:
     def gemm_bf16(self, A, B, D, *, M, N, K, batch=1, a_mn=False, b_mn=False, sym=False,
                   alpha=1.0, beta=0.0, C=None, scale=None, alpha_pow=0, beta_pow=0,
                   lda=None, ldb=None, ldc=None, ldd=None, strideA=None, strideB=None,
-                  strideC=None, strideD=None, stream=None):
+                  strideC=None, strideD=None, band=0, stream=None):
         """Batched bf16 tensor-core GEMM with the fused epilogue (see mo.h)."""
         import torch
 
@@ -241,6 +241,7 @@ class Context:
             d.c_f32 = int(C.dtype == torch.float32)
         d.D, d.ldd, d.strideD = D.data_ptr(), ldd or ld_of(D), strideD or stride_of(D)
         d.d_f32 = int(D.dtype == torch.float32)
+        d.band = band
         if self.workspace is None:
             self.attach_workspace(4096, stream)
         self._check(self.lib.mo_gemm_bf16(self.handle, byref(d), self._stream(stream)))

@@ -77,7 +77,8 @@ class GemmDesc(ctypes.Structure):
                 ("alpha", c_float), ("beta", c_float),
                 ("scale", c_void_p), ("alpha_pow", c_int), ("beta_pow", c_int),
                 ("C", c_void_p), ("ldc", c_int64), ("strideC", c_int64), ("c_f32", c_int),
-                ("D", c_void_p), ("ldd", c_int64), ("strideD", c_int64), ("d_f32", c_int)]
+                ("D", c_void_p), ("ldd", c_int64), ("strideD", c_int64), ("d_f32", c_int),
+                ("band", c_int)]
 
 
 # name -> (restype, argtypes); every entry point declared in include/mo.h

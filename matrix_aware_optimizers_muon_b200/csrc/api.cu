@@ -426,6 +426,7 @@ mo_status mo_gemm_bf16(mo_ctx* ctx, const mo_gemm_desc* d, void* stream) {
     return fail(ctx, MO_ERR_INVALID_ARG, "mo_gemm_bf16: C/D need 16-byte aligned bases and rows");
   if (d->alpha_pow < 0 || d->alpha_pow > 2 || d->beta_pow < 0 || d->beta_pow > 2)
     return fail(ctx, MO_ERR_INVALID_ARG, "mo_gemm_bf16: alpha_pow and beta_pow must be 0, 1 or 2");
+  if (d->band < 0) return fail(ctx, MO_ERR_INVALID_ARG, "mo_gemm_bf16: band must be >= 0");
   if (ctx->ws == nullptr) return fail(ctx, MO_ERR_NO_WORKSPACE, "mo_gemm_bf16: no workspace attached (status word)");
   mo_status st = enter(ctx);
   if (st != MO_OK) return st;
@@ -437,6 +438,7 @@ mo_status mo_gemm_bf16(mo_ctx* ctx, const mo_gemm_desc* d, void* stream) {
   op.alpha_pow = d->alpha_pow; op.beta_pow = d->beta_pow;
   op.C = d->C; op.ldc = d->ldc; op.strideC = d->strideC; op.c_f32 = d->c_f32;
   op.D = d->D; op.ldd = d->ldd; op.strideD = d->strideD; op.d_f32 = d->d_f32;
+  op.band = d->band;
   cudaError_t e = mo::launch_gemm(op, reinterpret_cast<int*>(ctx->ws), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(ctx, e, "mo_gemm_bf16");
   return MO_OK;

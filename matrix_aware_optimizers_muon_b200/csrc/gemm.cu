@@ -70,6 +70,30 @@ int planes_of(const unsigned char* pat, int nseg) {
   return m + 1;
 }
 
+// Row tiles per band of the tile order (see gemm_decode).  The plain column
+// order re-reads the A panel of a matrix from DRAM once per wave of tiles
+// when the panel does not fit in L2; bands of G row tiles read A once and
+// the B panel once per band.  Bands are used when the estimate of DRAM bytes
+// read drops by more than a third (symmetric products sweep about half of
+// the columns per band and of the rows per wave).
+int choose_band(int bm, int tiles_m, long long M, long long N, long long kseg, int pa, int pb, bool sym,
+                long long tiles_per_mat, long long units) {
+  const double budget = 48.0 * 1024 * 1024;         // A rows kept in the 126 MB L2
+  const double row_bytes = (double)bm * kseg * pa * 2.0;
+  const double a_bytes = (double)M * kseg * pa * 2.0;
+  const double b_bytes = (double)N * kseg * pb * 2.0;
+  if (a_bytes <= budget) return tiles_m;
+  int g = (int)(budget / row_bytes);
+  if (g < 1) g = 1;
+  if (g >= tiles_m) return tiles_m;
+  const int nb = (tiles_m + g - 1) / g;
+  const double waves = (double)tiles_per_mat / (double)units;
+  const double rereads = sym ? waves / 2 : waves;
+  const double plain = b_bytes + a_bytes * (rereads > 1.0 ? rereads : 1.0);
+  const double banded = a_bytes + b_bytes * (sym ? (nb + 1) / 2.0 : (double)nb);
+  return banded * 1.5 < plain ? g : tiles_m;
+}
+
 template <int BN, int A_MN, int B_MN, bool PAIR = false>
 cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   using Cfg = GemmCfg<BN, PAIR>;
@@ -132,6 +156,8 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   if (total >= (1ll << 31)) return cudaErrorInvalidValue;
   // one CTA per SM; a pair per two SMs
   const long long units = PAIR ? device_sm_count() / 2 : device_sm_count();
+  p.band = op.band > 0 ? op.band
+                       : choose_band(BM_T, p.tiles_m, op.M, op.N, kseg, pa, pb, op.sym != 0, tiles, units);
   const int grid = (int)((total < units ? total : units) * (PAIR ? 2 : 1));
   if (grid <= 0) return cudaSuccess;
   // executed tensor-core flops: computed tiles x 128 x BN x padded K x 2

@@ -61,6 +61,9 @@ struct GemmParams {
   const int* skip;
   // bf16 C read by TMA (tensor map tmC, 32 x 32 boxes, 64-byte swizzle)
   int c_tma;
+  // tile order: bands of `band` row tiles, each band column by column; a
+  // band of tiles_m rows (or more) is the plain column order
+  int band;
 };
 
 enum { EPI_AXPBY = 0, EPI_ADAM = 1 };
@@ -88,11 +91,34 @@ struct GemmCfg {
 // Tiles of one matrix in column order (M fastest, so the CTAs in flight
 // share B columns in L2).  For a symmetric product only the tiles touching
 // the upper triangle are enumerated: column tn holds rows tm with
-// tm * BM <= tn * BN + BN - 1, so the persistent CTAs get equal shares of
-// computed tiles.
+// tm * BM <= tn * BN + BN - 1, i.e. tm < q (tn + 1) with q = BN / BM (1 or
+// 2), so the persistent CTAs get equal shares of computed tiles.
+//
+// When the A panel of a matrix does not fit in L2 the host may split the
+// rows into bands of p.band tiles: band after band, each in column order
+// (rows fastest), so that a band's A rows stay in L2 while the B columns
+// stream past them once per band.
 __device__ __forceinline__ int sym_rows_in_col(const GemmParams& p, int BN, int tn) {
   const int r = (tn * BN + BN - 1) / p.bm + 1;
   return r < p.tiles_m ? r : p.tiles_m;
+}
+
+// Upper-triangle tiles of a symmetric product in the band of rows
+// [r0, r0 + rows): column tn holds clamp(q (tn + 1) - r0, 0, rows) of them.
+// Columns before a hold none, columns from f on hold all `rows`, the ones
+// in between a ramp; returned with a and f (both clamped to tiles_n).
+__device__ __forceinline__ long long sym_band_tiles(const GemmParams& p, int q, int r0, int rows, int& a,
+                                                    int& f) {
+  const int tn_all = p.tiles_n;
+  a = r0 / q;
+  f = (r0 + rows + q - 1) / q - 1;
+  if (a > tn_all) a = tn_all;
+  if (f > tn_all) f = tn_all;
+  if (f < a) f = a;
+  // sum over tn in [a, f) of q (tn + 1) - r0, then full columns
+  const long long ramp = (long long)q * ((long long)f * (f + 1) - (long long)a * (a + 1)) / 2 -
+                         (long long)r0 * (f - a);
+  return ramp + (long long)rows * (tn_all - f);
 }
 
 __device__ __forceinline__ bool gemm_decode(const GemmParams& p, int BN, int t, int& b, int& tm,
@@ -100,6 +126,42 @@ __device__ __forceinline__ bool gemm_decode(const GemmParams& p, int BN, int t, 
   b = t / p.tiles_per_mat;
   if (p.skip && p.skip[b]) return false;
   int u = t - b * p.tiles_per_mat;
+  if (p.band < p.tiles_m) {
+    const int G = p.band;
+    if (!p.sym) {
+      const int per_band = G * p.tiles_n;
+      const int k = u / per_band;
+      const int r0 = k * G;
+      const int rows = p.tiles_m - r0 < G ? p.tiles_m - r0 : G;
+      const int v = u - k * per_band;
+      tn = v / rows;
+      tm = r0 + (v - tn * rows);
+      return true;
+    }
+    const int q = BN / p.bm;
+    for (int r0 = 0; r0 < p.tiles_m; r0 += G) {
+      const int rows = p.tiles_m - r0 < G ? p.tiles_m - r0 : G;
+      int a, f;
+      const long long cnt = sym_band_tiles(p, q, r0, rows, a, f);
+      if (u >= cnt) {
+        u -= (int)cnt;
+        continue;
+      }
+      for (tn = a; tn < f; ++tn) {
+        const int c = q * (tn + 1) - r0;
+        if (u < c) {
+          tm = r0 + u;
+          return true;
+        }
+        u -= c;
+      }
+      tn = f + u / rows;
+      tm = r0 + (u - (tn - f) * rows);
+      return true;
+    }
+    tm = tn = 0;               // unreachable for t < tiles_per_mat * batch
+    return true;
+  }
   if (!p.sym) {
     tn = u / p.tiles_m;
     tm = u - tn * p.tiles_m;

@@ -73,6 +73,8 @@ struct GemmOp {
   // epilogue mode: 0 = alpha acc + beta C, 1 = Adam in the rotated basis
   int epi = 0;
   float adam_b2 = 0.f, adam_ibc1 = 1.f, adam_ibc2 = 1.f, adam_eps = 0.f;
+  // tile order: 0 = chosen by the launcher; n > 0 = bands of n row tiles
+  int band = 0;
   // plane-stacked K (split-precision products): K = nseg * kseg, segment s
   // uses plane pat_a[s] of A and pat_b[s] of B; planes are planeA/planeB
   // elements apart.  kseg must be a multiple of 64 when nseg > 1.

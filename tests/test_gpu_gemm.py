@@ -135,3 +135,62 @@ def test_gemm_in_place_fp32(ctx):
     torch.cuda.synchronize()
     ref = -0.1 * (_f64(A.cpu()) @ _f64(B.cpu()).T) + 0.9 * W0.numpy()
     assert np.abs(W.cpu().numpy() - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+BAND_CASES = [
+    # M, N, K, batch, sym, band, b_mn, with C
+    (1000, 1000, 192, 2, 1, 3, 0, 0),    # symmetric, ragged last band
+    (904, 904, 256, 1, 1, 1, 0, 0),      # symmetric, one row tile per band
+    (700, 520, 136, 1, 0, 2, 1, 1),      # MN-major B, C epilogue
+    (640, 384, 128, 3, 0, 4, 0, 0),      # batch, last band of one row tile
+]
+
+
+@pytest.mark.parametrize("M,N,K,batch,sym,band,b_mn,with_c", BAND_CASES)
+def test_gemm_banded_tile_order(ctx, M, N, K, batch, sym, band, b_mn, with_c):
+    """Bands of row tiles (the order used when A overflows L2) give the same
+    bits as the plain column order, and the right product."""
+    import torch
+    rng = np.random.default_rng(M + N + K + band)
+    A = _bf16(rng, (batch, M, K))
+    B = A if sym else _bf16(rng, (batch, K, N) if b_mn else (batch, N, K))
+    C = _bf16(rng, (batch, M, N)).cuda() if with_c else None
+    outs = []
+    for bd in (0, band):
+        D = torch.full((batch, M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ctx.gemm_bf16(A.cuda(), B.cuda(), D, M=M, N=N, K=K, batch=batch, b_mn=bool(b_mn), sym=bool(sym),
+                      alpha=1.0, beta=0.5 if with_c else 0.0, C=C, band=bd)
+        torch.cuda.synchronize()
+        outs.append(D.cpu())
+    assert ctx.device_status() == 0
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    a = _f64(A)
+    b = _f64(B) if b_mn else np.swapaxes(_f64(B), 1, 2)
+    ref = a @ b + (0.5 * _f64(C.cpu()) if with_c else 0.0)
+    _check(outs[1], ref, np.abs(a) @ np.abs(b) + (0.5 * np.abs(_f64(C.cpu())) if with_c else 0.0), 0)
+
+
+@pytest.mark.parametrize("sym", [0, 1])
+def test_gemm_band_chosen_for_large_panel(ctx, sym):
+    """8192 x 8192 x 8192: the 128 MB A panel overflows L2 and the launcher
+    takes bands; same bits as the column order forced with a band larger
+    than the tile grid, and sampled rows against float64."""
+    import torch
+    n = 8192
+    rng = np.random.default_rng(8192 + sym)
+    A = (torch.randn(n, n, generator=torch.Generator().manual_seed(11 + sym)) * 0.02).to(torch.bfloat16)
+    B = A if sym else (torch.randn(n, n, generator=torch.Generator().manual_seed(13)) * 0.02).to(torch.bfloat16)
+    Ad, Bd = A.cuda(), B.cuda()
+    outs = []
+    for bd in (0, 1 << 20):
+        D = torch.empty(n, n, dtype=torch.bfloat16, device="cuda")
+        ctx.gemm_bf16(Ad, Bd, D, M=n, N=n, K=n, b_mn=not sym, sym=bool(sym), band=bd)
+        torch.cuda.synchronize()
+        outs.append(D)
+    assert ctx.device_status() == 0
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    rows = np.sort(rng.choice(n, 6, replace=False))
+    a = _f64(A[rows])
+    b = _f64(B).T if sym else _f64(B)
+    ref = a @ b
+    _check(outs[0][rows].cpu(), ref, np.abs(a) @ np.abs(b), 0)

@@ -143,6 +143,9 @@ def test_gemm_rejects_misaligned(lib):
     d.lda = 16
     d.sym, d.N = 1, 32
     assert lib.mo_gemm_bf16(h, ctypes.byref(d), None) == _lib.MO_ERR_INVALID_ARG
+    d.sym, d.N, d.band = 0, 16, -1
+    assert lib.mo_gemm_bf16(h, ctypes.byref(d), None) == _lib.MO_ERR_INVALID_ARG
+    assert b"band" in lib.mo_last_error(h)
     lib.mo_ctx_destroy(h)
 
 

@@ -278,7 +278,10 @@ def run_ours(args, world, rank, local):
     launches = int(sum(v[2] for v in prof.values()))
     gemm_tf = flops_gemm * args.steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
     peak_tf = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    ew_bytes = 24.0 * params
+    # prep moves 14 B/param (G 4, B read + write 8, bf16 N 2); the Muon apply
+    # (W read + write 8, bf16 O 2) runs in the last update's epilogue, or as
+    # apply_kernel when no update product ran
+    ew_bytes = (14.0 + (10.0 if prof["apply"][2] > 0 else 0.0)) * params
     ew_gbs = ew_bytes * args.steps / (ew_ms / 1e3) / 1e9 if ew_ms > 0 else None
 
     value = flops_page * world / (ms / 1e3) / 1e12
@@ -309,9 +312,9 @@ def run_ours(args, world, rank, local):
             "unit": "TFLOP/s",
             "frac": round(gemm_tf / peak_tf, 4) if gemm_tf else None,
             "peak_source": f"{peak_kind} bf16_tflops_sustained",
-            # DRAM bytes of one update launch on the 4096 x 14336 bucket (96
-            # matrices): ncu captured 959.0 MB on the one-layer batch of 3;
-            # traffic grows with the matrices of a launch
+            # DRAM bytes of one update launch (an iteration before the last)
+            # on the 4096 x 14336 bucket (96 matrices): ncu captured 959.0 MB
+            # on the one-layer batch of 3; traffic grows with the matrices
             "traffic": 959.0e6 * args.layers,
             "traffic_kernel": "update GEMM, 4096x14336 bucket, one launch (ncu, scaled by matrices)",
             "alg_flops_per_step": flops_gemm,
@@ -321,7 +324,8 @@ def run_ours(args, world, rank, local):
         },
         "roofline_elementwise": {
             "bound": "hbm",
-            "kernel": "prep_kernel + apply_kernel (24 B/param)",
+            "kernel": ("prep_kernel (14 B/param; the apply runs in the last update's epilogue)"
+                       if prof["apply"][2] == 0 else "prep_kernel + apply_kernel (24 B/param)"),
             "achieved": round(ew_gbs, 1) if ew_gbs else None,
             "peak": peaks.get("hbm_gbs"),
             "unit": "GB/s",

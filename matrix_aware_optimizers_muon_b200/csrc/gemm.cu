@@ -132,9 +132,17 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   p.d_split = op.d_split;
   p.d_plane = op.d_plane;
   p.skip = op.skip;
-  // a strided bf16 C of the plain epilogue is read by TMA
+  p.ap_decay = op.ap_decay;
+  p.ap_step[0] = op.ap_step[0];
+  p.ap_step[1] = op.ap_step[1];
+  p.ap_tall_from = op.ap_tall_from;
+  p.ap_vec = op.ap_vec;
+  if (op.epi == EPI_APPLY && (op.sym || op.e_tab == nullptr || op.d_f32 || op.d_split))
+    return cudaErrorInvalidValue;
+  // a strided bf16 C of the plain (or Muon apply) epilogue is read by TMA
   p.c_tma = 0;
-  if (op.C != nullptr && op.c_tab == nullptr && !op.c_f32 && op.epi == 0 && !op.d_f32 && !op.d_split &&
+  if (op.C != nullptr && op.c_tab == nullptr && !op.c_f32 && (op.epi == EPI_AXPBY || op.epi == EPI_APPLY) &&
+      !op.d_f32 && !op.d_split &&
       (op.batch == 1 || op.strideC % 8 == 0) && op.ldc % 8 == 0 &&
       (reinterpret_cast<uintptr_t>(op.C) & 15) == 0) {
     if (!encode_bf16_c(&tc, op.C, op.M, op.N, op.ldc, op.strideC, op.batch)) return cudaErrorInvalidValue;

@@ -64,9 +64,17 @@ struct GemmParams {
   // tile order: bands of `band` row tiles, each band column by column; a
   // band of tiles_m rows (or more) is the plain column order
   int band;
+  // Muon apply (EPI_APPLY): O = bf16(alpha acc + beta C) is not stored;
+  // W <- ap_decay W - ap_step[tall] O instead, with W = e_tab[b] (fp32,
+  // contiguous), laid out like the product (M x N) or, for the matrices
+  // b >= ap_tall_from, as its transpose (N x M)
+  float ap_decay;
+  float ap_step[2];
+  int ap_tall_from;
+  int ap_vec;               // every W of the launch: 16-byte aligned rows
 };
 
-enum { EPI_AXPBY = 0, EPI_ADAM = 1 };
+enum { EPI_AXPBY = 0, EPI_ADAM = 1, EPI_APPLY = 2 };
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;
@@ -635,6 +643,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const bool plain_f32 = p.d_f32 && !p.d_split;
     const bool has_c = p.C != nullptr || p.c_tab != nullptr;
     const bool adam = p.epi == EPI_ADAM;
+    const bool apply = p.epi == EPI_APPLY;
     int acc = 0;
     uint32_t acc_phase = 0;
     // a pair's epilogue threads release the accumulator on the even CTA's barrier
@@ -649,6 +658,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const char* cbase = has_c ? reinterpret_cast<const char*>(c_base(p, b)) : nullptr;
       char* dbase = reinterpret_cast<char*>(d_base(p, b));
       float* vbase = adam ? p.e_tab[b] : nullptr;
+      float* wbase = apply ? p.e_tab[b] : nullptr;
+      const bool wtall = apply && b >= p.ap_tall_from;
+      const long long ldw = wtall ? p.M : p.N;      // W is contiguous: N x M (tall) or M x N
+      const float wstep = p.ap_step[wtall ? 1 : 0];
       if (row_ok) {
         // pull this row's epilogue inputs into L2 while the main loop runs,
         // so that the loads after the accumulator wait do not pay DRAM latency
@@ -663,6 +676,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const char* row = reinterpret_cast<const char*>(vbase + (long long)r * p.lde + n0);
           for (int off = 0; off < nn * 4; off += 128) prefetch_l2(row + off);
         }
+        if (apply && !wtall && nn > 0) {
+          const char* row = reinterpret_cast<const char*>(wbase + (long long)r * ldw + n0);
+          for (int off = 0; off < nn * 4; off += 128) prefetch_l2(row + off);
+        }
       }
       // bf16 C of full blocks comes by TMA, the first two 32-column blocks
       // requested now so that they arrive while the main loop runs
@@ -670,6 +687,17 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int n0 = tn * BN;
       // a symmetric product skips the 32 x 32 blocks below the diagonal
       const int cc_begin = p.sym ? (r0 - n0 > 0 ? r0 - n0 : 0) : 0;
+      if (apply && wtall && r0 < p.M) {
+        // the transposed W block of this warp: one 128-byte line per W row
+        const int nn = p.N - n0 < BN ? p.N - n0 : BN;
+        for (int c = lane; c < nn; c += 32) prefetch_l2(wbase + (long long)(n0 + c) * ldw + r0);
+      }
+      // Muon apply on a full tile: W blocks move with coalesced accesses,
+      // 16-byte vectors through shared memory (W laid out like the product)
+      // or one 128-byte W row per access (transposed W)
+      const bool wfull = apply && n0 + BN <= p.N && __all_sync(0xffffffffu, row_ok);
+      const bool wvec = wfull && !wtall && p.ap_vec;
+      const bool wtr = wfull && wtall;
       const bool ctma = p.c_tma && !adam && plain_bf16 && n0 + BN <= p.N && __all_sync(0xffffffffu, row_ok);
       auto issue_c = [&](int bi, int cc) {
         mbar_arrive_expect_tx(&cb[bi], 32 * 32 * 2);
@@ -723,6 +751,20 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           for (int j = 0; j < 8; ++j)
             cf[j] = *reinterpret_cast<const float4*>(c32 + (long long)(r0 + 4 * j + (lane >> 3)) * p.ldc + n0 + cc +
                                                      4 * (lane & 7));
+        } else if (wvec) {
+          // W rows r0 .. r0 + 31, columns n0 + cc .. + 31: eight 128-byte rows per load
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            cf[j] = *reinterpret_cast<const float4*>(wbase + (long long)(r0 + 4 * j + (lane >> 3)) * ldw + n0 + cc +
+                                                     4 * (lane & 7));
+        } else if (wtr) {
+          // transposed W: element (row r0 + lane, column n0 + cc + i) of the
+          // product is W[n0 + cc + i][r0 + lane], one 128-byte row per load
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float* w = wbase + (long long)(n0 + cc + 4 * j) * ldw + r0 + lane;
+            cf[j] = make_float4(w[0], w[ldw], w[2 * ldw], w[3 * ldw]);
+          }
         }
         uint32_t v[32];
         tmem_ld32(taddr + cc, v);
@@ -811,7 +853,45 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 32; ++i) x[i] = fmaf(beta, c[i], x[i]);
           }
-          if (diag) {
+          if (apply) {
+            // O = bf16(x), as the plain output would hold it; then the Muon
+            // apply W <- decay W - step O in fp32
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
+            if (wvec) {
+              __syncwarp();               // the previous block's reads of the staging rows are done
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(stg + stg32_off(4 * j + (lane >> 3), lane & 7)) = cf[j];
+              __syncwarp();
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const float4 w = *reinterpret_cast<const float4*>(stg + stg32_off(lane, u));
+                x[4 * u] = fmaf(p.ap_decay, w.x, -wstep * x[4 * u]);
+                x[4 * u + 1] = fmaf(p.ap_decay, w.y, -wstep * x[4 * u + 1]);
+                x[4 * u + 2] = fmaf(p.ap_decay, w.z, -wstep * x[4 * u + 2]);
+                x[4 * u + 3] = fmaf(p.ap_decay, w.w, -wstep * x[4 * u + 3]);
+              }
+              stage_store32_f32(stg, lane, x, wbase + (long long)r0 * ldw + c0, nullptr, ldw);
+            } else if (wtr) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                float* w = wbase + (long long)(c0 + 4 * j) * ldw + r0 + lane;
+                w[0] = fmaf(p.ap_decay, cf[j].x, -wstep * x[4 * j]);
+                w[ldw] = fmaf(p.ap_decay, cf[j].y, -wstep * x[4 * j + 1]);
+                w[2 * ldw] = fmaf(p.ap_decay, cf[j].z, -wstep * x[4 * j + 2]);
+                w[3 * ldw] = fmaf(p.ap_decay, cf[j].w, -wstep * x[4 * j + 3]);
+              }
+            } else if (row_ok) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                if (c0 + i < p.N) {
+                  float* w = wbase + (wtall ? (long long)(c0 + i) * ldw + r : (long long)r * ldw + c0 + i);
+                  *w = fmaf(p.ap_decay, *w, -wstep * x[i]);
+                }
+              }
+            }
+          } else if (diag) {
             if (plain_f32)
               stage_store32_f32_diag(stg, lane, x, reinterpret_cast<float*>(dbase) + (long long)r0 * p.ldd + c0, p.ldd);
             else

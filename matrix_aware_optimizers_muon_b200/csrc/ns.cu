@@ -6,7 +6,9 @@
 //                P = b A + c A A    (symmetric: upper tiles + mirror)
 //                X' = a X + P X }   (iteration 0 folds the 1/(||N||+eps)
 //                                    scale into the fp32 epilogues)
-//   apply (W <- (1 - lr wd) W - lr s O, un-oriented; or out = O)
+//   apply (W <- (1 - lr wd) W - lr s O, un-oriented; or out = O); for Muon
+//   the apply runs in the epilogue of the last update product instead, so
+//   O is never stored
 #include <algorithm>
 #include <cmath>
 #include <map>
@@ -36,9 +38,10 @@ Shape oriented(long long rows, long long cols) {
 
 struct Layout {
   long long ldx, lda, xstride, astride, tiles;
-  size_t x_bytes, a_bytes, part_bytes, inv_bytes;
+  size_t x_bytes, a_bytes, part_bytes, inv_bytes, tab_bytes;
   size_t total(int cnt) const {
-    return 2 * al(x_bytes * cnt) + 2 * al(a_bytes * cnt) + al(part_bytes * cnt) + al(inv_bytes * cnt);
+    return 2 * al(x_bytes * cnt) + 2 * al(a_bytes * cnt) + al(part_bytes * cnt) + al(inv_bytes * cnt) +
+           al(tab_bytes * cnt);
   }
 };
 
@@ -53,6 +56,7 @@ Layout layout_of(const Shape& s) {
   L.a_bytes = (size_t)L.astride * 2;
   L.part_bytes = (size_t)L.tiles * 4;
   L.inv_bytes = 4;
+  L.tab_bytes = 4 * sizeof(void*);     // device pointer tables (in, mom, out, flag)
   return L;
 }
 
@@ -154,7 +158,8 @@ cudaError_t ns_run_at(const std::vector<NsItem>& items, const NsCall& call, int*
       __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(p); p += al(L.a_bytes * cnt);
       __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(p); p += al(L.a_bytes * cnt);
       float* part = reinterpret_cast<float*>(p); p += al(L.part_bytes * cnt);
-      float* inv = reinterpret_cast<float*>(p);
+      float* inv = reinterpret_cast<float*>(p); p += al(L.inv_bytes * cnt);
+      void** tab = reinterpret_cast<void**>(p);
 
       // runs [first, first + count) of equal orientation, at most EW_MAX long
       struct Run { int first, count; bool tall; };
@@ -206,6 +211,30 @@ cudaError_t ns_run_at(const std::vector<NsItem>& items, const NsCall& call, int*
       cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
 
+      // Muon: the last update's epilogue applies O to W, through a device
+      // table of the chunk's W pointers (wide matrices first, then tall)
+      const bool fused_apply = call.muon && call.steps > 0;
+      int tall_from = cnt;
+      bool w_vec = true;
+      float decay = 1.f, step_of[2] = {0.f, 0.f};
+      if (fused_apply) {
+        std::vector<const void*> tin(cnt), tmom(cnt), tout(cnt), tflg(cnt);
+        for (int k = 0; k < cnt; ++k) {
+          const NsItem& it = items[idx[c0 + k]];
+          tin[k] = it.in; tmom[k] = it.mom; tout[k] = it.out; tflg[k] = it.flag;
+          if (is_tall(idx[c0 + k]) && tall_from == cnt) tall_from = k;
+          w_vec = w_vec && it.vec;
+        }
+        launch_upload_tables(tab, cnt, tin.data(), tmom.data(), tout.data(), tflg.data(), stream);
+        decay = (float)(1.0 - (double)call.lr * (double)call.wd);
+        for (int t = 0; t < 2; ++t) {
+          const double m = (double)(t ? s.np : s.mp), n = (double)(t ? s.mp : s.np);   // stored shape
+          const double scale = call.adjust_lr == 0 ? 0.2 * std::sqrt(std::max(m, n))
+                                                   : std::sqrt(std::max(1.0, m / n));
+          step_of[t] = (float)((double)call.lr * scale);
+        }
+      }
+
       // Newton-Schulz iterations on the oriented bf16 batch
       __nv_bfloat16* Xc = X0;
       __nv_bfloat16* Xn = X1;
@@ -237,13 +266,24 @@ cudaError_t ns_run_at(const std::vector<NsItem>& items, const NsCall& call, int*
         u.scale = inv; u.alpha_pow = it == 0 ? 1 : 0; u.beta_pow = it == 0 ? 1 : 0;
         u.C = Xc; u.ldc = L.ldx; u.strideC = L.xstride; u.c_f32 = 0;
         u.D = Xn; u.ldd = L.ldx; u.strideD = L.xstride; u.d_f32 = 0; u.kind = PK_UPDATE;
+        if (fused_apply && it == call.steps - 1) {
+          u.epi = 2;                   // Muon apply epilogue
+          u.e_tab = reinterpret_cast<float* const*>(tab + 2 * cnt);
+          u.ap_decay = decay;
+          u.ap_step[0] = step_of[0];
+          u.ap_step[1] = step_of[1];
+          u.ap_tall_from = tall_from;
+          u.ap_vec = w_vec ? 1 : 0;
+        }
         e = launch_gemm(u, status, stream);
         if (e != cudaSuccess) return e;
         std::swap(Xc, Xn);
       }
 
-      // pass 2: apply the scaled update (Muon) or store O (plain)
+      // pass 2: store O (plain), or apply the scaled update when no update
+      // product ran (zero iterations)
       for (const Run& r : runs) {
+        if (fused_apply) break;
         auto tv = table(r);
         const NsItem& it0 = items[idx[c0 + r.first]];
         const double m = (double)it0.rows, n = (double)it0.cols;

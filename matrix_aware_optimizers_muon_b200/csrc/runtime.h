@@ -70,11 +70,18 @@ struct GemmOp {
   void* const* d_tab = nullptr;
   float* const* e_tab = nullptr;
   long long lde = 0;
-  // epilogue mode: 0 = alpha acc + beta C, 1 = Adam in the rotated basis
+  // epilogue mode: 0 = alpha acc + beta C, 1 = Adam in the rotated basis,
+  // 2 = the Muon apply of O = bf16(alpha acc + beta C) to W = e_tab[b]
   int epi = 0;
   float adam_b2 = 0.f, adam_ibc1 = 1.f, adam_ibc2 = 1.f, adam_eps = 0.f;
   // tile order: 0 = chosen by the launcher; n > 0 = bands of n row tiles
   int band = 0;
+  // Muon apply (epi 2): W <- ap_decay W - ap_step[tall] O; matrices
+  // b >= ap_tall_from store W transposed (N x M), the others as M x N
+  float ap_decay = 1.f;
+  float ap_step[2] = {0.f, 0.f};
+  int ap_tall_from = 0;
+  int ap_vec = 0;        // every W: 16-byte aligned base and row stride
   // plane-stacked K (split-precision products): K = nseg * kseg, segment s
   // uses plane pat_a[s] of A and pat_b[s] of B; planes are planeA/planeB
   // elements apart.  kseg must be a multiple of 64 when nseg > 1.

@@ -281,3 +281,36 @@ def test_cuda_graph_replay_matches_eager(ctx):
         np.testing.assert_array_equal(_np(W[i]), We[i])
         np.testing.assert_array_equal(_np(B[i]), Be[i])
     del graph
+
+
+@pytest.mark.parametrize("shapes", [
+    [(192, 512), (512, 192), (256, 256)],     # wide, tall and square in the GEMM path
+    [(192, 600), (600, 192)],                 # ragged last tile (600 = 2 x 256 + 88)
+    [(200, 518), (518, 200)],                 # rows not 16-byte multiples: scalar W accesses
+])
+def test_apply_in_update_epilogue(ctx, shapes):
+    """Muon's apply runs in the last update product's epilogue.  With zero
+    momentum and no Nesterov the NS input is G itself, so ns_orthogonalize on
+    the same batch yields the same O; W must then be fma(decay, W0, -step O)
+    in fp32 (checked in float64: at most 1 ulp, double rounding aside)."""
+    import torch
+    rng = wl.rng_of("fused-apply-" + "-".join(f"{m}x{n}" for m, n in shapes))
+    Gs = [wl.gaussian(rng, s, 1e-3) for s in shapes]
+    W0 = [wl.gaussian(rng, s, 0.02) for s in shapes]
+    lr, wd = 0.02, 0.01
+    O = [t.cpu().numpy() for t in ctx.ns_orthogonalize([_cuda(g) for g in Gs])]
+    W = [_cuda(w) for w in W0]
+    B = [torch.zeros_like(w) for w in W]
+    ctx.muon_step(W, [_cuda(g) for g in Gs], B, lr=lr, weight_decay=wd, momentum=0.95, nesterov=False)
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    lr32, wd32 = np.float64(np.float32(lr)), np.float64(np.float32(wd))
+    decay = np.float32(1.0 - lr32 * wd32)
+    for (m, n), w0, o, w in zip(shapes, W0, O, W):
+        step = np.float32(lr32 * (0.2 * np.sqrt(max(m, n))))
+        neg = -(step * o.astype(np.float32))                      # fp32 product, as on the device
+        exp = (np.float64(decay) * w0.astype(np.float64) + neg.astype(np.float64)).astype(np.float32)
+        got = w.cpu().numpy()
+        ulp = np.abs(got.view(np.int32).astype(np.int64) - exp.view(np.int32).astype(np.int64))
+        assert ulp.max() <= 1, (m, n, int(ulp.max()))
+        assert (ulp == 0).mean() >= 0.999, (m, n, float((ulp == 0).mean()))

@@ -22,7 +22,7 @@ OP_MUON, OP_SOAP, OP_NS = 0, 1, 2
 
 # kernel kinds reported by mo_profile_read
 KINDS = ["prep", "norm", "gram", "poly", "update", "apply", "soap_ew", "soap_rot", "soap_qr", "gemm",
-         "soap_ema", "qr_chol", "qr_rowblock", "qr_trail", "ns_small"]
+         "soap_ema", "qr_chol", "qr_rowblock", "qr_trail", "ns_small", "tables"]
 
 
 class MuonMat(ctypes.Structure):

@@ -399,6 +399,7 @@ void launch_upload_tables(void** dst, int n, const void* const* in, const void* 
       u.p[2][i] = out[first + i];
       u.p[3][i] = flag[first + i];
     }
+    ProfScope prof(PK_TABLES, s);
     launch_pdl(upload_tables_kernel, dim3((u.n + 127) / 128), dim3(128), 0, s, false, dst + first, n, u);
   }
 }

@@ -25,6 +25,7 @@ enum ProfKind {
   PK_QR_ROWBLK = 12, // QR: panel / TRSM row blocks times the block inverse
   PK_QR_TRAIL = 13,  // QR: tensor-core trailing updates
   PK_SMALL = 14,     // fused small-matrix Newton-Schulz / Muon
+  PK_TABLES = 15,    // device pointer-table uploads
   PK_COUNT = 16
 };
 

@@ -339,6 +339,7 @@ void launch_upload_ptrs(void** dst, const void* const* src, int n, cudaStream_t 
   PtrUpload u;
   u.n = n;
   for (int i = 0; i < n && i < SOAP_MAXB; ++i) u.p[i] = src[i];
+  ProfScope prof(PK_TABLES, s);
   upload_ptrs_kernel<<<1, SOAP_MAXB, 0, s>>>(dst, u);
 }
 
@@ -415,6 +416,7 @@ void launch_adam_identity(const AdamIdArgs& a, cudaStream_t s) {
 }
 
 void launch_set_flags(const FlagTable& flags, int count, int32_t value, cudaStream_t s) {
+  ProfScope prof(PK_SOAP_EW, s);
   set_flags_kernel<<<1, SOAP_MAXB, 0, s>>>(flags, count, value);
 }
 

@@ -401,7 +401,7 @@ __device__ __forceinline__ uint32_t stg32_off(int row, int unit) {
 }
 
 __device__ __forceinline__ void stage_store32_f32(uint8_t* stg, int lane, const float (&x)[32], float* drow,
-                                                  float* dmir, long long ldd) {
+                                                  float* dmir, long long ldd, bool streaming = false) {
   uint8_t* srow = stg;
   uint8_t* scol = stg + 4096;
   __syncwarp();                       // earlier reads of the staging rows are done
@@ -418,7 +418,10 @@ __device__ __forceinline__ void stage_store32_f32(uint8_t* stg, int lane, const 
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int R = 4 * j + (lane >> 3);
-    *reinterpret_cast<float4*>(drow + (long long)R * ldd + 4 * u) = *reinterpret_cast<const float4*>(srow + stg32_off(R, u));
+    const float4 v = *reinterpret_cast<const float4*>(srow + stg32_off(R, u));
+    float4* dst = reinterpret_cast<float4*>(drow + (long long)R * ldd + 4 * u);
+    if (streaming) __stcs(dst, v);     // written once: evict-first in L2
+    else *dst = v;
     if (dmir)
       *reinterpret_cast<float4*>(dmir + (long long)R * ldd + 4 * u) = *reinterpret_cast<const float4*>(scol + stg32_off(R, u));
   }
@@ -752,18 +755,20 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             cf[j] = *reinterpret_cast<const float4*>(c32 + (long long)(r0 + 4 * j + (lane >> 3)) * p.ldc + n0 + cc +
                                                      4 * (lane & 7));
         } else if (wvec) {
-          // W rows r0 .. r0 + 31, columns n0 + cc .. + 31: eight 128-byte rows per load
+          // W rows r0 .. r0 + 31, columns n0 + cc .. + 31: eight 128-byte rows
+          // per load.  W is touched once, so its loads and stores are
+          // streaming (evict-first): the product's operands keep L2
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            cf[j] = *reinterpret_cast<const float4*>(wbase + (long long)(r0 + 4 * j + (lane >> 3)) * ldw + n0 + cc +
-                                                     4 * (lane & 7));
+            cf[j] = __ldcs(reinterpret_cast<const float4*>(wbase + (long long)(r0 + 4 * j + (lane >> 3)) * ldw + n0 +
+                                                           cc + 4 * (lane & 7)));
         } else if (wtr) {
           // transposed W: element (row r0 + lane, column n0 + cc + i) of the
           // product is W[n0 + cc + i][r0 + lane], one 128-byte row per load
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float* w = wbase + (long long)(n0 + cc + 4 * j) * ldw + r0 + lane;
-            cf[j] = make_float4(w[0], w[ldw], w[2 * ldw], w[3 * ldw]);
+            cf[j] = make_float4(__ldcs(w), __ldcs(w + ldw), __ldcs(w + 2 * ldw), __ldcs(w + 3 * ldw));
           }
         }
         uint32_t v[32];
@@ -872,15 +877,15 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 x[4 * u + 2] = fmaf(p.ap_decay, w.z, -wstep * x[4 * u + 2]);
                 x[4 * u + 3] = fmaf(p.ap_decay, w.w, -wstep * x[4 * u + 3]);
               }
-              stage_store32_f32(stg, lane, x, wbase + (long long)r0 * ldw + c0, nullptr, ldw);
+              stage_store32_f32(stg, lane, x, wbase + (long long)r0 * ldw + c0, nullptr, ldw, true);
             } else if (wtr) {
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
                 float* w = wbase + (long long)(c0 + 4 * j) * ldw + r0 + lane;
-                w[0] = fmaf(p.ap_decay, cf[j].x, -wstep * x[4 * j]);
-                w[ldw] = fmaf(p.ap_decay, cf[j].y, -wstep * x[4 * j + 1]);
-                w[2 * ldw] = fmaf(p.ap_decay, cf[j].z, -wstep * x[4 * j + 2]);
-                w[3 * ldw] = fmaf(p.ap_decay, cf[j].w, -wstep * x[4 * j + 3]);
+                __stcs(w, fmaf(p.ap_decay, cf[j].x, -wstep * x[4 * j]));
+                __stcs(w + ldw, fmaf(p.ap_decay, cf[j].y, -wstep * x[4 * j + 1]));
+                __stcs(w + 2 * ldw, fmaf(p.ap_decay, cf[j].z, -wstep * x[4 * j + 2]));
+                __stcs(w + 3 * ldw, fmaf(p.ap_decay, cf[j].w, -wstep * x[4 * j + 3]));
               }
             } else if (row_ok) {
 #pragma unroll

@@ -1,7 +1,10 @@
 // Batched bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM),
-// fed by TMA, with a fused epilogue  D = alpha_b * (A B) + beta_b * C.
+// fed by TMA, with a fused epilogue: D = alpha_b * (A B) + beta_b * C, the
+// Adam step of SOAP in the rotated basis (EPI_ADAM), or the Muon apply
+// W <- decay W - step bf16(alpha_b A B + beta_b C) into fp32 W (EPI_APPLY).
 //
-// One persistent CTA per SM, 6 warps:
+// One persistent CTA per SM (with PAIR, a cluster of two CTAs on two SMs
+// shares each 256-row tile through cta_group::2 MMAs), 6 warps:
 //   warp 0      TMA producer: fills a ring of shared-memory stages
 //   warp 1      MMA issuer: one elected thread issues tcgen05.mma into one
 //               of two TMEM accumulators (so the epilogue of tile i overlaps
@@ -15,6 +18,8 @@
 // product is known to be symmetric (X X^T, or A A with A symmetric): only
 // tiles that touch the upper triangle are computed, and each upper element
 // is stored at (r, c) and mirrored to (c, r), so both halves are bit-equal.
+// Tiles are taken in column order, or in bands of row tiles when the A
+// panel overflows L2 (gemm_decode); the order changes no result.
 #pragma once
 
 #include "ptx.cuh"

@@ -864,7 +864,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
-    ap.add_argument("--e2e-groups", type=int, default=8,
+    ap.add_argument("--e2e-groups", type=int, default=32,
                     help="e2e: layer groups whose gradient copies overlap the previous group's step")
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")

@@ -37,6 +37,38 @@ def _check_f32(t, name):
         raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
 
 
+def _check_state_shapes(i, d, keys):
+    """Shapes of one SOAP / SOAP-Muon matrix's tensors: the library gets
+    pointers only, so a mismatch here would address memory out of bounds."""
+    W = d["W"]
+    if W.dim() != 2:
+        raise ValueError(f"matrix {i}: W must be 2-D")
+    m, n = W.shape
+    for k in keys:
+        t = d.get(k)
+        if t is not None and tuple(t.shape) != (m, n):
+            raise ValueError(f"matrix {i}: {k} must have W's shape {(m, n)}")
+    for fac, q, side in (("L", "QL", m), ("R", "QR", n)):
+        for k in (fac, q):
+            t = d.get(k)
+            if t is not None and tuple(t.shape) != (side, side):
+                raise ValueError(f"matrix {i}: {k} must be {side} x {side}")
+
+
+def _check_extent(t, name, rows, cols, ld, stride, batch, dtypes):
+    """A strided batch of rows x cols matrices (row stride ld, matrix stride
+    stride, in elements) must lie inside the contiguous tensor t."""
+    import torch
+    if not t.is_cuda or not t.is_contiguous() or t.dtype not in dtypes:
+        raise ValueError(f"{name} must be a contiguous CUDA tensor of dtype {dtypes}")
+    if ld < cols:
+        raise ValueError(f"{name}: leading dimension {ld} < row length {cols}")
+    last = (batch - 1) * stride + (rows - 1) * ld + cols
+    if rows > 0 and cols > 0 and last > t.numel():
+        raise ValueError(f"{name}: the {batch} x {rows} x {cols} operand (ld {ld}, stride {stride}) "
+                         f"needs {last} elements, the tensor has {t.numel()}")
+
+
 class Context:
     """One library context on one CUDA device, with a torch-owned workspace."""
 
@@ -81,12 +113,20 @@ class Context:
         return mn.value, full.value
 
     def attach_workspace(self, nbytes, stream=None):
-        """Allocate ``nbytes`` of device memory with torch and attach it."""
+        """Allocate ``nbytes`` of device memory with torch and attach it.
+
+        Library work already enqueued may still use a workspace this one
+        replaces, on any stream, so the device is synchronised before the old
+        buffer goes back to torch's allocator (not during stream capture, where
+        nothing has run yet)."""
         import torch
         buf = torch.empty(int(nbytes), dtype=torch.uint8, device=f"cuda:{self.device}")
         self._check(self.lib.mo_set_workspace(self.handle, c_void_p(buf.data_ptr()), buf.numel(),
                                               self._stream(stream)))
-        self.workspace = buf
+        old, self.workspace = self.workspace, buf
+        if old is not None and not torch.cuda.is_current_stream_capturing():
+            torch.cuda.synchronize(self.device)
+        del old
         return buf
 
     def reserve(self, op, shapes, full=True, stream=None):
@@ -175,6 +215,7 @@ class Context:
         for i, d in enumerate(mats):
             for k in ("W", "G", "M", "V", "L", "QL", "R", "QR"):
                 _check_f32(d.get(k), f"{k}[{i}]")
+            _check_state_shapes(i, d, ("G", "M", "V"))
             W = d["W"]
             arr[i] = SoapMat(W.shape[0], W.shape[1], _ptr(W), _ptr(d.get("G")), _ptr(d["M"]),
                              _ptr(d["V"]), _ptr(d.get("L")), _ptr(d.get("QL")), _ptr(d.get("R")),
@@ -200,6 +241,7 @@ class Context:
         for i, d in enumerate(mats):
             for k in ("W", "G", "B", "V", "L", "QL", "R", "QR"):
                 _check_f32(d.get(k), f"{k}[{i}]")
+            _check_state_shapes(i, d, ("G", "B", "V"))
             W = d["W"]
             arr[i] = SoapMuonMat(W.shape[0], W.shape[1], _ptr(W), _ptr(d.get("G")), _ptr(d["B"]),
                                  _ptr(d["V"]), _ptr(d.get("L")), _ptr(d.get("QL")), _ptr(d.get("R")),
@@ -242,6 +284,12 @@ class Context:
         d.D, d.ldd, d.strideD = D.data_ptr(), ldd or ld_of(D), strideD or stride_of(D)
         d.d_f32 = int(D.dtype == torch.float32)
         d.band = band
+        bf16, outs = (torch.bfloat16,), (torch.bfloat16, torch.float32)
+        _check_extent(A, "A", K if a_mn else M, M if a_mn else K, d.lda, d.strideA, batch, bf16)
+        _check_extent(B, "B", K if b_mn else N, N if b_mn else K, d.ldb, d.strideB, batch, bf16)
+        _check_extent(D, "D", M, N, d.ldd, d.strideD, batch, outs)
+        if C is not None:
+            _check_extent(C, "C", M, N, d.ldc, d.strideC, batch, outs)
         if self.workspace is None:
             self.attach_workspace(4096, stream)
         self._check(self.lib.mo_gemm_bf16(self.handle, byref(d), self._stream(stream)))

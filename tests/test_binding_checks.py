@@ -50,3 +50,12 @@ def test_soap_state_shapes():
             _check_state_shapes(3, d, ("G", "M", "V"))
     with pytest.raises(ValueError, match="2-D"):
         _check_state_shapes(0, dict(ok, W=torch.zeros(m * n)), ("G", "M", "V"))
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No CPU fallback: without libmo.so the binding refuses to load."""
+    from matrix_aware_optimizers_muon_b200 import _lib
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libmo.so"))
+    with pytest.raises(ImportError, match="no CPU fallback"):
+        _lib.load()

@@ -178,6 +178,7 @@ static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3
 
 mo_status muon_step(mo_ctx* ctx, const mo_muon_mat* mats, int n, const mo_muon_cfg* cfg, void* stream) {
   ProfBind prof_bind(ctx);
+  mo::NvtxRange nvtx("mo muon_step");
   if (ctx == nullptr) return MO_ERR_INVALID_ARG;
   if (n < 0) return fail(ctx, MO_ERR_INVALID_ARG, "muon_step: n < 0");
   if (n == 0) return MO_OK;
@@ -232,6 +233,7 @@ mo_status muon_step(mo_ctx* ctx, const mo_muon_mat* mats, int n, const mo_muon_c
 mo_status ns_orthogonalize(mo_ctx* ctx, const float* const* in, float* const* out, const int64_t* rows,
                            const int64_t* cols, int n, const mo_ns_cfg* cfg, void* stream) {
   ProfBind prof_bind(ctx);
+  mo::NvtxRange nvtx("mo ns_orthogonalize");
   if (ctx == nullptr) return MO_ERR_INVALID_ARG;
   if (n < 0) return fail(ctx, MO_ERR_INVALID_ARG, "ns_orthogonalize: n < 0");
   if (n == 0) return MO_OK;
@@ -338,6 +340,7 @@ mo_status soap_step(mo_ctx* ctx, const mo_soap_mat* mats, int n, const mo_soap_c
   if (ctx == nullptr) return MO_ERR_INVALID_ARG;
   if (n < 0) return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: n < 0");
   ProfBind prof_bind(ctx);
+  mo::NvtxRange nvtx("mo soap_step");
   if (n == 0) return MO_OK;
   if (mats == nullptr || cfg == nullptr) return fail(ctx, MO_ERR_INVALID_ARG, "soap_step: null mats or cfg");
   return soap_impl(ctx, mats, n, cfg, step, stream, nullptr);
@@ -348,6 +351,7 @@ mo_status soap_muon_step(mo_ctx* ctx, const mo_soap_muon_mat* mats, int n, const
   if (ctx == nullptr) return MO_ERR_INVALID_ARG;
   if (n < 0) return fail(ctx, MO_ERR_INVALID_ARG, "soap_muon_step: n < 0");
   ProfBind prof_bind(ctx);
+  mo::NvtxRange nvtx("mo soap_muon_step");
   if (n == 0) return MO_OK;
   if (mats == nullptr || cfg == nullptr) return fail(ctx, MO_ERR_INVALID_ARG, "soap_muon_step: null mats or cfg");
   if (!(cfg->momentum >= 0.f && cfg->momentum < 1.f))
@@ -406,6 +410,7 @@ mo_status mo_soap_muon_workspace_bytes(mo_ctx* ctx, const mo_soap_muon_mat* mats
 
 mo_status mo_gemm_bf16(mo_ctx* ctx, const mo_gemm_desc* d, void* stream) {
   ProfBind prof_bind(ctx);
+  mo::NvtxRange nvtx("mo gemm_bf16");
   if (ctx == nullptr) return MO_ERR_INVALID_ARG;
   if (d == nullptr) return fail(ctx, MO_ERR_INVALID_ARG, "mo_gemm_bf16: null descriptor");
   if (d->M <= 0 || d->N <= 0 || d->K <= 0 || d->batch <= 0)

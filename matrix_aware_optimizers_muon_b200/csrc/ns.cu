@@ -120,6 +120,7 @@ cudaError_t ns_run_at(const std::vector<NsItem>& items, const NsCall& call, int*
           vec = al16(in[j]) && al16(out[j]) && (!call.muon || al16(mom[j]));
         }
         launch_upload_tables(tab, n, in.data(), mom.data(), out.data(), flg.data(), stream);
+        NvtxRange nvtx_small("mo newton-schulz small matrices");
         SmallArgs sa;
         sa.count = n; sa.rows = (int)rows; sa.cols = (int)cols; sa.tall = pass;
         sa.mode = call.muon ? 1 : 0;
@@ -151,6 +152,7 @@ cudaError_t ns_run_at(const std::vector<NsItem>& items, const NsCall& call, int*
     while (chunk > 1 && L.total(chunk) > avail) --chunk;
 
     for (int c0 = 0; c0 < (int)idx.size(); c0 += chunk) {
+      NvtxRange nvtx_chunk("mo newton-schulz bucket chunk");
       const int cnt = std::min(chunk, (int)idx.size() - c0);
       char* p = base;
       __nv_bfloat16* X0 = reinterpret_cast<__nv_bfloat16*>(p); p += al(L.x_bytes * cnt);
@@ -239,6 +241,7 @@ cudaError_t ns_run_at(const std::vector<NsItem>& items, const NsCall& call, int*
       __nv_bfloat16* Xc = X0;
       __nv_bfloat16* Xn = X1;
       for (int it = 0; it < call.steps; ++it) {
+        NvtxRange nvtx_it("mo newton-schulz iteration");
         GemmOp g;                      // A = X X^T
         g.A = Xc; g.lda = L.ldx; g.strideA = L.xstride; g.a_mn = 0;
         g.B = Xc; g.ldb = L.ldx; g.strideB = L.xstride; g.b_mn = 0;

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <vector>
 
@@ -42,6 +43,15 @@ struct Profiler {
 };
 
 extern thread_local Profiler* g_prof;
+
+// Named host range (NVTX) around a call or a phase, for timeline profilers;
+// the calls do nothing unless a profiler is attached to the process.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // RAII bracket around one launch (no-op when profiling is off).
 struct ProfScope {

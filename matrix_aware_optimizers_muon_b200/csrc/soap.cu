@@ -624,18 +624,25 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
     return cudaGetLastError();
   };
 
-  if ((e = phase1()) != cudaSuccess) return e;
+  // each phase under its own profiler range
+  auto ranged = [](const char* name, auto&& fn) -> cudaError_t {
+    NvtxRange nvtx(name);
+    return fn();
+  };
+  if ((e = ranged("mo soap factors + first moment", phase1)) != cudaSuccess) return e;
   if (ext == nullptr) {
-    if ((e = cfg.skip_refresh ? old_bases() : refresh()) != cudaSuccess) return e;
-    return rotate();
+    if ((e = cfg.skip_refresh ? ranged("mo soap bases kept", old_bases) : ranged("mo soap basis refresh", refresh)) !=
+        cudaSuccess)
+      return e;
+    return ranged("mo soap rotate + adam + apply", rotate);
   }
   // SOAP-Muon: precondition with the previous bases, orthogonalise and apply,
   // then refresh the bases for the next step
-  if ((e = old_bases()) != cudaSuccess) return e;
-  if ((e = rotate()) != cudaSuccess) return e;
+  if ((e = ranged("mo soap previous bases", old_bases)) != cudaSuccess) return e;
+  if ((e = ranged("mo soap precondition", rotate)) != cudaSuccess) return e;
   if ((e = soap_muon_ns(items, P, *ext, cfg, ws, ws_bytes, s, err)) != cudaSuccess || !err->empty()) return e;
   if (cfg.skip_refresh) return cudaGetLastError();
-  return refresh();
+  return ranged("mo soap basis refresh", refresh);
 }
 
 }  // namespace mo

@@ -314,3 +314,34 @@ def test_apply_in_update_epilogue(ctx, shapes):
         ulp = np.abs(got.view(np.int32).astype(np.int64) - exp.view(np.int32).astype(np.int64))
         assert ulp.max() <= 1, (m, n, int(ulp.max()))
         assert (ulp == 0).mean() >= 0.999, (m, n, float((ulp == 0).mean()))
+
+
+def _save_load(tensors):
+    """torch.save to memory and back onto the GPU: a checkpoint round trip."""
+    import io
+    import torch
+    buf = io.BytesIO()
+    torch.save([t.cpu() for t in tensors], buf)
+    buf.seek(0)
+    return [t.cuda() for t in torch.load(buf)]
+
+
+def test_checkpoint_resume_bitwise(ctx):
+    """All optimizer state is caller-owned: saving W and the momentum after
+    one step, reloading them and stepping again gives the same bits as
+    stepping on (Muon, wide and tall matrices in one bucket)."""
+    import torch
+    rng = wl.rng_of("checkpoint-muon")
+    shapes = [(192, 512), (512, 192)]
+    W = [_cuda(wl.gaussian(rng, s, 0.02)) for s in shapes]
+    B = [torch.zeros_like(w) for w in W]
+    G1 = [_cuda(wl.gaussian(rng, s, 1e-3)) for s in shapes]
+    G2 = [_cuda(wl.gaussian(rng, s, 1e-3)) for s in shapes]
+    ctx.muon_step(W, G1, B)
+    W2, B2 = _save_load(W), _save_load(B)
+    ctx.muon_step(W, G2, B)
+    ctx.muon_step(W2, G2, B2)
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    for a, b in zip(W + B, W2 + B2):
+        assert torch.equal(a, b)

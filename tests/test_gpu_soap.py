@@ -246,3 +246,28 @@ def test_rank_one_and_zero_gradients(ctx):
             c = abs(float(out["QL"][:, 0] @ u[:, 0])) / np.linalg.norm(u)
             assert c >= 1 - 1e-6
             assert np.isfinite(out["W"]).all()
+
+
+def test_checkpoint_resume_bitwise(ctx):
+    """SOAP state (W, M, V, L, Q_L, R, Q_R and the step count) saved after a
+    step and reloaded steps on to the same bits."""
+    import io
+    import torch
+    m = n = 256
+    st = wl.SpikeStream("soap-checkpoint", "x", 0, m, n, wl.CFG4_MINI)
+    keys = ("W", "M", "V", "L", "QL", "R", "QR")
+    S = dict(W=_cuda(st.W), M=torch.zeros(m, n, device="cuda"), V=torch.zeros(m, n, device="cuda"),
+             L=torch.zeros(m, m, device="cuda"), QL=torch.eye(m, device="cuda"),
+             R=torch.zeros(n, n, device="cuda"), QR=torch.eye(n, device="cuda"))
+    G1, G2 = _cuda(st.next()), _cuda(st.next())
+    ctx.soap_step([dict(S, G=G1)], 1, **HP)
+    buf = io.BytesIO()
+    torch.save({k: S[k].cpu() for k in keys}, buf)
+    buf.seek(0)
+    S2 = {k: v.cuda() for k, v in torch.load(buf).items()}
+    ctx.soap_step([dict(S, G=G2)], 2, **HP)
+    ctx.soap_step([dict(S2, G=G2)], 2, **HP)
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    for k in keys:
+        assert torch.equal(S[k], S2[k]), k

@@ -365,14 +365,33 @@ def e2e_measure(ctx, Ws, Gs, Bs, flops_page, world, barrier, args):
     copies, then one call) is timed beside it."""
     import torch
     steps = max(1, min(args.steps, 2))
+    need = sum(g.numel() * g.element_size() for g in Gs)
+    local_world = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
+    reason, host = None, None
     try:
-        host = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in Gs]
-        for h, g in zip(host, Gs):
-            h.copy_(g)
-        flags = torch.zeros(len(Gs), dtype=torch.int32, device=Gs[0].device)
-        flags_h = torch.empty(len(Gs), dtype=torch.int32, pin_memory=True)
-    except RuntimeError as exc:
-        return {"value": None, "unit": UNIT, "reason": f"pinned host allocation failed: {exc}"[:200]}
+        import psutil
+        avail = psutil.virtual_memory().available
+    except ImportError:
+        avail = None
+    if local_world > 1 and avail is not None and need * local_world > 0.8 * avail:
+        reason = (f"{local_world} ranks x {need / 1e9:.1f} GB of pinned host inputs exceed 80 % of the "
+                  f"host's available {avail / 1e9:.0f} GB")
+    else:
+        try:
+            host = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in Gs]
+            for h, g in zip(host, Gs):
+                h.copy_(g)
+            flags = torch.zeros(len(Gs), dtype=torch.int32, device=Gs[0].device)
+            flags_h = torch.empty(len(Gs), dtype=torch.int32, pin_memory=True)
+        except RuntimeError as exc:
+            reason, host = f"pinned host allocation failed: {exc}"[:200], None
+    # every rank takes the same path: the timing below is collective
+    ok = 0.0 if reason else 1.0
+    if world > 1:
+        ok = -max_over_ranks(-ok, world, Gs[0].device)
+    if ok < 1.0:
+        del host
+        return {"value": None, "unit": UNIT, "reason": reason or "another rank could not pin its host inputs"}
     h2d = sum(h.numel() * 4 for h in host)
     hp = dict(lr=0.02, weight_decay=0.01, momentum=0.95, reserve=False)
     n = len(Gs)

@@ -229,7 +229,9 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", device_id=dev)
+        import datetime
+        # ranks that wait for a failed peer end with an error after 5 minutes
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(minutes=5))
 
     def barrier():
         if world > 1:

@@ -55,6 +55,28 @@ def test_worked_example_cubic(golden):
     assert e7 < 2 * g["cubic_max_error_after_7"]
 
 
+def _sym_power(S, p):
+    """S^p for a symmetric positive definite S, from its eigendecomposition."""
+    w, Q = np.linalg.eigh(S)
+    return (Q * w ** p) @ Q.T
+
+
+@pytest.mark.parametrize("k", [1, 4])
+def test_shampoo_without_accumulation_is_the_scaled_polar_factor(golden, k):
+    """The lesson's Shampoo check: with k identical gradients and no
+    accumulation beyond them, L = k G G^T and R = k G^T G, and the Shampoo
+    direction L^{-1/4} G R^{-1/4} is the polar factor scaled by the printed
+    factor (1 for k = 1, 1/2 for k = 4).  The polar factor comes from the
+    oracle's cubic iteration run to convergence, the fractional powers from
+    numpy's eigh: the two constructions share nothing."""
+    g = golden("worked_example_2x2.json")
+    G = np.array(g["G"])
+    scale = g["shampoo_k_identical_gradients"][str(k)]
+    shampoo = _sym_power(k * G @ G.T, -0.25) @ G @ _sym_power(k * G.T @ G, -0.25)
+    polar = ns.newton_schulz(G, ns.CUBIC, 40, eps=0.0)
+    np.testing.assert_allclose(shampoo, scale * polar, rtol=0, atol=1e-12)
+
+
 def test_worked_example_singular_vectors_kept():
     # the quintic output is U diag(.) V^T with G's own singular vectors
     G = np.array([[3.0, 0.0], [4.0, 5.0]])

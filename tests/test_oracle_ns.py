@@ -55,6 +55,26 @@ def test_worked_example_cubic(golden):
     assert e7 < 2 * g["cubic_max_error_after_7"]
 
 
+def test_worked_example_polar_maximises_inner_product(golden):
+    """The lesson's duality check: among unit-spectral-norm directions the
+    polar factor maximises <G, O>, reaching the nuclear norm; G / sigma_max
+    and sign(G) / ||sign(G)||_2 fall short by the printed amounts.  The
+    polar factor is the oracle's cubic iteration run to convergence."""
+    g = golden("worked_example_2x2.json")
+    G = np.array(g["G"])
+    ip = g["inner_products_4dp"]
+    polar = ns.newton_schulz(G, ns.CUBIC, 40, eps=0.0)
+    nuclear = np.linalg.svd(G, compute_uv=False).sum()
+    S = np.sign(G)
+    got = {"polar": np.sum(G * polar),
+           "G_over_sigma_max": np.sum(G * G) / np.linalg.norm(G, 2),
+           "sign_G_over_spectral_norm": np.sum(G * S) / np.linalg.norm(S, 2)}
+    for k, v in got.items():
+        assert round(float(v), 4) == ip[k], (k, v)
+    assert round(float(nuclear), 4) == g["nuclear_norm_4dp"]
+    assert got["polar"] > max(got["G_over_sigma_max"], got["sign_G_over_spectral_norm"])
+
+
 def _sym_power(S, p):
     """S^p for a symmetric positive definite S, from its eigendecomposition."""
     w, Q = np.linalg.eigh(S)

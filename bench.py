@@ -359,14 +359,17 @@ def run_ours(args, world, rank, local):
 def e2e_measure(ctx, Ws, Gs, Bs, flops_page, world, barrier, args):
     """The Muon step end to end through the public API, with every gradient
     copied from pinned host memory and the per-matrix status flags read back
-    inside the timed region.  The step is taken as a training loop whose
+    inside the timed region, over five steps.  The updated weights and
+    momenta stay in device memory, where a training loop keeps them (the
+    library's contract: parameters and state are updated in place on the
+    device), so the flags are the step's only device-to-host result.  The step is taken as a training loop whose
     gradients arrive on the host would take it: the matrices are split into
     groups of whole layers; group k + 1's gradients copy on a side stream
     while muon_step runs on group k (each matrix's step is independent, so
     the result equals one call over all matrices).  The serial form (all
     copies, then one call) is timed beside it."""
     import torch
-    steps = max(1, min(args.steps, 2))
+    steps = 5
     need = sum(g.numel() * g.element_size() for g in Gs)
     local_world = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
     reason, host = None, None

@@ -38,6 +38,8 @@
  *    128 rows on pairs of CTAs (256-row tiles) instead of one CTA per
  *    128-row tile; the results are identical up to fp32 rounding of the
  *    accumulation order.
+ *  - Each call makes the context's device current while it runs and puts
+ *    the calling thread's current device back before it returns.
  *  - One context per host thread.
  */
 #ifndef MO_H_
@@ -89,12 +91,18 @@ MO_API mo_status mo_workspace_bytes(mo_ctx* ctx, int op, const int64_t* rows, co
 
 /* Attach caller-allocated device memory (256-byte aligned).  The library
  * keeps the pointer until the next call; the caller keeps ownership and must
- * not free it while work that uses it is in flight.  Attaching clears the
- * device status word with a stream-ordered memset on `stream`. */
+ * not free it while work that uses it is in flight.  Attaching a different
+ * buffer clears its header with a stream-ordered memset on `stream` and
+ * copies the previous workspace's status word into it (a 4-byte device copy
+ * on `stream`, which reads the old buffer: keep it alive until that copy has
+ * run), so a timeout recorded before the switch is still reported. */
 MO_API mo_status mo_set_workspace(mo_ctx* ctx, void* dev_ptr, size_t bytes, void* stream);
 
 /* Copy the device status word to *status (0 = no timeout recorded) and clear
- * it.  Synchronises `stream`.  Returns MO_ERR_DEVICE when the word was set. */
+ * it.  The word read is the attached workspace's, ORed with that of the
+ * fixed scratch array of ns_orthogonalize_static on ctx's device once a
+ * static call has set it up there; with neither, MO_ERR_NO_WORKSPACE.
+ * Synchronises `stream`.  Returns MO_ERR_DEVICE when the word was set. */
 MO_API mo_status mo_device_status(mo_ctx* ctx, void* stream, int32_t* status);
 
 /* ------------------------------------------------------------------ profiling
@@ -168,8 +176,11 @@ MO_API mo_status ns_orthogonalize(mo_ctx* ctx, const float* const* in, float* co
  * cannot allocate device memory when they call it: programs whose GPU
  * memory belongs to another allocator with nothing spare, runtimes that
  * forbid allocation after start-up, or plain C hosts with no allocator at
- * hand.  It computes exactly what ns_orthogonalize computes for ONE matrix,
- * but its scratch is a fixed device array of MO_STATIC_SCRATCH_BYTES inside
+ * hand.  It computes the same mathematics as ns_orthogonalize for ONE matrix
+ * (the batched-GEMM engine at every shape, so for m' <= 128 and n' <= 256,
+ * where ns_orthogonalize uses its fused small-matrix kernel, the last bits
+ * of the rounding may differ), but its scratch is a fixed device array of
+ * MO_STATIC_SCRATCH_BYTES inside
  * the library (held by every GPU that loads the library until the process
  * exits) instead of an attached workspace; the caller passes only the input
  * and output.  It calls no allocator.
@@ -179,9 +190,14 @@ MO_API mo_status ns_orthogonalize(mo_ctx* ctx, const float* const* in, float* co
  *    that device current) and caches it: make that first call before any
  *    stream capture.
  *  - All calls share the array and leave their contents behind; each call
- *    clears what must start at zero.  Calls that overlap on the GPU (for
- *    example on unordered streams) race on it.
- *  - ctx supplies the device and receives error messages. */
+ *    writes every scratch value before reading it.  Calls that overlap on
+ *    the GPU (for example on unordered streams) race on it.
+ *  - The array starts with a status word in which a kernel wait that gives
+ *    up records its code; it is not cleared by later calls, and
+ *    mo_device_status reads and clears it (no workspace needed).
+ *  - ctx supplies the device (made current for the call; the caller's
+ *    current device is restored before returning) and receives error
+ *    messages. */
 #define MO_STATIC_SCRATCH_BYTES (16u << 20)
 
 MO_API mo_status ns_orthogonalize_static(mo_ctx* ctx, const float* in, float* out, int64_t rows,

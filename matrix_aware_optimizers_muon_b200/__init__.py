@@ -82,6 +82,7 @@ class Context:
             raise MoError(st, "mo_ctx_create failed")
         self.handle = h
         self.workspace = None
+        self.retired = []       # workspaces replaced during stream capture, kept alive
 
     def close(self):
         if getattr(self, "handle", None):
@@ -116,16 +117,24 @@ class Context:
         """Allocate ``nbytes`` of device memory with torch and attach it.
 
         Library work already enqueued may still use a workspace this one
-        replaces, on any stream, so the device is synchronised before the old
-        buffer goes back to torch's allocator (not during stream capture, where
-        nothing has run yet)."""
+        replaces, on any stream, and the switch itself copies the old status
+        word on ``stream``.  Outside stream capture the device is synchronised
+        before the old buffer goes back to torch's allocator.  During capture
+        nothing can be synchronised: eager work enqueued before the capture
+        may still be running, and the captured copy reads the old buffer
+        whenever the graph replays.  So a buffer replaced during capture is
+        kept alive (``retired``) until the next attach outside capture."""
         import torch
         buf = torch.empty(int(nbytes), dtype=torch.uint8, device=f"cuda:{self.device}")
         self._check(self.lib.mo_set_workspace(self.handle, c_void_p(buf.data_ptr()), buf.numel(),
                                               self._stream(stream)))
         old, self.workspace = self.workspace, buf
-        if old is not None and not torch.cuda.is_current_stream_capturing():
-            torch.cuda.synchronize(self.device)
+        if old is not None:
+            if torch.cuda.is_current_stream_capturing():
+                self.retired.append(old)
+            else:
+                torch.cuda.synchronize(self.device)
+                self.retired.clear()
         del old
         return buf
 

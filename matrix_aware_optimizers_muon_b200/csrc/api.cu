@@ -44,15 +44,11 @@ struct ProfBind {
   ~ProfBind() { mo::g_prof = nullptr; }
 };
 
-// device of the context must be current for launches
-mo_status enter(mo_ctx* ctx) {
-  int cur = -1;
-  cudaError_t e = cudaGetDevice(&cur);
-  if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaGetDevice");
-  if (cur != ctx->device) {
-    e = cudaSetDevice(ctx->device);
-    if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaSetDevice");
-  }
+// device of the context must be current for launches; `scope` restores the
+// caller's device when the entry point returns
+mo_status enter(mo_ctx* ctx, mo::DeviceScope& scope) {
+  cudaError_t e = scope.enter(ctx->device);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaSetDevice");
   return MO_OK;
 }
 
@@ -103,26 +99,46 @@ mo_status mo_set_workspace(mo_ctx* ctx, void* dev_ptr, size_t bytes, void* strea
     return fail(ctx, MO_ERR_INVALID_ARG, "mo_set_workspace: null or too small (< 256 bytes)");
   if (reinterpret_cast<uintptr_t>(dev_ptr) % 256 != 0)
     return fail(ctx, MO_ERR_INVALID_ARG, "mo_set_workspace: pointer must be 256-byte aligned");
-  mo_status st = enter(ctx);
+  mo::DeviceScope dev_scope;
+  mo_status st = enter(ctx, dev_scope);
   if (st != MO_OK) return st;
-  ctx->ws = static_cast<char*>(dev_ptr);
-  ctx->ws_bytes = bytes;
-  cudaError_t e = cudaMemsetAsync(ctx->ws, 0, mo::WS_HEADER, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* old = ctx->ws;
+  char* ws = static_cast<char*>(dev_ptr);
+  cudaError_t e = cudaSuccess;
+  if (old != ws) {
+    e = cudaMemsetAsync(ws, 0, mo::WS_HEADER, s);
+    // a timeout code the old workspace still holds stays readable through
+    // mo_device_status after the switch
+    if (e == cudaSuccess && old != nullptr)
+      e = cudaMemcpyAsync(ws, old, sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+  }
   if (e != cudaSuccess) return cuda_fail(ctx, e, "mo_set_workspace");
+  ctx->ws = ws;
+  ctx->ws_bytes = bytes;
   return MO_OK;
 }
 
 mo_status mo_device_status(mo_ctx* ctx, void* stream, int32_t* status) {
   if (ctx == nullptr || status == nullptr) return MO_ERR_INVALID_ARG;
-  if (ctx->ws == nullptr) return fail(ctx, MO_ERR_NO_WORKSPACE, "mo_device_status: no workspace attached");
-  mo_status st = enter(ctx);
+  // the attached workspace's word and the word of the fixed scratch array
+  // that ns_orthogonalize_static uses on this device (once it has been set up)
+  int32_t* words[2] = {reinterpret_cast<int32_t*>(ctx->ws), mo::static_status_word(ctx->device)};
+  if (words[0] == nullptr && words[1] == nullptr)
+    return fail(ctx, MO_ERR_NO_WORKSPACE, "mo_device_status: no workspace attached and no static call made");
+  mo::DeviceScope dev_scope;
+  mo_status st = enter(ctx, dev_scope);
   if (st != MO_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int32_t v = 0;
-  cudaError_t e = cudaMemcpyAsync(&v, ctx->ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  int32_t got[2] = {0, 0};
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < 2 && e == cudaSuccess; ++i)
+    if (words[i]) e = cudaMemcpyAsync(&got[i], words[i], sizeof(int32_t), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->ws, 0, sizeof(int32_t), s);
+  for (int i = 0; i < 2 && e == cudaSuccess; ++i)
+    if (words[i]) e = cudaMemsetAsync(words[i], 0, sizeof(int32_t), s);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "mo_device_status");
+  const int32_t v = got[0] | got[1];
   *status = v;
   if (v != 0) return fail(ctx, MO_ERR_DEVICE, "device status " + std::to_string(v) + ": a kernel wait timed out");
   return MO_OK;
@@ -141,7 +157,8 @@ mo_status mo_profile_enable(mo_ctx* ctx, int enable) {
 mo_status mo_profile_read(mo_ctx* ctx, double* ms, double* flops, int64_t* launches, int nkinds) {
   if (ctx == nullptr || nkinds < 0 || (nkinds > 0 && (ms == nullptr || flops == nullptr || launches == nullptr)))
     return MO_ERR_INVALID_ARG;
-  mo_status st = enter(ctx);
+  mo::DeviceScope dev_scope;
+  mo_status st = enter(ctx, dev_scope);
   if (st != MO_OK) return st;
   for (int k = 0; k < nkinds; ++k) { ms[k] = 0; flops[k] = 0; launches[k] = 0; }
   if (ctx->prof.failed) return fail(ctx, MO_ERR_CUDA, "mo_profile_read: an event could not be created or recorded");
@@ -212,7 +229,8 @@ mo_status muon_step(mo_ctx* ctx, const mo_muon_mat* mats, int n, const mo_muon_c
   }
   if (items.empty()) return MO_OK;
   if (ctx->ws == nullptr) return fail(ctx, MO_ERR_NO_WORKSPACE, "muon_step: no workspace attached");
-  st = enter(ctx);
+  mo::DeviceScope dev_scope;
+  st = enter(ctx, dev_scope);
   if (st != MO_OK) return st;
 
   mo::NsCall call;
@@ -262,7 +280,8 @@ mo_status ns_orthogonalize(mo_ctx* ctx, const float* const* in, float* const* ou
     items.push_back(it);
   }
   if (ctx->ws == nullptr) return fail(ctx, MO_ERR_NO_WORKSPACE, "ns_orthogonalize: no workspace attached");
-  st = enter(ctx);
+  mo::DeviceScope dev_scope;
+  st = enter(ctx, dev_scope);
   if (st != MO_OK) return st;
   mo::NsCall call;
   call.muon = false;
@@ -317,7 +336,8 @@ mo_status soap_impl(mo_ctx* ctx, const mo_soap_mat* mats, int n, const mo_soap_c
   }
   if (items.empty()) return MO_OK;
   if (ctx->ws == nullptr) return fail(ctx, MO_ERR_NO_WORKSPACE, fn + ": no workspace attached");
-  mo_status st = enter(ctx);
+  mo::DeviceScope dev_scope;
+  mo_status st = enter(ctx, dev_scope);
   if (st != MO_OK) return st;
   std::string err;
   cudaError_t e = mo::soap_run(items, *cfg, step, ctx->ws, ctx->ws_bytes, static_cast<cudaStream_t>(stream), &err, ext);
@@ -433,7 +453,8 @@ mo_status mo_gemm_bf16(mo_ctx* ctx, const mo_gemm_desc* d, void* stream) {
     return fail(ctx, MO_ERR_INVALID_ARG, "mo_gemm_bf16: alpha_pow and beta_pow must be 0, 1 or 2");
   if (d->band < 0) return fail(ctx, MO_ERR_INVALID_ARG, "mo_gemm_bf16: band must be >= 0");
   if (ctx->ws == nullptr) return fail(ctx, MO_ERR_NO_WORKSPACE, "mo_gemm_bf16: no workspace attached (status word)");
-  mo_status st = enter(ctx);
+  mo::DeviceScope dev_scope;
+  mo_status st = enter(ctx, dev_scope);
   if (st != MO_OK) return st;
   mo::GemmOp op;
   op.A = d->A; op.lda = d->lda; op.strideA = d->strideA; op.a_mn = d->a_mn;

@@ -15,8 +15,10 @@
 // array's name is only a host-side stand-in, never a device address.
 //
 // Sharing: every call uses the same array and leaves its contents behind.
-// Each call clears the status word at its start; everything else it reads it
-// first writes.  Calls whose kernels overlap on the GPU (different streams
+// The array starts with a status word where a kernel wait that gives up
+// records its code; mo_device_status reads and clears it (with or without
+// an attached workspace), so a call that timed out is visible until then.
+// Everything else a call reads it first writes.  Calls whose kernels overlap on the GPU (different streams
 // without ordering) race on the array.
 #include <cmath>
 #include <mutex>
@@ -58,6 +60,14 @@ cudaError_t scratch_on(int dev, char** out) {
 
 }  // namespace
 
+namespace mo {
+int32_t* static_status_word(int dev) {
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  return reinterpret_cast<int32_t*>(g_scratch_addr[dev]);
+}
+}  // namespace mo
+
 extern "C" MO_API mo_status ns_orthogonalize_static(mo_ctx* ctx, const float* in, float* out,
                                                     int64_t rows, int64_t cols, const mo_ns_cfg* cfg,
                                                     void* stream) {
@@ -93,9 +103,8 @@ extern "C" MO_API mo_status ns_orthogonalize_static(mo_ctx* ctx, const float* in
                             " (use ns_orthogonalize with a workspace)");
 
   const int dev = mo::ctx_device(ctx);
-  int cur = -1;
-  cudaError_t e = cudaGetDevice(&cur);
-  if (e == cudaSuccess && cur != dev) e = cudaSetDevice(dev);
+  mo::DeviceScope dev_scope;                     // the caller's device is current again on return
+  cudaError_t e = dev_scope.enter(dev);
   char* ws = nullptr;
   if (e == cudaSuccess) e = scratch_on(dev, &ws);
   if (e != cudaSuccess)
@@ -111,8 +120,9 @@ extern "C" MO_API mo_status ns_orthogonalize_static(mo_ctx* ctx, const float* in
   float* part = reinterpret_cast<float*>(p); p += align_up(tiles * 4);
   float* inv = reinterpret_cast<float*>(p);
 
-  // the status word must start at zero; all other scratch is written before it is read
-  e = cudaMemsetAsync(status, 0, mo::WS_HEADER, s);
+  // The status word (zero when the library loads) is not cleared here: a
+  // timeout code an earlier call recorded stays until mo_device_status reads
+  // it.  All other scratch is written before it is read.
 
   mo::EwTable t;
   t.in[0] = in; t.mom[0] = nullptr; t.out[0] = out;

@@ -8,6 +8,37 @@
 
 namespace mo {
 
+// Makes a context's device current for the length of one API call and puts
+// the caller's current device back when the call returns, so that calling
+// into the library never changes which device the caller's thread uses.
+class DeviceScope {
+ public:
+  DeviceScope() = default;
+  DeviceScope(const DeviceScope&) = delete;
+  DeviceScope& operator=(const DeviceScope&) = delete;
+  cudaError_t enter(int dev) {
+    cudaError_t e = cudaGetDevice(&prev_);
+    if (e != cudaSuccess) return e;
+    if (prev_ != dev) {
+      e = cudaSetDevice(dev);
+      if (e == cudaSuccess) switched_ = true;
+    }
+    return e;
+  }
+  ~DeviceScope() {
+    if (switched_) (void)cudaSetDevice(prev_);
+  }
+
+ private:
+  int prev_ = -1;
+  bool switched_ = false;
+};
+
+// Device address of the status word at the start of the fixed scratch array
+// of ns_orthogonalize_static on device `dev`, or null while no call has set
+// the array up there.
+int32_t* static_status_word(int dev);
+
 // Allow `bytes` of dynamic shared memory for kernel `func` on the current
 // device: set once per (device, kernel), thread-safe.
 cudaError_t ensure_smem_attr(const void* func, int bytes);

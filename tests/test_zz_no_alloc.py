@@ -12,7 +12,9 @@ import numpy as np
 import pytest
 
 import workloads as wl
+from gates import ns_gate
 from gpu_env import context
+from oracle import ns as ons
 
 pytestmark = pytest.mark.gpu
 
@@ -58,3 +60,38 @@ def test_static_scratch_rejects_oversized_shapes():
     assert _static(ctx, x, y) == _lib.MO_ERR_UNSUPPORTED
     msg = ctx.lib.mo_last_error(ctx.handle).decode()
     assert "scratch" in msg and str(16 << 20) in msg
+
+
+@pytest.mark.parametrize("m,n", [(96, 200), (200, 96), (5, 7)])
+def test_static_small_shapes_against_oracle(m, n):
+    """Shapes that the workspace path sends to its fused small-matrix kernel
+    take the batched GEMM chain here (a single tile, K below 64, the TMA
+    boxes mostly zero fill); gated against the fp64 oracle on the resolved
+    subspace, with singular values in [0.6, 1.3], and against the noise
+    floor of the oracle's bf16 emulation."""
+    import torch
+    ctx = context()
+    G = wl.gaussian(wl.rng_of("no-alloc-small", m, n), (m, n), 1.0)
+    x = torch.from_numpy(G).cuda()
+    y = torch.full_like(x, float("nan"))
+    assert _static(ctx, x, y) == 0, ctx.lib.mo_last_error(ctx.handle)
+    torch.cuda.synchronize()
+    O = y.cpu().numpy().astype(np.float64)
+    assert np.isfinite(O).all()
+    ns_gate(G, O, ons.newton_schulz(G), ons.newton_schulz_bf16(G))
+
+
+def test_static_status_word_readable_without_workspace():
+    """A caller of the static entry point has no workspace: the status word
+    of the fixed array is read (and cleared) by mo_device_status all the
+    same, and the call leaves the caller's current device as it was."""
+    import torch
+    from matrix_aware_optimizers_muon_b200 import Context
+    ctx = Context(0)                      # no workspace attached
+    assert ctx.workspace is None
+    dev_before = torch.cuda.current_device()
+    x = torch.from_numpy(wl.gaussian(wl.rng_of("no-alloc-status"), (64, 96), 1.0)).cuda()
+    y = torch.empty_like(x)
+    assert _static(ctx, x, y) == 0, ctx.lib.mo_last_error(ctx.handle)
+    assert torch.cuda.current_device() == dev_before
+    assert ctx.device_status() == 0

@@ -11,7 +11,7 @@ def rel(a, b):
 
 
 def ns_gate(N, O_gpu, O_ref, O_emu, *, tau=1e-2, sub_tol=2e-2, band=(0.6, 1.3), floor=1.25,
-            floor_abs=2e-3, svd=None):
+            floor_abs=2e-3, svd=None, fro=None):
     """Newton-Schulz parity on the resolved subspace plus a noise-floor gate.
 
     The iteration multiplies near-null singular directions by up to a^5, so
@@ -21,6 +21,9 @@ def ns_gate(N, O_gpu, O_ref, O_emu, *, tau=1e-2, sub_tol=2e-2, band=(0.6, 1.3), 
         values inside ``band``;
     (2) on the full matrix: the GPU's error against fp64 is no worse than
         ``floor`` times the oracle's own bf16-emulation error (+ floor_abs).
+    ``svd`` may hold only the leading singular triplets of N (every
+    resolved one among them); ``fro`` is then N's Frobenius norm, against
+    which tau is taken (default: the norm of the given singular values).
     Returns a dict of the measured numbers (asserts inside).
     """
     N = np.asarray(N, dtype=np.float64)
@@ -29,7 +32,8 @@ def ns_gate(N, O_gpu, O_ref, O_emu, *, tau=1e-2, sub_tol=2e-2, band=(0.6, 1.3), 
         U, s, Vt = np.linalg.svd(N, full_matrices=False)
     else:
         U, s, Vt = svd
-    k = int(np.sum(s / np.linalg.norm(s) >= tau))
+    k = int(np.sum(s / (np.linalg.norm(s) if fro is None else fro) >= tau))
+    assert k < len(s) or svd is None or fro is None, "the given triplets may not hold every resolved one"
     Uk, Vk = U[:, :k], Vt[:k].T
     P = lambda O: Uk.T @ np.asarray(O, dtype=np.float64) @ Vk
     sub = rel(P(O_gpu), P(O_ref))

@@ -7,7 +7,7 @@ with the current gradient folded in; "初探优化器（一）", section 6.2 ste
 section 11.1 equations):
 
     1. L = bs L + (1 - bs) G G^T ;   R = bs R + (1 - bs) G^T G
-    2. Q_L = qr((L + dL I) Q_L) ;    Q_R = qr((R + dR I) Q_R)   (one power step)
+    2. Q_L = qr(L Q_L) ;             Q_R = qr(R Q_R)            (one power step)
     3. M = b1 M + (1 - b1) G                            (original space)
     4. M' = Q_L^T M Q_R ;            G' = Q_L^T G Q_R
     5. V = b2 V + (1 - b2) G' * G'                      (rotated space)
@@ -15,18 +15,22 @@ section 11.1 equations):
     6. D = Q_L Dbar Q_R^T
     7. W = (1 - lr wd) W - lr D
 
-The power step runs on the damped factor L + d I (the Shampoo family damps
-its factors: "Matrix optimizers: K-FAC, Shampoo and Muon", Shampoo algorithm,
-L0 = eps I, and the K-FAC damping A + gamma I; the LLM Optimizers guide,
-section 11.2, lists damping among the parts of production SOAP).  Damping
-keeps every eigenvector of L, so the basis the power iteration tracks is
-unchanged; it bounds cond(L + d I) by 1 + 1 / damping, which keeps the QR
-well defined when L is singular or nearly so (a cold start, a rank-one
-gradient, a factor wider than the gradient's rank).  The pages fix no value;
-this reading makes d relative, d = damping * trace(L) with damping = 1e-5,
-so that it does not depend on the gradient's scale, and d = 1 when
-trace(L) = 0 (a factor that has seen only zero gradients keeps its basis).
-The stored factor L is not damped.
+Step 2 is the pages' refresh as written: one power-iteration step on the
+factor, followed by a QR, with the current gradient already folded into the
+factor (the reading notes, section 4; "初探优化器（一）", section 6.2 step 2;
+the SOAP workload: "one power iteration Q <- qr(L Q)").  QR is LAPACK's
+Householder factorisation with the positive-diagonal convention
+(``oracle.qr``).  Where L Q is singular the QR is not unique; Householder
+then completes Q with trivial reflectors, so a zero factor (only zero
+gradients seen) gives Q = I.
+
+``damping > 0`` is an option that departs from the pages: the power step
+then runs on L + d I with d = damping * trace(L) (d = 1 when the trace is
+zero), the damping the Shampoo family applies to its factors ("Matrix
+optimizers: K-FAC, Shampoo and Muon", Shampoo, L0 = eps I; K-FAC's
+A + gamma I).  It keeps L's eigenvectors but changes how far the basis moves
+inside the low-eigenvalue subspace, and so changes the update; the default
+is 0.  The stored factor L is never damped.
 
 A side whose factor is ``None`` uses the identity basis (one-sided SOAP for
 very large axes, section 11.2 of the LLM Optimizers guide); with both sides
@@ -43,7 +47,7 @@ accumulation (stored intermediates are kept as h + l).  With both sides
 present the two-sided products are taken left factor first:
 
     s1: Gb = bf16(G);  L = bs L + (1 - bs) Gb Gb^T   (L itself is not rounded)
-    s2: Y = (L + d I) Q_L (not rounded);  Q_L = qr(Y)
+    s2: Y = L Q_L (not rounded);  Q_L = qr(Y)
     s4: M' = p(s(p(Q_L^T, M)), Q_R);   G' = p(s(p(Q_L^T, G)), Q_R)
     s6: D  = p(s(p(Q_L, Dbar)), Q_R^T)
   where p(A, B) is the three-plane product and s(x) = h + l;
@@ -59,8 +63,10 @@ from .qr import qr_positive
 
 
 def damping_of(F, damping):
-    """The power step's damping d for factor F: damping * trace(F), or 1 when
-    the trace is zero."""
+    """The power step's damping d for factor F: 0 without damping (the
+    pages' step); else damping * trace(F), or 1 when the trace is zero."""
+    if damping == 0.0:
+        return 0.0
     tr = float(np.trace(F))
     return damping * tr if tr != 0.0 else 1.0
 
@@ -68,7 +74,7 @@ def damping_of(F, damping):
 def soap_step(W, G, M, V, L=None, QL=None, R=None, QR=None, *, t=1,
               lr=3e-3, beta1=0.95, beta2=0.95, shampoo_beta=None, eps=1e-8,
               weight_decay=0.0, bias_correction=True, precision="fp64",
-              refresh=True, basis_refresh=True, damping=1e-5):
+              refresh=True, basis_refresh=True, damping=0.0):
     """One SOAP step.  Inputs are not modified; returns the new state.
 
     ``shampoo_beta`` defaults to ``beta2`` (one beta for both second-order
@@ -79,7 +85,8 @@ def soap_step(W, G, M, V, L=None, QL=None, R=None, QR=None, *, t=1,
     refresh interval f ("LLM Optimizers" guide, section 11.1: the bases are
     refreshed every f steps; "Matrix optimizers: K-FAC, Shampoo and Muon",
     SOAP step 3).
-    ``damping`` is the relative damping of the power step (see above).
+    ``damping`` is the optional relative damping of the power step (see
+    above; 0, the default, is the pages' undamped step).
     """
     if precision not in ("fp64", "bf16"):
         raise ValueError(f"unknown precision {precision!r}")
@@ -114,7 +121,8 @@ def soap_step(W, G, M, V, L=None, QL=None, R=None, QR=None, *, t=1,
 
     def power_step(F, Q):
         d = damping_of(F, damping)
-        return qr_positive((F + d * np.eye(F.shape[0])) @ Q)[0]
+        Y = F @ Q if d == 0.0 else (F + d * np.eye(F.shape[0])) @ Q
+        return qr_positive(Y)[0]
 
     # 1-2. factor EMAs with the current gradient, then one power step + QR
     if refresh:

@@ -19,8 +19,9 @@ steps below are the plainest reading of those notes:
     5. O = NS(P)            (the rescaling is Newton-Schulz's own Frobenius
                              normalisation; the pages leave the norm open)
     6. W = (1 - lr wd) W - lr s O,   s = 0.2 sqrt(max(m, n)) or sqrt(max(1, m/n))
-    7. L = bs L + (1 - bs) G G^T ;  R likewise ;  Q = qr((L + d I) Q)
-       (the damped power step of ``oracle.soap``; used from the next step on)
+    7. L = bs L + (1 - bs) G G^T ;  R likewise ;  Q = qr(L Q)
+       (the power step + QR of ``oracle.soap``; used from the next step on;
+        ``damping > 0`` is the same optional departure as there)
 
 A side whose factor is ``None`` uses the identity basis, as in SOAP.
 
@@ -43,7 +44,7 @@ def soap_muon_step(W, G, B, V, L=None, QL=None, R=None, QR=None, *, t=1,
                    lr=0.02, weight_decay=0.01, momentum=0.95, nesterov=True,
                    beta2=0.95, shampoo_beta=0.9, eps=1e-8, bias_correction=True,
                    ns_steps=5, coeffs=QUINTIC, ns_eps=1e-7,
-                   adjust_lr="match_rms_adamw", damping=1e-5, precision="fp64"):
+                   adjust_lr="match_rms_adamw", damping=0.0, precision="fp64"):
     """One SOAP-Muon step.  Inputs are not modified; returns the new state
     and the intermediates P (preconditioned momentum) and O."""
     if precision not in ("fp64", "bf16"):
@@ -113,11 +114,15 @@ def soap_muon_step(W, G, B, V, L=None, QL=None, R=None, QR=None, *, t=1,
     # 7. factor EMAs with the raw gradient and the basis refresh for the next step
     Gb = rnd(G) if emu else G
     QL_new, QR_new = QL, QR
+    def power_step(F, Q):
+        d = damping_of(F, damping)
+        return qr_positive(F @ Q if d == 0.0 else (F + d * np.eye(F.shape[0])) @ Q)[0]
+
     if left:
         L = shampoo_beta * L + (1.0 - shampoo_beta) * (Gb @ Gb.T)
-        QL_new = qr_positive((L + damping_of(L, damping) * np.eye(m)) @ QL)[0]
+        QL_new = power_step(L, QL)
     if right:
         R = shampoo_beta * R + (1.0 - shampoo_beta) * (Gb.T @ Gb)
-        QR_new = qr_positive((R + damping_of(R, damping) * np.eye(n)) @ QR)[0]
+        QR_new = power_step(R, QR)
     return {"W": W_new, "B": B, "V": V, "L": L, "QL": QL_new, "R": R, "QR": QR_new,
             "N": N, "P": P, "O": O, "dW": W_new - decayed}

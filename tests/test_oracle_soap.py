@@ -152,53 +152,64 @@ def test_first_step_from_zero_state():
                          beta2=0.9)
     np.testing.assert_allclose(out["L"], 0.1 * G @ G.T, atol=1e-14)
     np.testing.assert_allclose(out["R"], 0.1 * G.T @ G, atol=1e-14)
-    # Q_L's columns are the Gram-Schmidt orthonormalisation of the damped
-    # L_1's columns (damping 1e-5 of the trace, summed here by a Python loop)
-    L1 = out["L"].tolist()
-    d = 1e-5 * sum(L1[i][i] for i in range(m))
-    Qg, _ = _gram_schmidt([[L1[i][j] + (d if i == j else 0.0) for j in range(m)] for i in range(m)])
+    # Q_L's columns are the Gram-Schmidt orthonormalisation of L_1's columns
+    # (L_1 Q_0 = L_1), in a Python loop
+    Qg, _ = _gram_schmidt(out["L"].tolist())
     np.testing.assert_allclose(out["QL"], Qg, atol=1e-9)
     np.testing.assert_allclose(out["QL"].T @ out["QL"], np.eye(m), atol=1e-12)
-    # without damping the factor's own Gram-Schmidt basis
-    out0 = soap.soap_step(np.zeros((m, n)), G, np.zeros((m, n)), np.zeros((m, n)),
-                          np.zeros((m, m)), np.eye(m), None, None, beta2=0.9, damping=0.0)
-    Qg0, _ = _gram_schmidt(out0["L"].tolist())
-    np.testing.assert_allclose(out0["QL"], Qg0, atol=1e-9)
+    # the damped option: the Gram-Schmidt basis of L_1 + d I, d = 1e-5 trace(L_1)
+    out1 = soap.soap_step(np.zeros((m, n)), G, np.zeros((m, n)), np.zeros((m, n)),
+                          np.zeros((m, m)), np.eye(m), None, None, beta2=0.9, damping=1e-5)
+    L1 = out1["L"].tolist()
+    d = 1e-5 * sum(L1[i][i] for i in range(m))
+    Qg1, _ = _gram_schmidt([[L1[i][j] + (d if i == j else 0.0) for j in range(m)] for i in range(m)])
+    np.testing.assert_allclose(out1["QL"], Qg1, atol=1e-9)
 
 
-def test_damped_power_step_worked_example():
+def test_power_step_worked_example():
     """2 x 2 by hand: L = diag(3, 1), old basis the rotation with cos 0.6 and
-    sin 0.8.  trace(L) = 4, so d = 4e-5 and (L + d I) Q_old has first column
-    (3.00004 * 0.6, 1.00004 * 0.8) = (1.800024, 0.800032); the new basis is
-    that column normalised and its positive-diagonal completion.  The state
-    is chosen so that the EMA leaves L = diag(3, 1): beta2 = 0.5, L_prev =
-    diag(6, 2) - G G^T with G = diag(0, 0) -> L_prev = diag(6, 2)."""
+    sin 0.8.  L Q_old has columns (3 * 0.6, 1 * 0.8) = (1.8, 0.8) and
+    (3 * -0.8, 1 * 0.6) = (-2.4, 0.6); the new basis is the first column
+    normalised, (1.8, 0.8) / sqrt(3.88), and the orthogonal unit vector
+    (-0.8, 1.8) / sqrt(3.88), whose product with the second column,
+    (1.92 + 1.08) / sqrt(3.88), is positive (diag(R) > 0).  The state is
+    chosen so that the EMA leaves L = diag(3, 1): beta2 = 0.5, G = 0,
+    L_prev = diag(6, 2)."""
     L_prev = np.diag([6.0, 2.0])
     Q_old = np.array([[0.6, -0.8], [0.8, 0.6]])
     Z = np.zeros((2, 2))
     out = soap.soap_step(Z, Z, Z, Z, L_prev, Q_old, t=1, beta2=0.5)
     np.testing.assert_allclose(out["L"], np.diag([3.0, 1.0]), atol=0)
-    r = (1.800024 ** 2 + 0.800032 ** 2) ** 0.5
-    q1 = np.array([1.800024, 0.800032]) / r
-    expect = np.array([[q1[0], -q1[1]], [q1[1], q1[0]]])
-    np.testing.assert_allclose(out["QL"], expect, rtol=0, atol=1e-13)
-    # the undamped step differs at the 1e-5 level, far above the tolerance
-    r0 = (1.8 ** 2 + 0.8 ** 2) ** 0.5
-    assert abs(out["QL"][0, 0] - 1.8 / r0) > 1e-7
+    r = 3.88 ** 0.5
+    expect = np.array([[1.8, -0.8], [0.8, 1.8]]) / r
+    np.testing.assert_allclose(out["QL"], expect, rtol=0, atol=1e-14)
+    # the damped option (trace 4, d = 4e-5): (L + d I) Q_old has first column
+    # (3.00004 * 0.6, 1.00004 * 0.8) = (1.800024, 0.800032)
+    out1 = soap.soap_step(Z, Z, Z, Z, L_prev, Q_old, t=1, beta2=0.5, damping=1e-5)
+    r1 = (1.800024 ** 2 + 0.800032 ** 2) ** 0.5
+    q1 = np.array([1.800024, 0.800032]) / r1
+    np.testing.assert_allclose(out1["QL"], np.array([[q1[0], -q1[1]], [q1[1], q1[0]]]), rtol=0, atol=1e-13)
+    # the two differ at the 1e-5 level, far above the tolerances
+    assert abs(out1["QL"][0, 0] - out["QL"][0, 0]) > 1e-7
 
 
-def test_damping_keeps_an_exact_eigenbasis_and_a_zero_factor():
+def test_power_step_keeps_an_exact_eigenbasis_and_resets_a_zero_factor():
     rng = np.random.default_rng(31)
     m = 7
     U, _ = np.linalg.qr(rng.standard_normal((m, m)))
-    L = (U * np.array([9.0, 5.0, 3.0, 2.0, 1.0, 0.5, 0.1])) @ U.T
+    lam = np.array([9.0, 5.0, 3.0, 2.0, 1.0, 0.5, 0.1])
+    L = (U * lam) @ U.T
     Z = np.zeros((m, 3))
-    # shampoo_beta = 1: the factor is L itself; U is kept up to column signs
+    # shampoo_beta = 1: the factor is L itself; L U = U diag(lam) with lam > 0,
+    # so the positive-diagonal QR returns U exactly (R = diag(lam))
     out = soap.soap_step(Z, Z, Z, Z, L, U, None, None, shampoo_beta=1.0)
-    np.testing.assert_allclose(np.abs(np.sum(out["QL"] * U, axis=0)), np.ones(m), atol=1e-12)
-    # a factor that has seen only zero gradients keeps its basis: d = 1 and
-    # the positive-diagonal QR of an orthogonal U is U itself (R = I)
+    np.testing.assert_allclose(out["QL"], U, atol=1e-12)
+    # a factor that has seen only zero gradients: L Q = 0, whose Householder
+    # QR has only trivial reflectors, Q = I (R = 0, no column sign to fix)
     out = soap.soap_step(Z, Z, Z, Z, np.zeros((m, m)), U, None, None)
+    np.testing.assert_array_equal(out["QL"], np.eye(m))
+    # the damped option keeps the basis there instead: d = 1, qr(U) = U
+    out = soap.soap_step(Z, Z, Z, Z, np.zeros((m, m)), U, None, None, damping=1e-5)
     np.testing.assert_allclose(out["QL"], U, atol=1e-12)
 
 

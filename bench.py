@@ -475,8 +475,7 @@ def heads_gpu(count, dim, dev, cond=1e4):
     s = s * (dim / s.norm())
     U, _ = torch.linalg.qr(torch.randn(count, dim, dim, generator=g, device=dev))
     V, _ = torch.linalg.qr(torch.randn(count, dim, dim, generator=g, device=dev))
-    G = (U * s) @ V.transpose(1, 2)
-    return [G[i].contiguous() for i in range(count)]
+    return ((U * s) @ V.transpose(1, 2)).contiguous()
 
 
 def soap_flops(m, n, left, right):
@@ -532,13 +531,13 @@ def soap_bench(ctx, dev, steps=3, warm=10):
         f, r = soap_flops(d["W"].shape[0], d["W"].shape[1], "L" in d, "R" in d)
         fl += f
         rot += r
-    hp = dict(lr=3e-3, beta1=0.95, beta2=0.95, eps=1e-8, weight_decay=0.0)
+    hp = dict(lr=3e-3, beta1=0.95, beta2=0.95, eps=1e-8, weight_decay=0.0, damping=0.0)
     for t in range(1, warm + 1):
         fill()
         ctx.soap_step(mats, t, **hp)
     torch.cuda.synchronize()
-    ctx.profile(True)
-    ctx.profile_read()
+    # steps warm + 1 .. warm + steps timed as they run; the per-kernel
+    # breakdown comes from as many further steps with the launch events on
     total = 0.0
     for t in range(warm + 1, warm + 1 + steps):
         fill()
@@ -549,13 +548,20 @@ def soap_bench(ctx, dev, steps=3, warm=10):
         e.record()
         torch.cuda.synchronize()
         total += s.elapsed_time(e)
+    ctx.profile(True)
+    ctx.profile_read()
+    for t in range(warm + 1 + steps, warm + 1 + 2 * steps):
+        fill()
+        ctx.soap_step(mats, t, reserve=False, **hp)
+    torch.cuda.synchronize()
     prof = ctx.profile_read()
     ctx.profile(False)
     ms = total / steps
     k = {kk: round(v[0] / steps, 3) for kk, v in prof.items() if v[2]}
     rot_ms = prof["soap_rot"][0] / steps
     rot_exec = prof["soap_rot"][1] / steps
-    return {"workload": "soap_step 4 x 4096^2 (two-sided) + 4 x 4096x14336 (left side only), step 11",
+    return {"workload": f"soap_step 4 x 4096^2 (two-sided) + 4 x 4096x14336 (left side only), steps "
+                        f"{warm + 1}-{warm + steps} after {warm} warm steps; refresh qr(L Q), damping 0",
             "ms": round(ms, 3), "TFLOP/s": round(fl / (ms / 1e3) / 1e12, 1),
             "flops_per_step": fl, "matrices_per_s": round(len(mats) / (ms / 1e3), 1),
             "kernels_ms_per_step": k,
@@ -563,6 +569,7 @@ def soap_bench(ctx, dev, steps=3, warm=10):
                               "useful_TFLOP/s": round(rot / (rot_ms / 1e3) / 1e12, 1) if rot_ms else None,
                               "executed_TFLOP/s": round(rot_exec / (rot_ms / 1e3) / 1e12, 1) if rot_ms else None,
                               "note": "two-plane operands: 3 bf16 MMAs per useful product"},
+            "kernels_note": "kernels_ms_per_step: further steps with per-launch events (their overhead included)",
             "gpu_launches": int(sum(v[2] for v in prof.values()) / steps)}
 
 
@@ -578,13 +585,11 @@ def soap_muon_bench(ctx, dev, steps=3, warm=10):
         m, n = d["W"].shape
         f, _ = soap_flops(m, n, "L" in d, "R" in d)
         fl += f + page_flops(m, n)
-    hp = dict(lr=0.02, weight_decay=0.01, momentum=0.95, beta2=0.95, shampoo_beta=0.9, eps=1e-8)
+    hp = dict(lr=0.02, weight_decay=0.01, momentum=0.95, beta2=0.95, shampoo_beta=0.9, eps=1e-8, damping=0.0)
     for t in range(1, warm + 1):
         fill()
         ctx.soap_muon_step(mats, t, **hp)
     torch.cuda.synchronize()
-    ctx.profile(True)
-    ctx.profile_read()
     total = 0.0
     for t in range(warm + 1, warm + 1 + steps):
         fill()
@@ -595,10 +600,17 @@ def soap_muon_bench(ctx, dev, steps=3, warm=10):
         e.record()
         torch.cuda.synchronize()
         total += s.elapsed_time(e)
+    ctx.profile(True)
+    ctx.profile_read()
+    for t in range(warm + 1 + steps, warm + 1 + 2 * steps):
+        fill()
+        ctx.soap_muon_step(mats, t, reserve=False, **hp)
+    torch.cuda.synchronize()
     prof = ctx.profile_read()
     ctx.profile(False)
     ms = total / steps
-    return {"workload": "soap_muon_step on the SOAP matrices (4 x 4096^2 two-sided, 4 x 4096x14336 left side), step 11",
+    return {"workload": f"soap_muon_step on the SOAP matrices (4 x 4096^2 two-sided, 4 x 4096x14336 left side), "
+                        f"steps {warm + 1}-{warm + steps}; refresh qr(L Q), damping 0",
             "ms": round(ms, 3), "TFLOP/s": round(fl / (ms / 1e3) / 1e12, 1), "flops_per_step": fl,
             "matrices_per_s": round(len(mats) / (ms / 1e3), 1),
             "kernels_ms_per_step": {kk: round(v[0] / steps, 3) for kk, v in prof.items() if v[2]},
@@ -703,13 +715,16 @@ def extras(ctx, dev, args):
         del Gt, out
         ctx.workspace = None
         torch.cuda.empty_cache()
-    Ht = heads_gpu(4096, 128, dev)
-    Ho = [torch.empty_like(h) for h in Ht]
+    Ht = heads_gpu(4096, 128, dev)                    # one [4096, 128, 128] tensor
+    Ho = torch.empty_like(Ht)
     ctx.reserve(2, [(128, 128)] * 4096)
-    call = lambda: ctx.ns_orthogonalize(Ht, Ho, reserve=False)
-    ms_eager = time_steps(call, 5, 2)
-    # the same call replayed from a CUDA graph (no per-call host marshalling
-    # of 4096 tensors): the device time of the fused small-matrix kernel
+    call = lambda: ctx.ns_orthogonalize_batch(Ht, Ho, reserve=False)
+    ms_eager = time_steps(call, 20, 3)
+    # the per-matrix list form of the same call (4096 tensors marshalled)
+    Hl, Hol = list(Ht.unbind(0)), list(Ho.unbind(0))
+    ms_list = time_steps(lambda: ctx.ns_orthogonalize(Hl, Hol, reserve=False), 5, 2)
+    del Hl, Hol
+    # the same call replayed from a CUDA graph: the device time alone
     graph = capture_graph(call)
     ms = time_steps(graph.replay, 20, 3)
     del graph
@@ -721,10 +736,11 @@ def extras(ctx, dev, args):
     ctx.profile(False)
     fl = 4096 * page_flops(128, 128)
     sweep["heads_4096x128x128"] = {"ms": round(ms, 3), "TFLOP/s": round(fl / (ms / 1e3) / 1e12, 2),
-                                   "eager_call_ms": round(ms_eager, 3),
+                                   "eager_call_ms": round(ms_eager, 3), "list_call_ms": round(ms_list, 3),
                                    "ns_small_kernel_ms": round(kern[0], 3), "ns_small_launches": kern[2],
-                                   "note": "ms: CUDA-graph replay; eager_call_ms includes the "
-                                           "binding's per-tensor marshalling"}
+                                   "note": "ms: CUDA-graph replay; eager_call_ms: the strided batch call "
+                                           "(ns_orthogonalize_strided) eagerly; list_call_ms: the same "
+                                           "matrices as a list of 4096 tensors"}
     res["ns_sweep"] = sweep
     del Ht, Ho
     ctx.workspace = None

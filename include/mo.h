@@ -171,6 +171,21 @@ MO_API mo_status ns_orthogonalize(mo_ctx* ctx, const float* const* in, float* co
                            const int64_t* rows, const int64_t* cols, int n, const mo_ns_cfg* cfg,
                            void* stream);
 
+/* ------------------------------------------------------------------ strided batches
+ * The same calls for n matrices of one shape stored at a fixed stride (in
+ * elements) from one base pointer, e.g. the per-head matrices of a model
+ * held as one [n][rows][cols] tensor: the caller passes O(1) arguments
+ * whatever n is.  Matrix i of `in` starts at in + i * in_stride, and
+ * likewise for out, W, G and the momentum (one stride for the three).
+ * Strides must be at least rows * cols when n > 1.  Everything else,
+ * including validation, alignment rules and the nonfinite array (indexed by
+ * i), is that of ns_orthogonalize and muon_step. */
+MO_API mo_status ns_orthogonalize_strided(mo_ctx* ctx, const float* in, int64_t in_stride, float* out,
+                                          int64_t out_stride, int64_t rows, int64_t cols, int n,
+                                          const mo_ns_cfg* cfg, void* stream);
+MO_API mo_status muon_step_strided(mo_ctx* ctx, float* W, const float* G, float* momentum, int64_t stride,
+                                   int64_t rows, int64_t cols, int n, const mo_muon_cfg* cfg, void* stream);
+
 /* ------------------------------------------------------------------ no-allocation variant
  * The pages have no counterpart to this entry point; it serves callers that
  * cannot allocate device memory when they call it: programs whose GPU
@@ -208,14 +223,16 @@ MO_API mo_status ns_orthogonalize_static(mo_ctx* ctx, const float* in, float* ou
  * notes on SOAP, Muon, and Beyond", sections 1 and 4; "LLM Optimizers",
  * section 11.1; "初探优化器（一）", section 6.2), at step t >= 1:
  *   L <- bs L + (1 - bs) G G^T,   R <- bs R + (1 - bs) G^T G
- *   Q_L <- qr((L + dL I) Q_L),    Q_R <- qr((R + dR I) Q_R)
- *                                 (one power step + QR, diag(R) > 0,
- *                                  fp32-accurate; dL = damping * trace(L),
- *                                  or 1 when the trace is zero: the damping
- *                                  of the Shampoo family, "Matrix optimizers:
- *                                  K-FAC, Shampoo and Muon", Shampoo; it keeps
- *                                  the eigenvectors and bounds cond by
- *                                  1 + 1 / damping)
+ *   Q_L <- qr(L Q_L),             Q_R <- qr(R Q_R)
+ *                                 (one power step + QR, the current gradient
+ *                                  included; diag(R) > 0; fp32-accurate: every
+ *                                  refresh product takes fp16 two-plane
+ *                                  operands; CholeskyQR passes, plain or
+ *                                  shifted per matrix, until the basis is
+ *                                  orthonormal to 5e-5.  Where L Q is singular
+ *                                  its QR is not unique and the basis is
+ *                                  completed arbitrarily (a zero factor gives
+ *                                  Q = I, as Householder QR does))
  *   M <- b1 M + (1 - b1) G        (original space)
  *   M' = Q_L^T M Q_R,  G' = Q_L^T G Q_R
  *   V <- b2 V + (1 - b2) G' * G'
@@ -240,14 +257,18 @@ typedef struct {
 typedef struct {
   float lr, beta1, beta2, shampoo_beta, eps, weight_decay;
   int bias_correction;  /* 1: divide by 1 - beta^t (default) */
-  int32_t* nonfinite;   /* optional device int32[n]: the QR met a non-positive pivot */
+  int32_t* nonfinite;   /* optional device int32[n]: 1 when a basis refresh did
+                           not reach an orthonormal basis (non-finite input,
+                           or more CholeskyQR passes needed than allowed) */
   int skip_refresh;     /* 1: update L, R but keep Q_L, Q_R this step (the steps
                            between refreshes when the basis is refreshed only
                            every f steps); 0: refresh every step (default) */
-  float damping;        /* relative damping of the power step, in (0, 1e-2]
-                           (1e-5 by default in the binding); with damping
-                           below 1e-6 the fp32 Cholesky QR may meet a
-                           non-positive pivot on singular factors */
+  float damping;        /* 0 (default): the pages' power step qr(L Q).  In
+                           (0, 1e-2]: an option that departs from the pages,
+                           qr((L + d I) Q) with d = damping * trace(L) (1 when
+                           the trace is 0), the damping of the Shampoo family
+                           ("Matrix optimizers: K-FAC, Shampoo and Muon",
+                           Shampoo); it changes the update */
 } mo_soap_cfg;
 
 MO_API mo_status soap_step(mo_ctx* ctx, const mo_soap_mat* mats /* host array */, int n,
@@ -301,7 +322,8 @@ typedef struct {
   int bias_correction;  /* 1: V / (1 - b2^t) */
   int ns_steps; float a, b, c, ns_eps;
   int adjust_lr;        /* 0: 0.2 sqrt(max(m, n)); 1: sqrt(max(1, m / n)) */
-  float damping;        /* relative damping of the power step, (0, 1e-2] */
+  float damping;        /* as in mo_soap_cfg: 0 = qr(L Q) (default), or the
+                           damped option in (0, 1e-2] */
   int32_t* nonfinite;   /* optional device int32[n] */
   int skip_refresh;     /* 1: keep the bases (factors still update) */
 } mo_soap_muon_cfg;

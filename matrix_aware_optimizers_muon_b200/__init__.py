@@ -83,6 +83,7 @@ class Context:
         self.handle = h
         self.workspace = None
         self.retired = []       # workspaces replaced during stream capture, kept alive
+        self._batch_reserved = {}
 
     def close(self):
         if getattr(self, "handle", None):
@@ -212,13 +213,64 @@ class Context:
                                               self._stream(stream)))
         return outputs
 
+    def _reserve_batch(self, op, rows, cols, n, stream):
+        """reserve() for n matrices of one shape, remembered per workspace so
+        that repeated calls on the same batch cost no workspace query."""
+        key = (op, rows, cols, n)
+        if self.workspace is not None and self._batch_reserved.get(key) == self.workspace.data_ptr():
+            return
+        self.reserve(op, [(rows, cols)] * n, stream=stream)
+        self._batch_reserved[key] = self.workspace.data_ptr()
+
+    @staticmethod
+    def _check_batch(t, name, shape=None):
+        _check_f32(t, name)
+        if t.dim() != 3 or (shape is not None and tuple(t.shape) != tuple(shape)):
+            raise ValueError(f"{name} must be a 3-D [n, rows, cols] tensor" +
+                             (f" of shape {tuple(shape)}" if shape is not None else ""))
+
+    def ns_orthogonalize_batch(self, X, out=None, *, ns_steps=5, coeffs=QUINTIC, eps=1e-7, nonfinite=None,
+                               stream=None, reserve=True):
+        """out[i] = NS(X[i]) for a contiguous fp32 tensor X of shape [n, rows,
+        cols] (e.g. per-head matrices): one call whatever n is."""
+        import torch
+        self._check_batch(X, "X")
+        if out is None:
+            out = torch.empty_like(X)
+        self._check_batch(out, "out", X.shape)
+        n, r, c = X.shape
+        if reserve:
+            self._reserve_batch(OP_NS, r, c, n, stream)
+        cfg = NsCfg(ns_steps, coeffs[0], coeffs[1], coeffs[2], eps, _ptr(nonfinite))
+        self._check(self.lib.ns_orthogonalize_strided(self.handle, _ptr(X), r * c, _ptr(out), r * c, r, c, n,
+                                                      byref(cfg), self._stream(stream)))
+        return out
+
+    def muon_step_batch(self, W, G, B, *, lr=0.02, weight_decay=0.01, momentum=0.95, nesterov=True,
+                        momentum_ema=False, ns_steps=5, coeffs=QUINTIC, eps=1e-7,
+                        adjust_lr="match_rms_adamw", nonfinite=None, stream=None, reserve=True):
+        """One Muon step on n matrices of one shape held as contiguous fp32
+        [n, rows, cols] tensors W, G and B."""
+        self._check_batch(W, "W")
+        self._check_batch(G, "G", W.shape)
+        self._check_batch(B, "B", W.shape)
+        n, r, c = W.shape
+        if reserve:
+            self._reserve_batch(OP_MUON, r, c, n, stream)
+        modes = {"match_rms_adamw": 0, "original": 1}
+        cfg = MuonCfg(lr, weight_decay, momentum, int(nesterov), int(momentum_ema), ns_steps,
+                      coeffs[0], coeffs[1], coeffs[2], eps, modes[adjust_lr], _ptr(nonfinite))
+        self._check(self.lib.muon_step_strided(self.handle, _ptr(W), _ptr(G), _ptr(B), r * c, r, c, n,
+                                               byref(cfg), self._stream(stream)))
+
     def soap_step(self, mats, step, *, lr=3e-3, beta1=0.95, beta2=0.95, shampoo_beta=None,
                   eps=1e-8, weight_decay=0.0, bias_correction=True, nonfinite=None, stream=None,
-                  reserve=True, refresh=True, damping=1e-5):
+                  reserve=True, refresh=True, damping=0.0):
         """One SOAP step.  ``mats`` is a list of dicts with keys W, G, M, V and
         optionally L, QL, R, QR (missing or None: identity basis on that side).
         ``refresh=False`` keeps the bases this step (factors still update).
-        ``damping``: the power step runs on L + damping * trace(L) I."""
+        ``damping``: 0 is the pages' power step qr(L Q); a positive value
+        runs it on L + damping * trace(L) I instead (an option)."""
         n = len(mats)
         arr = (SoapMat * max(n, 1))()
         for i, d in enumerate(mats):
@@ -241,7 +293,7 @@ class Context:
 
     def soap_muon_step(self, mats, step, *, lr=0.02, weight_decay=0.01, momentum=0.95, nesterov=True,
                        beta2=0.95, shampoo_beta=0.9, eps=1e-8, bias_correction=True, ns_steps=5,
-                       coeffs=QUINTIC, ns_eps=1e-7, adjust_lr="match_rms_adamw", damping=1e-5,
+                       coeffs=QUINTIC, ns_eps=1e-7, adjust_lr="match_rms_adamw", damping=0.0,
                        nonfinite=None, refresh=True, stream=None, reserve=True):
         """One SOAP-Muon step.  ``mats``: dicts with W, G, B (Muon momentum), V
         and optionally L, QL, R, QR (missing or None: identity basis)."""

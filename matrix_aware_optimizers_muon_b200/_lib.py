@@ -103,6 +103,10 @@ SIGNATURES = {
                                              POINTER(c_size_t)]),
     "ns_orthogonalize_static": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64,
                                         POINTER(NsCfg), c_void_p]),
+    "ns_orthogonalize_strided": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_int64, c_int64, c_int64,
+                                         c_int, POINTER(NsCfg), c_void_p]),
+    "muon_step_strided": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int,
+                                  POINTER(MuonCfg), c_void_p]),
     "mo_profile_enable": (c_int, [c_void_p, c_int]),
     "mo_profile_read": (c_int, [c_void_p, POINTER(ctypes.c_double), POINTER(ctypes.c_double),
                                 POINTER(c_int64), c_int]),

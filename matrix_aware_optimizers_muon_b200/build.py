@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmo.so")
-SOURCES = ["api.cu", "gemm.cu", "elementwise.cu", "ns.cu", "soap.cu", "profile.cu", "ns_static.cu", "soap_kernels.cu", "ns_small.cu"]
+SOURCES = ["api.cu", "gemm.cu", "elementwise.cu", "ns.cu", "soap.cu", "profile.cu", "ns_static.cu", "soap_kernels.cu", "ns_small.cu", "qr.cu"]
 HEADERS_DIRS = [CSRC, os.path.join(ROOT, "include")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

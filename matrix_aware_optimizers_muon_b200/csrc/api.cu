@@ -294,6 +294,49 @@ mo_status ns_orthogonalize(mo_ctx* ctx, const float* const* in, float* const* ou
   return MO_OK;
 }
 
+// Strided batches of equal shape: the per-matrix pointer lists are built
+// here, so the caller passes O(1) arguments for any number of matrices.
+mo_status ns_orthogonalize_strided(mo_ctx* ctx, const float* in, int64_t in_stride, float* out,
+                                   int64_t out_stride, int64_t rows, int64_t cols, int n, const mo_ns_cfg* cfg,
+                                   void* stream) {
+  if (ctx == nullptr) return MO_ERR_INVALID_ARG;
+  if (n < 0) return fail(ctx, MO_ERR_INVALID_ARG, "ns_orthogonalize_strided: n < 0");
+  if (n == 0) return MO_OK;
+  if (in == nullptr || out == nullptr || cfg == nullptr)
+    return fail(ctx, MO_ERR_INVALID_ARG, "ns_orthogonalize_strided: null argument");
+  if (rows <= 0 || cols <= 0 || (n > 1 && (in_stride < rows * cols || out_stride < rows * cols)))
+    return fail(ctx, MO_ERR_INVALID_ARG, "ns_orthogonalize_strided: bad shape or a stride below rows * cols");
+  std::vector<const float*> ins(n);
+  std::vector<float*> outs(n);
+  std::vector<int64_t> r(n, rows), c(n, cols);
+  for (int i = 0; i < n; ++i) {
+    ins[i] = in + (size_t)i * in_stride;
+    outs[i] = out + (size_t)i * out_stride;
+  }
+  return ns_orthogonalize(ctx, ins.data(), outs.data(), r.data(), c.data(), n, cfg, stream);
+}
+
+mo_status muon_step_strided(mo_ctx* ctx, float* W, const float* G, float* momentum, int64_t stride, int64_t rows,
+                            int64_t cols, int n, const mo_muon_cfg* cfg, void* stream) {
+  if (ctx == nullptr) return MO_ERR_INVALID_ARG;
+  if (n < 0) return fail(ctx, MO_ERR_INVALID_ARG, "muon_step_strided: n < 0");
+  if (n == 0) return MO_OK;
+  if (W == nullptr || G == nullptr || momentum == nullptr || cfg == nullptr)
+    return fail(ctx, MO_ERR_INVALID_ARG, "muon_step_strided: null argument");
+  if (rows <= 0 || cols <= 0 || (n > 1 && stride < rows * cols))
+    return fail(ctx, MO_ERR_INVALID_ARG, "muon_step_strided: bad shape or a stride below rows * cols");
+  std::vector<mo_muon_mat> mats(n);
+  for (int i = 0; i < n; ++i) {
+    const size_t off = (size_t)i * stride;
+    mats[i].rows = rows;
+    mats[i].cols = cols;
+    mats[i].W = W + off;
+    mats[i].G = G + off;
+    mats[i].momentum = momentum + off;
+  }
+  return muon_step(ctx, mats.data(), n, cfg, stream);
+}
+
 // ---------------------------------------------------------------- SOAP
 
 namespace {
@@ -309,8 +352,8 @@ mo_status soap_impl(mo_ctx* ctx, const mo_soap_mat* mats, int n, const mo_soap_c
   auto beta_ok = [](float b) { return b >= 0.f && b < 1.f; };
   if (!beta_ok(cfg->beta1) || !beta_ok(cfg->beta2) || !beta_ok(cfg->shampoo_beta))
     return fail(ctx, MO_ERR_INVALID_ARG, fn + ": betas must be in [0, 1)");
-  if (!(cfg->damping > 0.f && cfg->damping <= 1e-2f))
-    return fail(ctx, MO_ERR_INVALID_ARG, fn + ": damping must be in (0, 1e-2]");
+  if (!(cfg->damping >= 0.f && cfg->damping <= 1e-2f))
+    return fail(ctx, MO_ERR_INVALID_ARG, fn + ": damping must be in [0, 1e-2]");
   std::vector<mo::SoapItem> items;
   for (int i = 0; i < n; ++i) {
     const mo_soap_mat& m = mats[i];

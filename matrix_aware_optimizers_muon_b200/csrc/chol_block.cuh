@@ -11,8 +11,8 @@
 // 256 threads; A and X are [128][129] fp32 (row stride 129), T is [32][97]
 // scratch.  A holds the block on entry (lower triangle read) and L on exit
 // (lower triangle); X receives L^{-1} (lower triangle; the upper triangle is
-// not written).  Returns through *bad whether a pivot was not positive
-// (NaN included).
+// not written).  Returns through *bad whether a pivot was not above the
+// floor (0 by default: not positive; NaN included).
 #pragma once
 
 namespace mo {
@@ -24,10 +24,12 @@ constexpr int CB_T_LD = 97;
 // Step J of the warp-level 32 x 32 factorisation (lane i holds row i in
 // r[0..31]); a template so that every register index is a constant.
 template <int J>
-__device__ __forceinline__ void chol32_step(float (&r)[32], int lane, bool& ok, float* inv_diag) {
+__device__ __forceinline__ void chol32_step(float (&r)[32], int lane, bool& ok, float* inv_diag, float floor,
+                                            float& mp) {
   if constexpr (J < 32) {
     const float d = __shfl_sync(0xffffffffu, r[J], J);
-    ok = ok && (d > 0.f);
+    ok = ok && (d > floor);
+    mp = fminf(mp, d);
     const float sq = sqrtf(d);
     const float inv = 1.0f / sq;
     if (lane == J) {
@@ -41,11 +43,15 @@ __device__ __forceinline__ void chol32_step(float (&r)[32], int lane, bool& ok, 
       const float lcj = __shfl_sync(0xffffffffu, r[J], c);
       if (c <= lane) r[c] = fmaf(-r[J], lcj, r[c]);
     }
-    chol32_step<J + 1>(r, lane, ok, inv_diag);
+    chol32_step<J + 1>(r, lane, ok, inv_diag, floor, mp);
   }
 }
 
-__device__ __forceinline__ void chol128_factor(float* A, float* inv_diag, int* bad) {
+// `floor`: a pivot (diagonal of the Schur complement before its square root)
+// at or below it sets *bad; *minpiv (optional, shared) receives the smallest
+// pivot met.
+__device__ __forceinline__ void chol128_factor(float* A, float* inv_diag, int* bad, float floor = 0.f,
+                                               float* minpiv = nullptr) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int kb = 0; kb < 4; ++kb) {
     const int b0 = 32 * kb;
@@ -55,7 +61,9 @@ __device__ __forceinline__ void chol128_factor(float* A, float* inv_diag, int* b
 #pragma unroll
       for (int c = 0; c < 32; ++c) r[c] = c <= lane ? A[(b0 + lane) * CB_LD + b0 + c] : 0.f;
       bool ok = true;
-      chol32_step<0>(r, lane, ok, inv_diag + b0);
+      float mp = __int_as_float(0x7f800000);
+      chol32_step<0>(r, lane, ok, inv_diag + b0, floor, mp);
+      if (lane == 0 && minpiv != nullptr) *minpiv = fminf(*minpiv, mp);
 #pragma unroll
       for (int c = 0; c < 32; ++c)
         if (c <= lane) A[(b0 + lane) * CB_LD + b0 + c] = r[c];

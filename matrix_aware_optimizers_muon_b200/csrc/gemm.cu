@@ -31,7 +31,7 @@ void load_encode_fn() {
 // (row stride ld, matrix stride bstride, plane stride pstride, all in
 // elements); box = 64 x box_rows.
 bool encode_bf16_4d(CUtensorMap* map, const void* ptr, long long rows, long long cols, long long ld,
-                    long long bstride, int batch, long long pstride, int planes, int box_rows) {
+                    long long bstride, int batch, long long pstride, int planes, int box_rows, bool f16 = false) {
   std::call_once(g_encode_once, load_encode_fn);
   if (g_encode == nullptr) return false;
   const long long bs = batch > 1 ? bstride : rows * ld;
@@ -40,7 +40,8 @@ bool encode_bf16_4d(CUtensorMap* map, const void* ptr, long long rows, long long
   cuuint64_t strides[3] = {(cuuint64_t)(ld * 2), (cuuint64_t)(bs * 2), (cuuint64_t)(ps * 2)};
   cuuint32_t box[4] = {64u, (cuuint32_t)box_rows, 1u, 1u};
   cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
+  CUresult r = g_encode(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                        const_cast<void*>(ptr), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -104,11 +105,13 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   if (nseg > 8 || (nseg > 1 && op.K % (nseg * GEMM_BK) != 0)) return cudaErrorInvalidValue;
   const long long kseg = op.K / nseg;
   const int pa = planes_of(op.pat_a, nseg), pb = planes_of(op.pat_b, nseg);
-  const bool ok_a = A_MN ? encode_bf16_4d(&ta, op.A, kseg, op.M, op.lda, op.strideA, op.batch, op.planeA, pa, 64)
-                         : encode_bf16_4d(&ta, op.A, op.M, kseg, op.lda, op.strideA, op.batch, op.planeA, pa, GEMM_BM);
-  const bool ok_b = B_MN ? encode_bf16_4d(&tb, op.B, kseg, op.N, op.ldb, op.strideB, op.batch, op.planeB, pb, 64)
+  const bool h = op.ab_f16 != 0;
+  const bool ok_a = A_MN ? encode_bf16_4d(&ta, op.A, kseg, op.M, op.lda, op.strideA, op.batch, op.planeA, pa, 64, h)
+                         : encode_bf16_4d(&ta, op.A, op.M, kseg, op.lda, op.strideA, op.batch, op.planeA, pa, GEMM_BM,
+                                          h);
+  const bool ok_b = B_MN ? encode_bf16_4d(&tb, op.B, kseg, op.N, op.ldb, op.strideB, op.batch, op.planeB, pb, 64, h)
                          : encode_bf16_4d(&tb, op.B, op.N, kseg, op.ldb, op.strideB, op.batch, op.planeB, pb,
-                                          Cfg::BN_LOCAL);
+                                          Cfg::BN_LOCAL, h);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
 
   GemmParams p;
@@ -137,6 +140,7 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   p.ap_step[1] = op.ap_step[1];
   p.ap_tall_from = op.ap_tall_from;
   p.ap_vec = op.ap_vec;
+  p.ab_f16 = op.ab_f16;
   if (op.epi == EPI_APPLY && (op.sym || op.e_tab == nullptr || op.d_f32 || op.d_split))
     return cudaErrorInvalidValue;
   // a strided bf16 C of the plain (or Muon apply) epilogue is read by TMA

@@ -1,4 +1,4 @@
-// Batched bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM),
+// Batched bf16 (or fp16) GEMM on the 5th-generation tensor cores (tcgen05 + TMEM),
 // fed by TMA, with a fused epilogue: D = alpha_b * (A B) + beta_b * C, the
 // Adam step of SOAP in the rotated basis (EPI_ADAM), or the Muon apply
 // W <- decay W - step bf16(alpha_b A B + beta_b C) into fp32 W (EPI_APPLY).
@@ -77,6 +77,9 @@ struct GemmParams {
   float ap_step[2];
   int ap_tall_from;
   int ap_vec;               // every W of the launch: 16-byte aligned rows
+  // A and B hold fp16 (not bf16) values: the same kind::f16 MMA with the
+  // operand type fields of the instruction descriptor set to f16
+  int ab_f16;
 };
 
 enum { EPI_AXPBY = 0, EPI_ADAM = 1, EPI_APPLY = 2 };
@@ -466,7 +469,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   constexpr int STAGES = Cfg::STAGES;
   constexpr int BM_T = PAIR ? 2 * GEMM_BM : GEMM_BM;     // rows per tile
   constexpr int BN_L = Cfg::BN_LOCAL;                     // B rows staged by this CTA
-  constexpr uint32_t IDESC = idesc_bf16_f32(BM_T, BN, A_MN, B_MN);
+  constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM_T, BN, A_MN, B_MN);
+  const uint32_t IDESC = p.ab_f16 ? idesc_as_f16(IDESC_BF16) : IDESC_BF16;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

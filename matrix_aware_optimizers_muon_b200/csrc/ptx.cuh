@@ -308,6 +308,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
          | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// The same descriptor with A and B read as fp16 (type code 0 in both
+// operand type fields of kind::f16) instead of bf16 (code 1).
+__host__ __device__ constexpr uint32_t idesc_as_f16(uint32_t bf16_desc) {
+  return bf16_desc & ~((7u << 7) | (7u << 10));
+}
+
 __device__ __forceinline__ uint32_t elect_one_lane() {
   return (threadIdx.x & 31u) == 0u;
 }

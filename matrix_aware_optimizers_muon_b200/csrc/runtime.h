@@ -71,7 +71,8 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-// One batched GEMM D_b = alpha_b * (A_b B_b) + beta_b * C_b on bf16 operands.
+// One batched GEMM D_b = alpha_b * (A_b B_b) + beta_b * C_b on bf16 (or,
+// with ab_f16, fp16) operands.
 // Operand storage (row-major, element strides):
 //   A: a_mn ? [K rows][M cols] : [M rows][K cols]
 //   B: b_mn ? [K rows][N cols] : [N rows][K cols]
@@ -125,6 +126,8 @@ struct GemmOp {
   long long d_plane = 0;
   // per-matrix skip flags in device memory (optional)
   const int* skip = nullptr;
+  // A and B hold fp16 values (both; the MMA takes one type for the two)
+  int ab_f16 = 0;
 };
 
 // Launch the tcgen05 GEMM.  Returns cudaSuccess or the launch/encode error.

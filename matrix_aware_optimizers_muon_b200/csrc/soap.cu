@@ -5,15 +5,11 @@
 //   EMAs:  L <- bs L + (1-bs) Gb Gb^T ; R <- bs R + (1-bs) Gb^T Gb
 //          (symmetric tcgen05 products written into the caller's L / R)
 // Phase 2 (per bucket of equal factor size k, all sides of all matrices):
-//   power: Y = (L + d I) Q, d = damping * trace(L), fp32-accurate
-//          (3-plane bf16 split, 6 plane products)
-//   QR:    shifted CholeskyQR3: up to three passes of
-//            column-normalise Y, C = Y^T Y (fp32-accurate), [shift C],
-//            blocked Cholesky C = L L^T with 128-wide diagonal blocks and
-//            Y <- Y L^{-T} (right-looking, tensor-core trailing updates);
-//          the third pass is skipped per matrix when its Gram is already
-//          within 5e-5 of the identity (every warm step)
-//          -> Q (unique QR, diag(R) > 0) into the caller's Q and bf16(Q)
+//   the refresh Q <- qr(F Q) of qr.cuh: the power step as an fp16
+//   two-plane product, then CholeskyQR passes (left-looking blocked
+//   Cholesky of the Gram with the solve for Q in the same products), plain
+//   or shifted per matrix as the conditioning needs, until the basis is
+//   orthonormal -> Q (unique QR, diag(R) > 0) into the caller's Q and bf16(Q)
 // Phase 3 (per group): rotations with two-plane bf16 operands (x = h + l,
 //   three bf16 MMAs lh + hl + hh per product), Adam in the rotated basis
 //   fused into the epilogue of the G' product, rotation back fused with
@@ -28,6 +24,7 @@
 
 #include "ns_plan.h"
 #include "profile.h"
+#include "qr.cuh"
 #include "runtime.h"
 #include "soap_kernels.cuh"
 #include "soap_plan.h"
@@ -39,24 +36,10 @@ namespace {
 constexpr size_t AL = 1024;
 size_t al(size_t x) { return (x + AL - 1) / AL * AL; }
 
-// plane products of the fp32-accurate GEMMs: x = h + m + l, and
-// x y ~ hh + hm + mh + hl + lh + mm  (dropped terms are below 2^-24).  The
-// small products are accumulated first and hh last: the tensor core's fp32
-// accumulation loses low-order bits of each addend that is small next to
-// the running sum, so adding the small terms into an accumulator that
-// already holds hh would cost most of their accuracy.
-const unsigned char PAT_A[6] = {1, 2, 0, 1, 0, 0};
-const unsigned char PAT_B[6] = {1, 0, 2, 0, 1, 0};
-
-void set_planes(GemmOp& g, long long planeA, long long planeB) {
-  g.nseg = 6;
-  for (int i = 0; i < 6; ++i) { g.pat_a[i] = PAT_A[i]; g.pat_b[i] = PAT_B[i]; }
-  g.planeA = planeA;
-  g.planeB = planeB;
-}
-
-// two-plane products of the rotations: x = h + l, x y ~ lh + hl + hh
-// (small products first, as above)
+// two-plane products: x = h + l, x y ~ lh + hl + hh (bf16 planes for the
+// rotations, fp16 planes with ab_f16 for the refresh).  The small products
+// are accumulated first and hh last: the tensor core's fp32 accumulation
+// loses low-order bits of each addend that is small next to the running sum.
 void set_planes2(GemmOp& g, long long planeA, long long planeB) {
   const unsigned char pa[3] = {1, 0, 0}, pb[3] = {0, 1, 0};
   g.nseg = 3;
@@ -81,10 +64,14 @@ struct Job {
   bool left;       // left factor (k = m) or right (k = n)
 };
 
+// Per bucket of equal factor side k (kp = k rounded up to 128): the stacked
+// fp32 [C; Y] and fp16 planes [L; Q] of the refresh ([q][2 kp][kp] each, two
+// planes), the diagonal-block inverses, column scales, the optional damping
+// and the pass-control state.
 struct Bucket {
   long long k, kp;
   std::vector<Job> jobs;
-  size_t y, c, ypl, qpl, ppl, qjpl, dinv, invd, damp, qdev, qskip;
+  size_t cy, lq, dinv, invd, damp, ctl;
 };
 
 struct Plan {
@@ -147,17 +134,12 @@ Plan make_plan(const std::vector<SoapItem>& items, bool with_p = false) {
   }
   for (Bucket& b : P.buckets) {
     const size_t q = b.jobs.size(), kk = (size_t)b.kp * b.kp;
-    b.y = off; off += al(q * kk * 4);
-    b.c = off; off += al(q * kk * 4);
-    b.ypl = off; off += al(3 * q * kk * 2);
-    b.qpl = off; off += al(3 * q * kk * 2);
-    b.ppl = off; off += al(3 * q * b.kp * QR_B * 2);
-    b.qjpl = off; off += al(3 * q * b.kp * QR_B * 2);
+    b.cy = off; off += al(q * 2 * kk * 4);
+    b.lq = off; off += al(2 * q * 2 * kk * 2);
     b.dinv = off; off += al(q * QR_B * QR_B * 4);
     b.invd = off; off += al(q * b.kp * 4);
     b.damp = off; off += al(q * 4);
-    b.qdev = off; off += al(q * 4);
-    b.qskip = off; off += al(q * 4);
+    b.ctl = off; off += al(qr_ctl_bytes((int)q));
   }
   P.total = off;
   return P;
@@ -325,159 +307,126 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     return cudaGetLastError();
   };
-  // the per-step refresh: damped power step + shifted CholeskyQR3 per bucket
+  // the per-step refresh Q <- qr(F Q) per bucket (qr.cuh): the power step,
+  // then CholeskyQR passes until the basis is orthonormal
   auto refresh = [&]() -> cudaError_t {
     for (const Bucket& bk : P.buckets) {
       const int q = (int)bk.jobs.size();
-      const long long k = bk.k, kp = bk.kp, kk = kp * kp;
-      float* Y = at<float>(ws, bk.y);
-      float* C = at<float>(ws, bk.c);
-      __nv_bfloat16* Ypl = at<__nv_bfloat16>(ws, bk.ypl);
-      __nv_bfloat16* Qpl = at<__nv_bfloat16>(ws, bk.qpl);
-      __nv_bfloat16* Ppl = at<__nv_bfloat16>(ws, bk.ppl);
-      __nv_bfloat16* Qjpl = at<__nv_bfloat16>(ws, bk.qjpl);
+      const long long k = bk.k, kp = bk.kp, kk = kp * kp, ms = 2 * kk, pst = (long long)q * ms;
+      float* CY = at<float>(ws, bk.cy);           // [C; Y]
+      __half* LQ = at<__half>(ws, bk.lq);         // planes of [L; Q]
       float* Dinv = at<float>(ws, bk.dinv);
       float* invd = at<float>(ws, bk.invd);
+      const QrCtl ctl = qr_ctl_at(ws + bk.ctl, q);
       FlagTable flags;
       for (int j = 0; j < q; ++j) flags.f[j] = items[bk.jobs[j].item].flag;
+      auto factor_of = [&](int j) -> const float* {
+        const mo_soap_mat& m = items[bk.jobs[j].item].m;
+        return bk.jobs[j].left ? m.L : m.R;
+      };
+      auto basis_of = [&](int j) -> const float* {
+        const mo_soap_mat& m = items[bk.jobs[j].item].m;
+        return bk.jobs[j].left ? m.QL : m.QR;
+      };
+      launch_qr_init(ctl, q, s);
 
-      // power step: Y = (L + d I) Q, d = damping * trace(L) (planes of the
-      // damped L into Ypl, planes of the old Q into Qpl)
-      float* damp = at<float>(ws, bk.damp);
-      {
+      // power step Y = F Q_old (F + d I with the optional damping), both as
+      // fp16 planes padded with the identity; F's planes scaled per matrix
+      const float* delta = nullptr;
+      if (cfg.damping > 0.f) {
         DampArgs da;
-        da.count = q; da.k = (int)k; da.rho = cfg.damping; da.delta = damp;
-        for (int j = 0; j < q; ++j) {
-          const mo_soap_mat& m = items[bk.jobs[j].item].m;
-          da.F[j] = bk.jobs[j].left ? m.L : m.R;
-        }
+        da.count = q; da.k = (int)k; da.rho = cfg.damping; da.delta = at<float>(ws, bk.damp);
+        for (int j = 0; j < q; ++j) da.F[j] = factor_of(j);
         launch_damping(da, s);
+        delta = da.delta;
       }
-      SplitArgs sa;
-      sa.count = q; sa.rows_valid = (int)k; sa.cols_valid = (int)k; sa.rows_pad = (int)kp; sa.cols_pad = (int)kp;
-      sa.lds = k; sa.col_scale = nullptr; sa.write_back = nullptr; sa.ldw = 0; sa.wb_stride = 0;
-      sa.ldd = kp; sa.mat_stride = kk; sa.plane_stride = (long long)q * kk; sa.nplanes = 3; sa.pad_identity = 1;
-      for (int j = 0; j < q; ++j) {
-        const mo_soap_mat& m = items[bk.jobs[j].item].m;
-        sa.src[j] = bk.jobs[j].left ? m.L : m.R;
-      }
-      sa.dst = Ypl;
-      sa.diag_add = damp;
-      launch_split(sa, s);
-      sa.diag_add = nullptr;
-      for (int j = 0; j < q; ++j) {
-        const mo_soap_mat& m = items[bk.jobs[j].item].m;
-        sa.src[j] = bk.jobs[j].left ? m.QL : m.QR;
-      }
-      sa.dst = Qpl;
-      launch_split(sa, s);
+      FactorScaleArgs fs;
+      fs.count = q; fs.k = (int)k; fs.delta = delta;
+      for (int j = 0; j < q; ++j) fs.F[j] = factor_of(j);
+      launch_factor_scale(fs, ctl, s);
+      Split16Args sp;
+      sp.count = q; sp.rows_valid = sp.cols_valid = (int)k; sp.rows_pad = sp.cols_pad = (int)kp;
+      sp.lds = k; sp.dst = LQ; sp.ldd = kp; sp.mat_stride = ms; sp.plane_stride = pst; sp.pad_identity = 1;
+      for (int j = 0; j < q; ++j) sp.src[j] = factor_of(j);
+      sp.diag_add = delta;
+      sp.mscale = ctl.fscale;
+      launch_split16(sp, s);
+      for (int j = 0; j < q; ++j) sp.src[j] = basis_of(j);
+      sp.diag_add = nullptr;
+      sp.mscale = nullptr;
+      sp.cscale = QR_Y_SCALE;
+      sp.dst = LQ + kk;
+      launch_split16(sp, s);
       {
         GemmOp op;
-        op.A = Ypl; op.lda = kp; op.strideA = kk;          // L [i][p]: K-major
-        op.B = Qpl; op.ldb = kp; op.strideB = kk; op.b_mn = 1;   // Q [p][j]: MN-major
-        set_planes(op, (long long)q * kk, (long long)q * kk);
-        op.M = (int)kp; op.N = (int)kp; op.K = (int)(6 * kp); op.batch = q;
-        op.D = Y; op.ldd = kp; op.strideD = kk; op.d_f32 = 1;
+        op.A = LQ; op.lda = kp; op.strideA = ms;                           // F [i][p]: K-major
+        op.B = LQ + kk; op.ldb = kp; op.strideB = ms; op.b_mn = 1;        // Q_old [p][j]: MN-major
+        set_planes2(op, pst, pst);
+        op.ab_f16 = 1;
+        op.M = (int)kp; op.N = (int)kp; op.K = (int)(3 * kp); op.batch = q;
+        op.alpha = 1.f / QR_Y_SCALE; op.scale = ctl.fiscale; op.alpha_pow = 1;
+        op.D = CY + kk; op.ldd = kp; op.strideD = ms; op.d_f32 = 1;
         op.kind = PK_SOAP_QR;
         if ((e = launch_gemm(op, status, s)) != cudaSuccess) return e;
       }
 
-      // shifted CholeskyQR3
       const int nb = (int)(kp / QR_B);
-      for (int pass = 0; pass < 3; ++pass) {
-        launch_colnorm(Y, kp, kk, q, (int)kp, (int)kp, invd, s);
-        SplitArgs sy;
-        sy.count = q; sy.rows_valid = (int)kp; sy.cols_valid = (int)kp; sy.rows_pad = (int)kp; sy.cols_pad = (int)kp;
-        for (int j = 0; j < q; ++j) sy.src[j] = Y + (size_t)j * kk;
-        sy.lds = kp; sy.col_scale = invd; sy.write_back = Y; sy.ldw = kp; sy.wb_stride = kk;
-        sy.dst = Ypl; sy.ldd = kp; sy.mat_stride = kk; sy.plane_stride = (long long)q * kk;
-        sy.nplanes = 3; sy.pad_identity = 0;
-        launch_split(sy, s);
-        {   // C = Y^T Y, fp32-accurate, symmetric
-          GemmOp op;
-          op.A = Ypl; op.lda = kp; op.strideA = kk; op.a_mn = 1;
-          op.B = Ypl; op.ldb = kp; op.strideB = kk; op.b_mn = 1;
-          set_planes(op, (long long)q * kk, (long long)q * kk);
-          op.M = (int)kp; op.N = (int)kp; op.K = (int)(6 * kp); op.batch = q; op.sym = 1;
-          op.D = C; op.ldd = kp; op.strideD = kk; op.d_f32 = 1;
-          op.kind = PK_SOAP_QR;
-          if ((e = launch_gemm(op, status, s)) != cudaSuccess) return e;
+      for (int pass = 0; pass < QR_MAX_PASSES; ++pass) {
+        // normalise Y's columns (a zero column becomes e_c), planes of the
+        // result into the Q part of [L; Q], C = Y^T Y into the C part
+        launch_colnorm2(CY + kk, kp, ms, q, (int)kp, (int)kp, invd, ctl.done, s);
+        Split16Args sy;
+        sy.count = q; sy.rows_valid = sy.cols_valid = sy.rows_pad = sy.cols_pad = (int)kp;
+        for (int j = 0; j < q; ++j) sy.src[j] = CY + (size_t)j * ms + kk;
+        sy.lds = kp; sy.col_scale = invd; sy.cscale = QR_Y_SCALE;
+        sy.write_back = CY + kk; sy.ldw = kp; sy.wb_stride = ms;
+        sy.dst = LQ + kk; sy.ldd = kp; sy.mat_stride = ms; sy.plane_stride = pst;
+        sy.skip = ctl.done;
+        launch_split16(sy, s);
+        {
+          GemmOp g;
+          g.A = LQ + kk; g.lda = kp; g.strideA = ms; g.a_mn = 1;
+          g.B = LQ + kk; g.ldb = kp; g.strideB = ms; g.b_mn = 1;
+          set_planes2(g, pst, pst);
+          g.ab_f16 = 1;
+          g.M = (int)kp; g.N = (int)kp; g.K = (int)(3 * kp); g.batch = q; g.sym = 1;
+          g.alpha = 1.f / (QR_Y_SCALE * QR_Y_SCALE);
+          g.D = CY; g.ldd = kp; g.strideD = ms; g.d_f32 = 1;
+          g.kind = PK_SOAP_QR;
+          g.skip = ctl.done;
+          if ((e = launch_gemm(g, status, s)) != cudaSuccess) return e;
         }
-        // The first pass shifts the Gram matrix (unit diagonal, trace kp) by
-        // 1e-5 of its trace, above its fp32 rounding error.  With the damped
-        // factor, cond(Y) <= 1 + 1 / damping (1e5 at the default), and the
-        // shifted pass leaves a Q whose Gram the two unshifted passes
-        // factor safely (cond(Q) below the fp32 limit of Cholesky QR).
-        if (pass == 0) launch_shift_diag(C, kp, kk, q, (int)kp, 1e-5f * (float)kp, s);
-        // The last pass only corrects what is left of the previous pass's
-        // rounding.  A basis whose Gram is within 5e-5 of the identity keeps
-        // its (column-normalised) Q and every kernel of the pass skips it:
-        // the tensor core's fp32 accumulation leaves the Gram of an exactly
-        // orthonormal 4096-column basis about 2e-5 off the identity, so the
-        // pass could not lower the error below that floor, and the two-plane
-        // rotations that use the basis resolve 2^-16 = 1.5e-5.  Cold starts
-        // (deviation 1e-2 and more after the shifted pass) run all three.
-        const int* skip = nullptr;
-        if (pass == 2) {
-          launch_identity_check(C, kp, kk, q, (int)kp, 5e-5f, at<int>(ws, bk.qdev), at<int>(ws, bk.qskip), s);
-          skip = at<int>(ws, bk.qskip);
-        }
-        for (int jb = 0; jb < nb; ++jb) {
-          const long long k0 = (long long)jb * QR_B;
-          const long long rem = kp - k0 - QR_B;
-          launch_chol_diag(C, kp, kk, q, (int)k0, Dinv, flags, s, skip);
-          if (rem > 0) {      // panel L21 = C21 L11^{-T}, kept only as planes
-            RowBlockArgs ra;
-            ra.count = q; ra.rows = (int)rem;
-            ra.in = C + (k0 + QR_B) * kp + k0; ra.ld_in = kp; ra.in_stride = kk;
-            ra.out = nullptr; ra.ld_out = 0; ra.out_stride = 0;
-            ra.Dinv = Dinv;
-            ra.planes = Ppl; ra.plane_stride = (long long)q * kp * QR_B; ra.mat_stride = kp * QR_B;
-            ra.skip = skip;
-            launch_rowblock_dinv(ra, s);
-          }
-          {                   // Q_j = Y_j L_jj^{-T} (in place) and its planes
-            RowBlockArgs ra;
-            ra.count = q; ra.rows = (int)kp;
-            ra.in = Y + k0; ra.ld_in = kp; ra.in_stride = kk;
-            ra.out = Y + k0; ra.ld_out = kp; ra.out_stride = kk;
-            ra.Dinv = Dinv;
-            ra.planes = Qjpl; ra.plane_stride = (long long)q * kp * QR_B; ra.mat_stride = kp * QR_B;
-            ra.skip = skip;
-            launch_rowblock_dinv(ra, s);
-          }
-          if (rem > 0) {
-            GemmOp op;        // C22 -= L21 L21^T
-            op.A = Ppl; op.lda = QR_B; op.strideA = kp * QR_B;
-            op.B = Ppl; op.ldb = QR_B; op.strideB = kp * QR_B;
-            set_planes(op, (long long)q * kp * QR_B, (long long)q * kp * QR_B);
-            op.M = (int)rem; op.N = (int)rem; op.K = 6 * QR_B; op.batch = q; op.sym = 1;
-            op.alpha = -1.f; op.beta = 1.f;
-            float* c22 = C + (k0 + QR_B) * kp + (k0 + QR_B);
-            op.C = c22; op.ldc = kp; op.strideC = kk; op.c_f32 = 1;
-            op.D = c22; op.ldd = kp; op.strideD = kk; op.d_f32 = 1;
-            op.kind = PK_QR_TRAIL;
-            op.skip = skip;
-            if ((e = launch_gemm(op, status, s)) != cudaSuccess) return e;
-            GemmOp t;         // Y[:, k0+128:] -= Q_j L21^T
-            t.A = Qjpl; t.lda = QR_B; t.strideA = kp * QR_B;
-            t.B = Ppl; t.ldb = QR_B; t.strideB = kp * QR_B;
-            set_planes(t, (long long)q * kp * QR_B, (long long)q * kp * QR_B);
-            t.M = (int)kp; t.N = (int)rem; t.K = 6 * QR_B; t.batch = q;
-            t.alpha = -1.f; t.beta = 1.f;
-            float* yr = Y + (k0 + QR_B);
-            t.C = yr; t.ldc = kp; t.strideC = kk; t.c_f32 = 1;
-            t.D = yr; t.ldd = kp; t.strideD = kk; t.d_f32 = 1;
+        // done / plain / shifted per matrix, the shift on C's diagonal
+        launch_qr_control(CY, kp, ms, q, (int)kp, ctl, s);
+        for (int j = 0; j < nb; ++j) {
+          const long long r0 = (long long)j * QR_B;
+          if (j > 0) {     // [C; Y][r0 :, j] -= [L; Q][r0 :, < j] L[j, < j]^T
+            GemmOp t;
+            t.A = LQ + r0 * kp; t.lda = kp; t.strideA = ms;
+            t.B = LQ + r0 * kp; t.ldb = kp; t.strideB = ms;
+            set_planes2(t, pst, pst);
+            t.ab_f16 = 1;
+            t.M = (int)(2 * kp - r0); t.N = QR_B; t.K = (int)(3 * r0); t.batch = q;
+            t.alpha = -1.f / (QR_PLANE_SCALE * QR_PLANE_SCALE); t.beta = 1.f;
+            t.C = CY + r0 * kp + r0; t.ldc = kp; t.strideC = ms; t.c_f32 = 1;
+            t.D = CY + r0 * kp + r0; t.ldd = kp; t.strideD = ms; t.d_f32 = 1;
             t.kind = PK_QR_TRAIL;
-            t.skip = skip;
+            t.skip = ctl.skip;
             if ((e = launch_gemm(t, status, s)) != cudaSuccess) return e;
           }
+          launch_qr_chol(CY, kp, ms, q, j, Dinv, ctl, s);
+          PanelArgs pa;
+          pa.q = q; pa.j = j; pa.r0 = (int)(r0 + QR_B); pa.r1 = (int)(2 * kp); pa.f32_from = (int)kp;
+          pa.CY = CY; pa.ld = kp; pa.mat_stride = ms; pa.Dinv = Dinv;
+          pa.LQ = LQ; pa.plane_stride = pst; pa.skip = ctl.skip;
+          launch_qr_panel(pa, s);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
       }
+      launch_qr_finish(ctl, flags, q, s);
       // the new bases: fp32 into the caller's Q, bf16 into the group buffers
       CopyOutArgs co;
-      co.count = q; co.k = (int)k; co.Y = Y; co.ld = kp; co.mat_stride = kk;
+      co.count = q; co.k = (int)k; co.Y = CY + kk; co.ld = kp; co.mat_stride = ms;
       for (int j = 0; j < q; ++j) {
         const mo_soap_mat& m = items[bk.jobs[j].item].m;
         co.dst[j] = bk.jobs[j].left ? m.QL : m.QR;
@@ -492,7 +441,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
         SplitArgs one;
         one.count = 1; one.rows_valid = (int)k; one.cols_valid = (int)k;
         one.rows_pad = (int)kpad; one.cols_pad = (int)kpad;
-        one.src[0] = Y + (size_t)j * kk; one.lds = kp;
+        one.src[0] = CY + (size_t)j * ms + kk; one.lds = kp;
         one.col_scale = nullptr; one.write_back = nullptr; one.ldw = 0; one.wb_stride = 0;
         one.dst = at<__nv_bfloat16>(ws, jb.left ? g.qlp : g.qrp) + (size_t)jb.pos * kpad * kpad;
         one.ldd = kpad; one.mat_stride = 0;

@@ -59,45 +59,9 @@ struct DampArgs {
 };
 void launch_damping(const DampArgs& a, cudaStream_t s);
 
-// inv_d[b][c] = 1 / ||Y[b][:, c]||_2 over rows < rows (fixed summation order)
-void launch_colnorm(const float* Y, long long ld, long long mat_stride, int count, int rows, int cols,
-                    float* inv_d, cudaStream_t s);
-
-// C[b][i][i] += shift for i < n
-void launch_shift_diag(float* C, long long ld, long long mat_stride, int count, int n, float shift,
-                       cudaStream_t s);
-
 struct FlagTable {
   int32_t* f[SOAP_MAXB];           // per-matrix flag slots (entries may be null)
 };
-
-// Cholesky of the 128 x 128 diagonal block at (k0, k0) of each C[b] (lower
-// factor, fp32, in shared memory) and its inverse -> Dinv[b] (128 x 128,
-// lower).  A non-positive pivot sets *flag[b] = 1 (if given) and the block
-// inverse to NaN.
-void launch_chol_diag(const float* C, long long ld, long long mat_stride, int count, int k0,
-                      float* Dinv, const FlagTable& flags, cudaStream_t s, const int* skip = nullptr);
-
-// skip[b] = 1 when every entry of the leading k x k block of C[b] (row
-// stride ld) is within tol of the identity, else 0 (NaN never skips).
-// dev is scratch of `count` ints.  One Gram of an already orthonormal basis
-// lets the last CholeskyQR pass be skipped for that matrix.
-void launch_identity_check(const float* C, long long ld, long long mat_stride, int count, int k, float tol,
-                           int* dev, int* skip, cudaStream_t s);
-
-// out = in * Dinv^T for 128-wide row blocks: in/out are rows x 128 fp32
-// views (row stride ld); out may alias in.  Optionally writes the three bf16
-// planes of out to planes (+ p * plane_stride + b * mat_stride, row stride
-// 128) and skips the fp32 store.
-struct RowBlockArgs {
-  int count, rows;
-  const float* in; long long ld_in, in_stride;
-  float* out; long long ld_out, out_stride;         // may be null
-  const float* Dinv;                                 // [count][128][128]
-  __nv_bfloat16* planes; long long plane_stride, mat_stride;
-  const int* skip = nullptr;                         // per-matrix: leave untouched
-};
-void launch_rowblock_dinv(const RowBlockArgs& a, cudaStream_t s);
 
 // Final basis: Qout[b] (caller fp32 k x k) = Y[b][:k, :k]
 struct CopyOutArgs {

@@ -47,3 +47,28 @@ def ns_gate(N, O_gpu, O_ref, O_emu, *, tau=1e-2, sub_tol=2e-2, band=(0.6, 1.3), 
         assert band[0] <= sv.min() and sv.max() <= band[1], out
     assert full_gpu <= floor * full_emu + floor_abs, out
     return out
+
+
+def basis_gate(Q, Y, *, tau=1e-4, c=5e-6, orth=1e-4):
+    """A refreshed basis Q (GPU) against the positive-diagonal QR of Y = F Q_old
+    (fp64 oracle).
+
+    Column j of the Q factor is determined by Y's first j + 1 columns to
+    about u / r_j, where r_j = R_jj / ||y_j|| is the part of column j outside
+    the span of the columns before it.  Columns with r_j >= tau are
+    "resolved" and must agree within c / r_j; for the others (a singular or
+    nearly singular factor: a cold start, a rank-deficient gradient) any
+    orthonormal completion is a valid QR, so only orthonormality is checked.
+    Returns (resolved mask, per-column errors)."""
+    from oracle.qr import qr_positive
+    Q = np.asarray(Q, dtype=np.float64)
+    Y = np.asarray(Y, dtype=np.float64)
+    assert np.abs(Q.T @ Q - np.eye(Q.shape[1])).max() <= orth
+    Qr, R = qr_positive(Y)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.abs(np.diag(R)) / np.linalg.norm(Y, axis=0)
+    sel = r >= tau
+    err = np.linalg.norm(Q - Qr, axis=0)
+    bad = np.nonzero(sel & (err > c / np.where(sel, r, 1.0)))[0]
+    assert bad.size == 0, dict(columns=bad[:8].tolist(), err=err[bad[:8]].tolist(), r=r[bad[:8]].tolist())
+    return sel, err

@@ -117,17 +117,19 @@ def test_ns_rejects_overlap_and_nulls(lib):
 
 def test_soap_rejects_bad_arguments(lib):
     h = _ctx(lib)
-    cfg = _lib.SoapCfg(3e-3, 0.95, 0.95, 0.95, 1e-8, 0.0, 1, None, 0, 1e-5)
+    cfg = _lib.SoapCfg(3e-3, 0.95, 0.95, 0.95, 1e-8, 0.0, 1, None, 0, 0.0)
     good = _lib.SoapMat(8, 8, 16, 16, 16, 16, 16, 16, None, None)
     mats = (_lib.SoapMat * 1)(good)
     assert lib.soap_step(h, mats, 1, ctypes.byref(cfg), 0, None) == _lib.MO_ERR_INVALID_ARG
     half = _lib.SoapMat(8, 8, 16, 16, 16, 16, 16, None, None, None)
     mats = (_lib.SoapMat * 1)(half)
     assert lib.soap_step(h, mats, 1, ctypes.byref(cfg), 1, None) == _lib.MO_ERR_INVALID_ARG
-    bad_cfg = _lib.SoapCfg(3e-3, 1.0, 0.95, 0.95, 1e-8, 0.0, 1, None, 0, 1e-5)
+    bad_cfg = _lib.SoapCfg(3e-3, 1.0, 0.95, 0.95, 1e-8, 0.0, 1, None, 0, 0.0)
     mats = (_lib.SoapMat * 1)(good)
     assert lib.soap_step(h, mats, 1, ctypes.byref(bad_cfg), 1, None) == _lib.MO_ERR_INVALID_ARG
-    for damping in (0.0, -1e-5, 0.5, float("nan")):
+    # damping 0 is the pages' undamped power step (valid); negative, above
+    # 1e-2 or NaN is refused
+    for damping in (-1e-5, 0.5, float("nan")):
         bad_cfg = _lib.SoapCfg(3e-3, 0.95, 0.95, 0.95, 1e-8, 0.0, 1, None, 0, damping)
         assert lib.soap_step(h, mats, 1, ctypes.byref(bad_cfg), 1, None) == _lib.MO_ERR_INVALID_ARG
         assert b"damping" in lib.mo_last_error(h)
@@ -157,12 +159,12 @@ def test_soap_muon_rejects_bad_arguments(lib):
     def cfg(**kw):
         base = dict(lr=0.02, weight_decay=0.01, momentum=0.95, nesterov=1, beta2=0.95,
                     shampoo_beta=0.9, eps=1e-8, bias_correction=1, ns_steps=5, a=3.4445,
-                    b=-4.7750, c=2.0315, ns_eps=1e-7, adjust_lr=0, damping=1e-5,
+                    b=-4.7750, c=2.0315, ns_eps=1e-7, adjust_lr=0, damping=0.0,
                     nonfinite=None, skip_refresh=0)
         base.update(kw)
         return _lib.SoapMuonCfg(**base)
 
-    for bad in (dict(momentum=1.0), dict(adjust_lr=2), dict(ns_steps=0), dict(damping=0.0),
+    for bad in (dict(momentum=1.0), dict(adjust_lr=2), dict(ns_steps=0), dict(damping=-1e-5),
                 dict(beta2=1.0), dict(lr=float("nan"))):
         assert lib.soap_muon_step(h, mats, 1, ctypes.byref(cfg(**bad)), 1, None) == _lib.MO_ERR_INVALID_ARG, bad
         assert lib.mo_last_error(h).startswith(b"soap_muon_step")
@@ -177,4 +179,21 @@ def test_soap_muon_rejects_bad_arguments(lib):
     smats = (_lib.SoapMat * 1)(_lib.SoapMat(8, 8, 16, 16, 16, 16, 16, 16, None, None))
     assert lib.mo_soap_workspace_bytes(h, smats, 1, ctypes.byref(plain)) == 0
     assert size.value > plain.value          # P and the Newton-Schulz scratch on top
+    lib.mo_ctx_destroy(h)
+
+
+def test_strided_batches_validate(lib):
+    h = _ctx(lib)
+    cfg = _lib.NsCfg(5, 3.4445, -4.7750, 2.0315, 1e-7, None)
+    # a stride below rows * cols would overlap the matrices
+    assert lib.ns_orthogonalize_strided(h, 16, 100, 4096, 100, 10, 20, 3, ctypes.byref(cfg), None) == \
+        _lib.MO_ERR_INVALID_ARG
+    assert b"stride" in lib.mo_last_error(h)
+    # well formed, but no workspace attached: refused before any launch
+    assert lib.ns_orthogonalize_strided(h, 16, 200, 1 << 20, 200, 10, 20, 3, ctypes.byref(cfg), None) == \
+        _lib.MO_ERR_NO_WORKSPACE
+    mcfg = _lib.MuonCfg(0.02, 0.01, 0.95, 1, 0, 5, 3.4445, -4.7750, 2.0315, 1e-7, 0, None)
+    assert lib.muon_step_strided(h, 16, 16, 16, 10, 4, 4, 2, ctypes.byref(mcfg), None) == _lib.MO_ERR_INVALID_ARG
+    assert lib.muon_step_strided(h, 16, 1 << 20, 1 << 21, 16, 4, 4, 2, ctypes.byref(mcfg), None) == \
+        _lib.MO_ERR_NO_WORKSPACE
     lib.mo_ctx_destroy(h)

@@ -217,12 +217,18 @@ def test_soap_full_size_sampled(ctx):
         # the refresh with the emulation's bf16 factor-EMA operands
         Gb = rnd(S["G"])
         L_emu = 0.95 * S["L"] + 0.05 * (Gb @ Gb.T)
-        d = osoap.damping_of(L_emu, 1e-5)
-        Q_emu, _ = qr_positive((L_emu + d * np.eye(L_emu.shape[0])) @ S["QL"])
+        Y = L_emu @ S["QL"]
+        Q_emu, R_emu = qr_positive(Y)
         assert rel(out["L"], L_emu) <= 1e-4
         Q = out["QL"]
         idx = np.random.default_rng(i).choice(Q.shape[0], 256, replace=False)
         assert np.abs(Q[:, idx].T @ Q[:, idx] - np.eye(256)).max() <= 1e-4
+        # warm factor: every column of qr(L Q_old) resolved, agreement
+        # column by column within 5e-6 / r_j and over the whole basis
+        r = np.abs(np.diag(R_emu)) / np.linalg.norm(Y, axis=0)
+        assert r.min() >= 1e-4, r.min()
+        err = np.linalg.norm(Q - Q_emu, axis=0)
+        assert (err <= 5e-6 / r).all(), (err / (5e-6 / r)).max()
         assert rel(Q, Q_emu) <= 5e-3
         assert rel(out["W"] - S["W"], ref["dW"]) <= 2e-2
     del mats

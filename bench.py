@@ -523,9 +523,9 @@ def soap_workload(dev, sq=4096, wide=14336, n_sq=4, n_wide=4, rank=32, noise=1e-
     return mats, fill
 
 
-def soap_bench(ctx, dev, steps=3, warm=10):
+def soap_bench(ctx, dev, steps=3, warm=10, side=4096):
     import torch
-    mats, fill = soap_workload(dev)
+    mats, fill = soap_workload(dev, sq=side, wide=side * 14336 // 4096)
     fl, rot = 0.0, 0.0
     for d in mats:
         f, r = soap_flops(d["W"].shape[0], d["W"].shape[1], "L" in d, "R" in d)
@@ -560,7 +560,7 @@ def soap_bench(ctx, dev, steps=3, warm=10):
     k = {kk: round(v[0] / steps, 3) for kk, v in prof.items() if v[2]}
     rot_ms = prof["soap_rot"][0] / steps
     rot_exec = prof["soap_rot"][1] / steps
-    return {"workload": f"soap_step 4 x 4096^2 (two-sided) + 4 x 4096x14336 (left side only), steps "
+    return {"workload": f"soap_step 4 x {side}^2 (two-sided) + 4 x {side}x{side * 14336 // 4096} (left side only), steps "
                         f"{warm + 1}-{warm + steps} after {warm} warm steps; refresh qr(L Q), damping 0",
             "ms": round(ms, 3), "TFLOP/s": round(fl / (ms / 1e3) / 1e12, 1),
             "flops_per_step": fl, "matrices_per_s": round(len(mats) / (ms / 1e3), 1),
@@ -815,7 +815,7 @@ def run_soap_only(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     ctx = Context(local)
-    res = soap_bench(ctx, dev, steps=args.steps, warm=max(args.warmup, 1))
+    res = soap_bench(ctx, dev, steps=args.steps, warm=max(args.warmup, 1), side=args.soap_side)
     return {"metric": METRIC, "value": res["TFLOP/s"], "unit": UNIT, "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": {"workload": res["workload"]},
@@ -914,6 +914,9 @@ def main():
                          "gemm-vs-cublas: the NS products against cuBLAS at the sustained clock")
     ap.add_argument("--seconds", type=float, default=3.0, help="gemm-vs-cublas: timed seconds per phase")
     ap.add_argument("--once", action="store_true", help="gemm-vs-cublas: each product once, batch 3")
+    ap.add_argument("--soap-side", type=int, default=4096,
+                    help="soap: side of the square matrices and factors (4096 = the benchmark workload; "
+                         "1024 for small profiling cases)")
     ap.add_argument("--layers", type=int, default=32,
                     help="dense-GPT layers (32 = the benchmark workload; fewer for small profiling cases)")
     args = ap.parse_args()

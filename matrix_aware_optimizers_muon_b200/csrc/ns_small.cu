@@ -1,9 +1,10 @@
 // Fused Newton-Schulz (and Muon step) for small matrices: m' <= 128 and
 // n' <= 256 after orientation.  One persistent CTA walks over the matrices;
-// for each it keeps X (m' x n'), A = X X^T and P = b A + c A A in shared
-// memory (128-byte-swizzled K-major tiles, zero padded to 128 x 256 / 128 x
-// 128) and the fp32 products in tensor memory, so HBM sees only the inputs
-// and the outputs.  The arithmetic and rounding points are those of the
+// for each it keeps X (m' x n') and A = X X^T in shared memory (128-byte-
+// swizzled K-major tiles, zero padded to 128 x 256 / 128 x 128), with P =
+// b A + c A A written over A row by row once A A is in tensor memory, and
+// the fp32 products in tensor memory, so HBM sees only the inputs and the
+// outputs.  The arithmetic and rounding points are those of the
 // batched path: N = G + beta B (Muon) or the input, Nb = bf16(N),
 // inv = 1 / (||N||_F + eps) applied in fp32 inside iteration 0, every stored
 // iterate rounded to bf16.
@@ -25,11 +26,13 @@ namespace {
 constexpr int SM_THREADS = 160;
 constexpr int CHUNK = 128 * 128;                 // bytes of one 64-column chunk of 128 rows
 constexpr int A_BYTES = 2 * CHUNK;               // 128 x 128
-constexpr uint32_t TMEM_COLS = 256;
-constexpr int VU = 8;                            // float4 accesses in flight per thread
+constexpr int VU = 4;                            // float4 accesses in flight per thread
 
-// X holds npad / 64 chunks; with npad <= 128 two CTAs fit on one SM.
-constexpr int smem_bytes(int npad) { return (npad / 64) * CHUNK + 2 * A_BYTES + 1024 + 256; }
+// X holds npad / 64 chunks and A (then P) 2: with npad <= 128 three CTAs fit
+// on one SM (shared memory), with 128 tensor-memory columns each.
+constexpr int smem_bytes(int npad) { return (npad / 64) * CHUNK + A_BYTES + 1024 + 256; }
+// tensor-memory columns: the widest product (128 for A and A A, npad for P X)
+__host__ __device__ constexpr uint32_t tmem_cols(int npad) { return npad <= 128 ? 128u : 256u; }
 
 // byte offset of element (r, c) inside a swizzled chunked tile
 __device__ __forceinline__ uint32_t swz(int r, int c) {
@@ -78,16 +81,17 @@ __device__ __forceinline__ void load_unit(const uint8_t* tile, int r, int u, flo
   }
 }
 
-__global__ void __launch_bounds__(SM_THREADS, 2) ns_small_kernel(const SmallArgs a) {
+__global__ void __launch_bounds__(SM_THREADS, 3) ns_small_kernel(const SmallArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int np = a.tall ? a.rows : a.cols;      // oriented cols (<= 256)
   const int npad = (np + 63) & ~63;             // K of the Gram, N of the update
   const int xbytes = (npad >> 6) * CHUNK;
   uint8_t* X = smem;
-  uint8_t* A = smem + xbytes;
-  uint8_t* P = A + A_BYTES;
-  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(P + A_BYTES);
+  uint8_t* A = smem + xbytes;                   // A, then P over it
+  uint8_t* P = A;
+  const uint32_t TMEM_COLS = tmem_cols(npad);
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(A + A_BYTES);
   uint64_t* work_bar = mma_bar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(work_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -228,7 +232,8 @@ __global__ void __launch_bounds__(SM_THREADS, 2) ns_small_kernel(const SmallArgs
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(work_bar);
-        // ---- P = b A + c A A
+        // ---- P = b A + c A A, over A: A A has been read into tensor
+        // memory, and each thread reads and rewrites only its own row
         ok = mbar_wait(mma_bar, mma_phase, abort_flag, a.status, DEV_TIMEOUT_ACC_FULL);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         mma_phase ^= 1u;
@@ -410,9 +415,12 @@ cudaError_t launch_ns_small(const SmallArgs& a, int sm_count, cudaStream_t s) {
   const int np = a.tall ? a.rows : a.cols;
   const int npad = (np + 63) & ~63;
   const int smem = smem_bytes(npad);
-  // two CTAs per SM when both fit in shared memory (one's loads and stores
-  // then overlap the other's tensor-core phases)
-  const int per_sm = 2 * (smem + 1024) <= 228 * 1024 ? 2 : 1;
+  // as many CTAs per SM (up to three) as shared and tensor memory hold: one's
+  // loads, stores and epilogues then overlap the others' tensor-core phases
+  int per_sm = (228 * 1024) / (smem + 1024);
+  const int by_tmem = (int)(512 / tmem_cols(npad));
+  per_sm = per_sm < by_tmem ? per_sm : by_tmem;
+  per_sm = per_sm > 3 ? 3 : (per_sm < 1 ? 1 : per_sm);
   const int grid = a.count < per_sm * sm_count ? a.count : per_sm * sm_count;
   ProfScope prof(PK_SMALL, s, 0.0);
   return launch_pdl(ns_small_kernel, dim3(grid), dim3(SM_THREADS), (size_t)smem, s, false, a);

@@ -32,7 +32,7 @@ struct SmallArgs {
 void launch_upload_tables(void** dst, int n, const void* const* in, const void* const* mom,
                           const void* const* out, const void* const* flag, cudaStream_t s);
 
-// One persistent launch over all matrices (grid: up to two CTAs per SM).
+// One persistent launch over all matrices (grid: up to three CTAs per SM).
 cudaError_t launch_ns_small(const SmallArgs& a, int sm_count, cudaStream_t s);
 
 }  // namespace mo

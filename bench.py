@@ -822,6 +822,60 @@ def run_soap_only(args, world, rank, local):
             "soap": res}
 
 
+def run_moe_only(args, world, rank, local):
+    """The MoE Muon step alone (profiling and ncu runs): --moe-layers x
+    --moe-experts experts, three matrices each, steps timed with CUDA events
+    after the warm-up, then one step with the per-launch events on."""
+    import torch
+    from matrix_aware_optimizers_muon_b200 import Context
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ctx = Context(local)
+    Ws, Gs, Bs, shapes = moe_workload(dev, layers=args.moe_layers, experts=args.moe_experts)
+    ctx.reserve(0, shapes)
+    call = lambda: ctx.muon_step(Ws, Gs, Bs, reserve=False)
+    ms = time_steps(call, args.steps, max(args.warmup, 3))
+    ctx.profile(True)
+    ctx.profile_read()
+    call()
+    torch.cuda.synchronize()
+    prof = ctx.profile_read()
+    ctx.profile(False)
+    fl = sum(page_flops(m, n) for m, n in shapes)
+    gemm = ("gram", "poly", "update")
+    g_ms = sum(prof[k][0] for k in gemm)
+    g_fl = sum(prof[k][1] for k in gemm)
+    return {"metric": METRIC, "value": round(fl / (ms / 1e3) / 1e12, 1), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"muon_step MoE experts: {args.moe_layers} layers x {args.moe_experts} experts x "
+                                   f"(gate, up 768x2048; down 2048x768), {len(shapes)} matrices"},
+            "matrices_per_s": round(len(shapes) / (ms / 1e3), 1),
+            "kernels_ms": {k: round(v[0], 3) for k, v in prof.items() if v[2]},
+            "gemm_executed_TFLOP/s": {k: round(prof[k][1] / (prof[k][0] / 1e3) / 1e12, 1) for k in gemm if prof[k][0]},
+            "gemm_executed_TFLOP/s_all": round(g_fl / (g_ms / 1e3) / 1e12, 1) if g_ms else None}
+
+
+def run_heads_only(args, world, rank, local):
+    """Newton-Schulz on --heads matrices of 128 x 128 in one strided call
+    (profiling and ncu runs)."""
+    import torch
+    from matrix_aware_optimizers_muon_b200 import Context
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ctx = Context(local)
+    Ht = heads_gpu(args.heads, 128, dev)
+    Ho = torch.empty_like(Ht)
+    ctx.reserve(2, [(128, 128)] * args.heads)
+    call = lambda: ctx.ns_orthogonalize_batch(Ht, Ho, reserve=False)
+    ms = time_steps(call, args.steps, max(args.warmup, 3))
+    fl = args.heads * page_flops(128, 128)
+    return {"metric": METRIC, "value": round(fl / (ms / 1e3) / 1e12, 1), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"ns_orthogonalize_strided on {args.heads} matrices of 128 x 128"}}
+
+
 def gemm_vs_cublas(args, local):
     """The Newton-Schulz products of the dense-GPT 4096 x 14336 bucket (and a
     square 8192^3 product) through this library's GEMM and through cuBLAS
@@ -909,9 +963,13 @@ def main():
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--workload", choices=["muon", "soap", "gemm-vs-cublas"], default="muon",
+    ap.add_argument("--workload", choices=["muon", "soap", "moe", "heads", "gemm-vs-cublas"], default="muon",
                     help="muon: the dense-GPT Muon step (the benchmark line); soap: the SOAP step alone; "
+                         "moe: the MoE Muon step alone; "
                          "gemm-vs-cublas: the NS products against cuBLAS at the sustained clock")
+    ap.add_argument("--heads", type=int, default=4096, help="heads: matrices of 128 x 128")
+    ap.add_argument("--moe-layers", type=int, default=4, help="moe: layers (4 = the benchmark workload)")
+    ap.add_argument("--moe-experts", type=int, default=128, help="moe: experts per layer (128 = the benchmark)")
     ap.add_argument("--seconds", type=float, default=3.0, help="gemm-vs-cublas: timed seconds per phase")
     ap.add_argument("--once", action="store_true", help="gemm-vs-cublas: each product once, batch 3")
     ap.add_argument("--soap-side", type=int, default=4096,
@@ -925,6 +983,10 @@ def main():
         out = run_reference(args, world, rank)
     elif args.workload == "soap":
         out = run_soap_only(args, world, rank, local)
+    elif args.workload == "moe":
+        out = run_moe_only(args, world, rank, local)
+    elif args.workload == "heads":
+        out = run_heads_only(args, world, rank, local)
     elif args.workload == "gemm-vs-cublas":
         out = gemm_vs_cublas(args, local)
     else:

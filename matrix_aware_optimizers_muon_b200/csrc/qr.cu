@@ -263,9 +263,21 @@ __global__ void __launch_bounds__(256) qr_chol_kernel(const float* C, long long 
   __shared__ float mp;
   const int tid = threadIdx.x;
   const float* src = C + (size_t)b * stride + (long long)k0 * ld + k0;
-  for (int e = tid; e < CB * CB; e += blockDim.x) {
-    const int r = e >> 7, col = e & 127;
-    A[r * CB_LD + col] = src[(long long)r * ld + col];
+  // the 128 x 128 block as 4096 float4 loads, 16 per thread, all in flight
+  // before the first shared-memory store (rows of C are 16-byte aligned)
+  {
+    float4 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = tid + 256 * i, r = e >> 5, c4 = (e & 31) * 4;
+      v[i] = *reinterpret_cast<const float4*>(src + (long long)r * ld + c4);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = tid + 256 * i, r = e >> 5, c4 = (e & 31) * 4;
+      float* a = A + r * CB_LD + c4;
+      a[0] = v[i].x; a[1] = v[i].y; a[2] = v[i].z; a[3] = v[i].w;
+    }
   }
   if (tid == 0) {
     bad = 0;
@@ -284,9 +296,12 @@ __global__ void __launch_bounds__(256) qr_chol_kernel(const float* C, long long 
   if (tid == 0 && mp > 0.f) atomicMin(c.minpiv + b, __float_as_uint(mp));
   chol128_inverse(A, inv_diag, X, T);
   float* dst = Dinv + (size_t)b * CB * CB;
-  for (int e = tid; e < CB * CB; e += blockDim.x) {
-    const int r = e >> 7, col = e & 127;
-    dst[e] = col <= r ? X[r * CB_LD + col] : 0.f;
+#pragma unroll 4
+  for (int i = 0; i < 16; ++i) {
+    const int e = tid + 256 * i, r = e >> 5, c4 = (e & 31) * 4;
+    const float* x = X + r * CB_LD + c4;
+    reinterpret_cast<float4*>(dst)[e] = make_float4(c4 <= r ? x[0] : 0.f, c4 + 1 <= r ? x[1] : 0.f,
+                                                    c4 + 2 <= r ? x[2] : 0.f, c4 + 3 <= r ? x[3] : 0.f);
   }
 }
 
@@ -304,14 +319,35 @@ __global__ void __launch_bounds__(256) qr_panel_kernel(const PanelArgs a) {
   const int r0 = a.r0 + blockIdx.x * 64;
   const long long col0 = (long long)a.j * QR_B;
   const float* dinv = a.Dinv + (size_t)b * QR_B * QR_B;
-  for (int e = threadIdx.x; e < QR_B * QR_B; e += blockDim.x) {
-    const int cc = e >> 7, p = e & 127;
-    Dt[p * LDD + cc] = dinv[e];
-  }
   float* cy = a.CY + (size_t)b * a.mat_stride + col0;
-  for (int e = threadIdx.x; e < 64 * QR_B; e += blockDim.x) {
-    const int r = e >> 7, p = e & 127;
-    Rt[p * LDR + r] = (r0 + r < a.r1) ? cy[(long long)(r0 + r) * a.ld + p] : 0.f;
+  // Dinv (4096 float4) and the 64 x 128 rows (2048 float4): 24 loads per
+  // thread, all issued before the transposing shared-memory stores
+  {
+    float4 d[16], y[8];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) d[i] = reinterpret_cast<const float4*>(dinv)[threadIdx.x + 256 * i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = threadIdx.x + 256 * i, r = e >> 5, p4 = (e & 31) * 4;
+      y[i] = (r0 + r < a.r1) ? *reinterpret_cast<const float4*>(cy + (long long)(r0 + r) * a.ld + p4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = threadIdx.x + 256 * i, cc = e >> 5, p4 = (e & 31) * 4;     // Dinv[cc][p4 ..]
+      Dt[(p4 + 0) * LDD + cc] = d[i].x;
+      Dt[(p4 + 1) * LDD + cc] = d[i].y;
+      Dt[(p4 + 2) * LDD + cc] = d[i].z;
+      Dt[(p4 + 3) * LDD + cc] = d[i].w;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = threadIdx.x + 256 * i, r = e >> 5, p4 = (e & 31) * 4;
+      Rt[(p4 + 0) * LDR + r] = y[i].x;
+      Rt[(p4 + 1) * LDR + r] = y[i].y;
+      Rt[(p4 + 2) * LDR + r] = y[i].z;
+      Rt[(p4 + 3) * LDR + r] = y[i].w;
+    }
   }
   __syncthreads();
   const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
@@ -350,9 +386,25 @@ __global__ void __launch_bounds__(256) qr_panel_kernel(const PanelArgs a) {
   }
 }
 
-__global__ void qr_finish_kernel(const QrCtl c, const FlagTable f, int q) {
+__global__ void qr_finish_flags_kernel(const QrCtl c, const FlagTable f, int q) {
   const int b = threadIdx.x;
   if (b < q && !c.done[b] && f.f[b] != nullptr) *f.f[b] = 1;
+}
+
+struct Fallback {
+  const float* q[SOAP_MAXB];
+};
+
+// Row r of matrix b (one CTA per row): the previous basis, identity-padded.
+__global__ void qr_fallback_kernel(const QrCtl c, float* Y, long long ld, long long stride, int k, int kp,
+                                   const Fallback f) {
+  const int b = blockIdx.y;
+  if (c.done[b]) return;
+  const int r = blockIdx.x;
+  float* y = Y + (size_t)b * stride + (long long)r * ld;
+  const float* src = f.q[b] + (long long)r * k;
+  for (int col = threadIdx.x; col < kp; col += blockDim.x)
+    y[col] = (r < k && col < k) ? src[col] : (r == col ? 1.f : 0.f);
 }
 
 }  // namespace
@@ -429,9 +481,13 @@ void launch_qr_panel(const PanelArgs& a, cudaStream_t s) {
   qr_panel_kernel<<<grid, 256, smem, s>>>(a);
 }
 
-void launch_qr_finish(const QrCtl& c, const FlagTable& flags, int q, cudaStream_t s) {
+void launch_qr_finish(const QrCtl& c, const FlagTable& flags, int q, float* Y, long long ld,
+                      long long mat_stride, int k, int kp, const float* const* Qold, cudaStream_t s) {
   ProfScope prof(PK_SOAP_QR, s);
-  qr_finish_kernel<<<1, SOAP_MAXB, 0, s>>>(c, flags, q);
+  qr_finish_flags_kernel<<<1, SOAP_MAXB, 0, s>>>(c, flags, q);
+  Fallback f;
+  for (int b = 0; b < q && b < SOAP_MAXB; ++b) f.q[b] = Qold[b];
+  qr_fallback_kernel<<<dim3(kp, q), 256, 0, s>>>(c, Y, ld, mat_stride, k, kp, f);
 }
 
 }  // namespace mo

@@ -25,13 +25,15 @@
 //     the basis done: Y is Q and the matrix skips every later kernel;
 //   - the first attempt is plain, with a pivot floor of 1e-4 (of the unit
 //     diagonal): below it the factor of an ill-conditioned Gram would be
-//     inaccurate, so the attempt is abandoned for that matrix (Y kept) and
-//     the next pass is shifted;
+//     inaccurate, so the attempt is abandoned for that matrix and the next
+//     pass is shifted (the block columns already solved stay: Y times an
+//     upper-triangular matrix with a positive diagonal has Y's Q);
 //   - a shifted pass factors C + s I with s = 1e-5 ||C||_F * mult (shifted
 //     CholeskyQR: the result is still Y's Q, better conditioned); it is
 //     repeated while its smallest pivot stays below 10 s, and mult grows
 //     tenfold when even the shifted factorisation fails;
-//   - matrices not done after the last pass get their flag set.
+//   - matrices not done after the last pass get their flag set and keep
+//     their previous basis.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -140,7 +142,11 @@ struct PanelArgs {
 };
 void launch_qr_panel(const PanelArgs& a, cudaStream_t s);
 
-// After the last pass: flag[b] = 1 for every matrix whose basis is not done.
-void launch_qr_finish(const QrCtl& c, const FlagTable& flags, int q, cudaStream_t s);
+// After the last pass: flag[b] = 1 for every matrix whose basis is not done,
+// and its Y (kp x kp, row stride ld) reset to its previous basis Qold[b]
+// (k x k, padded with the identity), so that a failed refresh keeps the old
+// basis instead of a non-orthonormal iterate.
+void launch_qr_finish(const QrCtl& c, const FlagTable& flags, int q, float* Y, long long ld,
+                      long long mat_stride, int k, int kp, const float* const* Qold, cudaStream_t s);
 
 }  // namespace mo

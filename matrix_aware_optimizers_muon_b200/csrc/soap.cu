@@ -423,7 +423,11 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
       }
-      launch_qr_finish(ctl, flags, q, s);
+      {
+        const float* qold[SOAP_MAXB];
+        for (int j = 0; j < q; ++j) qold[j] = basis_of(j);
+        launch_qr_finish(ctl, flags, q, CY + kk, kp, ms, (int)k, (int)kp, qold, s);
+      }
       // the new bases: fp32 into the caller's Q, bf16 into the group buffers
       CopyOutArgs co;
       co.count = q; co.k = (int)k; co.Y = CY + kk; co.ld = kp; co.mat_stride = ms;

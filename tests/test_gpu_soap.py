@@ -285,9 +285,10 @@ def test_checkpoint_resume_bitwise(ctx):
 
 
 def test_nonfinite_gradient_flags_and_propagates(ctx):
-    """A NaN in one matrix's gradient: its factor, basis and weights become
-    non-finite and its flag is set (the refresh never reaches an orthonormal
-    basis); the other matrix of the same call is unaffected."""
+    """A NaN in one matrix's gradient: its factor and weights become
+    non-finite, its flag is set (the refresh never reaches an orthonormal
+    basis) and it keeps its previous bases; the other matrix of the same
+    call is unaffected."""
     import torch
     m = n = 128
     rng = wl.rng_of("soap-nan")
@@ -310,6 +311,8 @@ def test_nonfinite_gradient_flags_and_propagates(ctx):
     f = flags.cpu().numpy()
     assert f[0] == 1 and f[1] == 0, f
     assert not np.isfinite(_np(ds[0]["W"])).all()
+    np.testing.assert_array_equal(_np(ds[0]["QL"]), np.eye(m))
+    np.testing.assert_array_equal(_np(ds[0]["QR"]), np.eye(n))
     S, G = refs[1]
     emu = osoap.soap_step(S["W"], G, S["M"], S["V"], S["L"], S["QL"], S["R"], S["QR"], t=1,
                           precision="bf16", **HP)

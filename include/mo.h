@@ -95,7 +95,11 @@ MO_API mo_status mo_workspace_bytes(mo_ctx* ctx, int op, const int64_t* rows, co
  * buffer clears its header with a stream-ordered memset on `stream` and
  * copies the previous workspace's status word into it (a 4-byte device copy
  * on `stream`, which reads the old buffer: keep it alive until that copy has
- * run), so a timeout recorded before the switch is still reported. */
+ * run), so a timeout recorded before the switch is still reported.
+ * dev_ptr == NULL with bytes == 0 detaches the workspace: its status word is
+ * first read into the context (synchronising `stream`; skipped while
+ * `stream` is capturing) and reported by the next mo_device_status; call
+ * this before freeing a workspace that will not be replaced. */
 MO_API mo_status mo_set_workspace(mo_ctx* ctx, void* dev_ptr, size_t bytes, void* stream);
 
 /* Copy the device status word to *status (0 = no timeout recorded) and clear

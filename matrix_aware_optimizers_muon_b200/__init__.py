@@ -81,7 +81,7 @@ class Context:
         if st != 0:
             raise MoError(st, "mo_ctx_create failed")
         self.handle = h
-        self.workspace = None
+        self._workspace = None
         self.retired = []       # workspaces replaced during stream capture, kept alive
         self._batch_reserved = {}
 
@@ -95,6 +95,24 @@ class Context:
             self.close()
         except Exception:
             pass
+
+    # ------------------------------------------------------------ workspace
+    @property
+    def workspace(self):
+        """The attached workspace tensor (None when detached)."""
+        return self._workspace
+
+    @workspace.setter
+    def workspace(self, value):
+        """Only None may be assigned: it detaches the workspace in the library
+        (reading its status word first) and drops the tensor.  Use
+        attach_workspace() or reserve() to attach one."""
+        if value is not None:
+            raise ValueError("assign None to detach; use attach_workspace() or reserve() to attach")
+        if self._workspace is not None:
+            self._check(self.lib.mo_set_workspace(self.handle, None, 0, self._stream(None)))
+            self._workspace = None
+            self._batch_reserved.clear()
 
     # ------------------------------------------------------------ helpers
     def _stream(self, stream):
@@ -129,7 +147,7 @@ class Context:
         buf = torch.empty(int(nbytes), dtype=torch.uint8, device=f"cuda:{self.device}")
         self._check(self.lib.mo_set_workspace(self.handle, c_void_p(buf.data_ptr()), buf.numel(),
                                               self._stream(stream)))
-        old, self.workspace = self.workspace, buf
+        old, self._workspace = self._workspace, buf
         if old is not None:
             if torch.cuda.is_current_stream_capturing():
                 self.retired.append(old)

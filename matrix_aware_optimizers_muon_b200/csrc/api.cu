@@ -19,6 +19,7 @@ struct mo_ctx {
   int device = 0;
   char* ws = nullptr;
   size_t ws_bytes = 0;
+  int32_t detached_status = 0;   // status word of a workspace detached before it was read
   std::string err;
   bool profiling = false;
   mo::Profiler prof;
@@ -95,6 +96,26 @@ mo_status mo_workspace_bytes(mo_ctx* ctx, int op, const int64_t* rows, const int
 
 mo_status mo_set_workspace(mo_ctx* ctx, void* dev_ptr, size_t bytes, void* stream) {
   if (ctx == nullptr) return MO_ERR_INVALID_ARG;
+  if (dev_ptr == nullptr && bytes == 0) {
+    // detach: keep the status word in the context, then forget the buffer
+    if (ctx->ws == nullptr) return MO_OK;
+    mo::DeviceScope dev_scope;
+    mo_status st = enter(ctx, dev_scope);
+    if (st != MO_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &cap);
+    if (e == cudaSuccess && cap == cudaStreamCaptureStatusNone) {
+      int32_t v = 0;
+      e = cudaMemcpyAsync(&v, ctx->ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+      if (e == cudaSuccess) ctx->detached_status |= v;
+    }
+    ctx->ws = nullptr;
+    ctx->ws_bytes = 0;
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "mo_set_workspace (detach)");
+    return MO_OK;
+  }
   if (dev_ptr == nullptr || bytes < mo::WS_HEADER)
     return fail(ctx, MO_ERR_INVALID_ARG, "mo_set_workspace: null or too small (< 256 bytes)");
   if (reinterpret_cast<uintptr_t>(dev_ptr) % 256 != 0)
@@ -124,7 +145,7 @@ mo_status mo_device_status(mo_ctx* ctx, void* stream, int32_t* status) {
   // the attached workspace's word and the word of the fixed scratch array
   // that ns_orthogonalize_static uses on this device (once it has been set up)
   int32_t* words[2] = {reinterpret_cast<int32_t*>(ctx->ws), mo::static_status_word(ctx->device)};
-  if (words[0] == nullptr && words[1] == nullptr)
+  if (words[0] == nullptr && words[1] == nullptr && ctx->detached_status == 0)
     return fail(ctx, MO_ERR_NO_WORKSPACE, "mo_device_status: no workspace attached and no static call made");
   mo::DeviceScope dev_scope;
   mo_status st = enter(ctx, dev_scope);
@@ -138,7 +159,8 @@ mo_status mo_device_status(mo_ctx* ctx, void* stream, int32_t* status) {
   for (int i = 0; i < 2 && e == cudaSuccess; ++i)
     if (words[i]) e = cudaMemsetAsync(words[i], 0, sizeof(int32_t), s);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "mo_device_status");
-  const int32_t v = got[0] | got[1];
+  const int32_t v = got[0] | got[1] | ctx->detached_status;
+  ctx->detached_status = 0;
   *status = v;
   if (v != 0) return fail(ctx, MO_ERR_DEVICE, "device status " + std::to_string(v) + ": a kernel wait timed out");
   return MO_OK;

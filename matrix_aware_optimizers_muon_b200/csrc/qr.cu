@@ -80,6 +80,18 @@ __device__ __forceinline__ void store_planes_h8(__half* d, long long plane_strid
   *reinterpret_cast<uint4*>(d + plane_stride) = pack_half8(r);
 }
 
+// A uniform value in [-1, 1) from a 32-bit integer hash (the finaliser of
+// MurmurHash3, Appleby) of the element's coordinates and a seed.
+__device__ __forceinline__ float hash_uniform(unsigned b, unsigned r, unsigned c, unsigned seed) {
+  unsigned h = (r * 0x9E3779B1u) ^ (c * 0x85EBCA77u) ^ (b * 0xC2B2AE3Du) ^ (seed * 0x27D4EB2Fu);
+  h ^= h >> 16;
+  h *= 0x85EBCA6Bu;
+  h ^= h >> 13;
+  h *= 0xC2B2AE35u;
+  h ^= h >> 16;
+  return (float)(h >> 8) * (2.0f / 16777216.0f) - 1.0f;
+}
+
 __global__ void split16_kernel(const Split16Args a) {
   const int b = blockIdx.z;
   if (a.skip && a.skip[b]) return;
@@ -98,17 +110,23 @@ __global__ void split16_kernel(const Split16Args a) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) x[i] = (rv && c0 + i < a.cols_valid) ? src[c0 + i] : 0.f;
   }
+  const bool noisy = a.noise_on && a.noise_on[b];
+  const float namp = noisy ? a.noise_amp * rsqrtf((float)a.cols_pad) : 0.f;
+  bool pad[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int c = c0 + i;
+    pad[i] = false;
     if (rv && c < a.cols_valid) {
       if (a.diag_add && r == c) x[i] += a.diag_add[b];
       if (a.col_scale) {
         const float s = a.col_scale[(size_t)b * a.cols_pad + c];
         x[i] = s == 0.f ? (r == c ? 1.f : 0.f) : x[i] * s;     // a zero column becomes e_c
       }
+      if (noisy) x[i] = fmaf(namp, hash_uniform(b, r, c, a.noise_seed), x[i]);
     } else {
-      x[i] = (a.pad_identity && r == c) ? 1.f : 0.f;
+      pad[i] = a.pad_identity && r == c;
+      x[i] = pad[i] ? 1.f : 0.f;
     }
   }
   if (a.write_back) {
@@ -117,8 +135,9 @@ __global__ void split16_kernel(const Split16Args a) {
     reinterpret_cast<float4*>(w)[1] = make_float4(x[4], x[5], x[6], x[7]);
   }
   const float sc = a.mscale ? a.mscale[b] : a.cscale;
+  const float pad_val = fminf(sc, 16384.f);      // a positive diagonal that fits fp16
 #pragma unroll
-  for (int i = 0; i < 8; ++i) x[i] *= sc;
+  for (int i = 0; i < 8; ++i) x[i] = pad[i] ? pad_val : x[i] * sc;
   store_planes_h8(a.dst + (size_t)b * a.mat_stride + (long long)r * a.ldd + c0, a.plane_stride, x);
 }
 

@@ -28,6 +28,12 @@
 //     inaccurate, so the attempt is abandoned for that matrix and the next
 //     pass is shifted (the block columns already solved stay: Y times an
 //     upper-triangular matrix with a positive diagonal has Y's Q);
+//   - CholeskyQR only rescales and combines Y's columns, so columns that are
+//     exactly dependent (a rank-deficient factor) would stay dependent: the
+//     pass after a failed attempt perturbs the normalised columns by a
+//     seeded pseudo-random 1e-6 of their norm (the precision of the fp16
+//     planes), which a Householder QR's completion from rounding residue
+//     stands in for;
 //   - a shifted pass factors C + s I with s = 1e-5 ||C||_F * mult (shifted
 //     CholeskyQR: the result is still Y's Q, better conditioned); it is
 //     repeated while its smallest pivot stays below 10 s, and mult grows
@@ -48,6 +54,7 @@ constexpr int QR_CHECK_BLOCKS = 64;    // partial sums per matrix for the Gram c
 constexpr float QR_TAU_DONE = 5e-5f;
 constexpr float QR_PLAIN_FLOOR = 1e-4f;
 constexpr float QR_SHIFT_REL = 1e-5f;
+constexpr float QR_NOISE = 1e-6f;              // relative perturbation after a failed attempt
 constexpr float QR_PLANE_SCALE = 4096.f;       // 2^12: planes of L and Q (|L|, |Q| <= 16)
 constexpr float QR_Y_SCALE = 16384.f;          // 2^14: planes of the normalised Y and of Q_old (|x| <= 1)
 
@@ -107,7 +114,16 @@ struct Split16Args {
   long long ldd, mat_stride, plane_stride;
   int pad_identity = 0;
   const int* skip = nullptr;
+  // optional: matrices with noise_on[b] != 0 get, after the column scale, a
+  // pseudo-random perturbation of noise_amp / sqrt(cols_pad) per entry
+  // (uniform in [-1, 1), a hash of b, r, c and noise_seed)
+  const int* noise_on = nullptr;
+  float noise_amp = 0.f;
+  unsigned noise_seed = 0u;
 };
+// The padded diagonal (pad_identity) is written as min(scale, 2^14) in the
+// planes, whatever the scale, so that it never overflows fp16; write_back
+// receives 1 there.
 void launch_split16(const Split16Args& a, cudaStream_t s);
 
 // inv_d[b][c] = 1 / ||Y[b][:, c]|| (0 for a zero column, NaN for an

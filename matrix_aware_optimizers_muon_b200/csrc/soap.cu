@@ -382,6 +382,9 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
         sy.write_back = CY + kk; sy.ldw = kp; sy.wb_stride = ms;
         sy.dst = LQ + kk; sy.ldd = kp; sy.mat_stride = ms; sy.plane_stride = pst;
         sy.skip = ctl.done;
+        sy.noise_on = ctl.fail;                  // set by a failed attempt of the previous pass
+        sy.noise_amp = QR_NOISE;
+        sy.noise_seed = (unsigned)pass;
         launch_split16(sy, s);
         {
           GemmOp g;

@@ -197,3 +197,10 @@ def test_strided_batches_validate(lib):
     assert lib.muon_step_strided(h, 16, 1 << 20, 1 << 21, 16, 4, 4, 2, ctypes.byref(mcfg), None) == \
         _lib.MO_ERR_NO_WORKSPACE
     lib.mo_ctx_destroy(h)
+
+
+def test_detach_without_workspace_is_a_no_op(lib):
+    h = _ctx(lib)
+    assert lib.mo_set_workspace(h, None, 0, None) == 0
+    assert lib.mo_set_workspace(h, None, 64, None) == _lib.MO_ERR_INVALID_ARG
+    lib.mo_ctx_destroy(h)

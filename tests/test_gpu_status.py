@@ -23,3 +23,20 @@ def test_status_word_carried_to_new_workspace():
     assert ctx.workspace.data_ptr() != old.data_ptr()
     assert ctx.device_status() == 7
     assert ctx.device_status() == 0                  # cleared by the read
+
+
+def test_status_word_kept_when_workspace_detached():
+    """Dropping the workspace (ctx.workspace = None) detaches it in the
+    library after reading its status word, which the next read reports."""
+    require_gpu()
+    import torch
+    from matrix_aware_optimizers_muon_b200 import Context, build
+    build.build()
+    ctx = Context(0)
+    ctx.attach_workspace(1 << 20)
+    ctx.workspace[:4].view(torch.int32).fill_(5)
+    ctx.workspace = None
+    torch.cuda.empty_cache()                         # the buffer may be unmapped now
+    assert ctx.device_status() == 5
+    ctx.attach_workspace(1 << 20)                    # a fresh buffer after the detach: no copy from the old one
+    assert ctx.device_status() == 0

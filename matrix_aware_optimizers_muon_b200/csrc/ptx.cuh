@@ -13,6 +13,15 @@
 #define MO_WAIT_LIMIT_NS 2000000000ull   // 2 s of wall time per wait
 #endif
 
+// Suspend-time hint of a waiting thread's mbarrier test, in nanoseconds: the
+// thread may sleep up to this long unless the phase completes first, so a
+// long wait (an epilogue warp waiting for its next accumulator, the TMA
+// producer for a free stage) issues a few tests instead of spinning.
+// 0 = no hint (the hardware's own default limit).
+#ifndef MO_WAIT_HINT_NS
+#define MO_WAIT_HINT_NS 20000u
+#endif
+
 namespace mo {
 
 // device status codes written by kernels that give up a wait
@@ -56,6 +65,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
+#if MO_WAIT_HINT_NS > 0
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"((uint32_t)MO_WAIT_HINT_NS)
+      : "memory");
+#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -63,6 +81,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
+#endif
   return ok != 0;
 }
 

@@ -53,31 +53,40 @@ def ns_gate(N, O_gpu, O_ref, O_emu, *, tau=1e-2, sub_tol=2e-2, band=(0.6, 1.3), 
     return out
 
 
-def basis_gate(Q, Y, *, tau=1e-3, c0=5e-4, c1=2e-5, orth=1e-4):
-    """A refreshed basis Q (GPU) against the positive-diagonal QR of Y = F Q_old
-    (fp64 oracle).
+def basis_gate(Q, F, Q_old, *, tau=1e-3, c_kappa=5e-7, c_r=2e-5, c0=1e-5, orth=1e-4):
+    """A refreshed basis Q (GPU) against the positive-diagonal QR of the power
+    product Y = F Q_old (fp64 oracle).
 
-    Column j of the Q factor is determined by Y's first j + 1 columns; how
-    well depends on r_j = R_jj / ||y_j||, the part of column j outside the
-    span of the columns before it.  fp32-level arithmetic (the power product
-    F Q_old on a factor stored in fp32, then the QR) gives errors of about
-    3e-5 on well-separated columns, growing like 1 / r_j.  Columns with
-    r_j >= tau are "resolved" and must agree within c0 + c1 / r_j; for the
-    others (a singular or nearly singular factor: a cold start, a
-    rank-deficient gradient) any orthonormal completion is a valid QR, so
-    only orthonormality is checked.  Returns (resolved mask, per-column
-    errors)."""
+    Two things limit how well fp32-level arithmetic determines column j:
+      - the power product: y_j = F q_j is computed with an error of about u
+        ||F|| ||q_j||, i.e. a relative error u kappa_j with kappa_j =
+        ||F||_2 / ||y_j|| (columns in F's small-eigenvalue directions cancel
+        against the large ones);
+      - the QR: column j of Q depends on y_j's part outside the span of the
+        columns before it, r_j = R_jj / ||y_j||, to about u / r_j.
+    Columns with r_j >= tau are "resolved" and must agree within
+    c_kappa kappa_j + c_r / r_j + c0; for the others (a singular or nearly
+    singular factor: a cold start, a rank-deficient gradient) any
+    orthonormal completion is a valid QR, so only orthonormality is checked.
+    Returns (resolved mask, per-column errors)."""
+    from scipy.linalg import eigh
     from oracle.qr import qr_positive
     Q = np.asarray(Q, dtype=np.float64)
-    Y = np.asarray(Y, dtype=np.float64)
+    F = np.asarray(F, dtype=np.float64)
+    Y = F @ np.asarray(Q_old, dtype=np.float64)
     dev = float(np.abs(Q.T @ Q - np.eye(Q.shape[1])).max())
     assert dev <= orth, dict(orthonormality=dev)
     Qr, R = qr_positive(Y)
+    k = F.shape[0]
+    norm_f = float(np.abs(eigh((F + F.T) / 2, eigvals_only=True, subset_by_index=[k - 1, k - 1])[0]))
     with np.errstate(divide="ignore", invalid="ignore"):
-        r = np.abs(np.diag(R)) / np.linalg.norm(Y, axis=0)
+        ny = np.linalg.norm(Y, axis=0)
+        r = np.abs(np.diag(R)) / ny
+        kappa = norm_f / ny
     sel = r >= tau
     err = np.linalg.norm(Q - Qr, axis=0)
-    bound = c0 + c1 / np.where(sel, r, 1.0)
+    bound = c_kappa * np.where(sel, kappa, 0.0) + c_r / np.where(sel, r, 1.0) + c0
     bad = np.nonzero(sel & (err > bound))[0]
-    assert bad.size == 0, dict(columns=bad[:8].tolist(), err=err[bad[:8]].tolist(), r=r[bad[:8]].tolist())
+    assert bad.size == 0, dict(columns=bad[:8].tolist(), err=err[bad[:8]].tolist(), r=r[bad[:8]].tolist(),
+                               kappa=kappa[bad[:8]].tolist())
     return sel, err

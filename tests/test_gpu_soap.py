@@ -68,7 +68,7 @@ def check_step(ctx, m, n, left, right, steps=10, tag="soap"):
         assert res[fac] <= 1e-4, res                               # bf16-operand EMA, fp32 state
         Q = out[q]
         res[q + "_orth"] = float(np.abs(Q.T @ Q - np.eye(Q.shape[0])).max())
-        sel, _ = basis_gate(Q, emu[fac] @ S[q].astype(np.float64))  # qr(L Q_old), column by column
+        sel, _ = basis_gate(Q, emu[fac], S[q])  # qr(L Q_old), column by column
         assert sel.all(), res                                      # warm factors: every column resolved
         res[q] = rel(Q, emu[q])
         assert res[q] <= 5e-3, res                                 # fp32-accurate refresh
@@ -185,24 +185,25 @@ def test_cold_start_square_two_sided(ctx):
         resolved = {}
         for fac, q in (("L", "QL"), ("R", "QR")):
             Q = out[q]
-            resolved[q], _ = basis_gate(Q, emu[fac] @ S[q].astype(np.float64))
+            resolved[q], _ = basis_gate(Q, emu[fac], S[q])
             if t > 1:
                 assert resolved[q].all(), (t, q)
                 assert rel(Q, emu[q]) <= 5e-3, (t, q, rel(Q, emu[q]))
         dW = out["W"] - S["W"]
         if t == 1:
-            # Dbar = M' / |G'| is sign-like at step 1: where G' is at rounding
-            # level (M' and G' are rotated separately) its entries carry no
-            # information and differ between any two roundings.  So Dbar,
-            # recovered from dW with the GPU's own bases, is compared on the
-            # entries |G'| >= 1e-4 max|G'| whose row and column basis vectors
-            # are resolved (fp64 and the emulation agree there to 1.5e-4),
-            # and the update's size to 1 %.
+            # Dbar = M' / |G'| = sign(G') (to eps) at step 1, so what the
+            # update carries is the sign pattern of G' in the new bases.  Where
+            # G' is small next to the bases' uncertainty its sign is not
+            # determined, so Dbar, recovered from dW with the GPU's own bases,
+            # is compared by sign on the entries whose row and column basis
+            # vectors are resolved and |G'| >= 1e-3 max|G'|; and the update's
+            # size to 1 %.
             Dg = out["QL"].T @ (-dW / HP["lr"]) @ out["QR"]
-            mask = np.abs(emu["Gr"]) >= 1e-4 * np.abs(emu["Gr"]).max()
+            mask = np.abs(emu["Gr"]) >= 1e-3 * np.abs(emu["Gr"]).max()
             mask &= resolved["QL"][:, None] & resolved["QR"][None, :]
-            assert mask.mean() > 0.5
-            assert rel(Dg[mask], emu["Dbar"][mask]) <= 1e-2, rel(Dg[mask], emu["Dbar"][mask])
+            assert mask.sum() >= 1000, mask.sum()
+            agree = np.mean(np.sign(Dg[mask]) == np.sign(emu["Dbar"][mask]))
+            assert agree >= 0.99, agree
             ratio = np.linalg.norm(dW) / (HP["lr"] * np.sqrt(m * n))
             ratio_emu = np.linalg.norm(emu["dW"]) / (HP["lr"] * np.sqrt(m * n))
             assert abs(ratio - ratio_emu) <= 1e-2, (ratio, ratio_emu)
@@ -243,7 +244,7 @@ def test_rank_one_and_zero_gradients(ctx):
         emu = osoap.soap_step(S["W"], G, S["M"], S["V"], S["L"], S["QL"], S["R"], S["QR"], t=1,
                               precision="bf16", **HP)
         for fac, q in (("L", "QL"), ("R", "QR")):
-            basis_gate(out[q], emu[fac] @ S[q].astype(np.float64))
+            basis_gate(out[q], emu[fac], S[q])
         if not G.any():
             np.testing.assert_array_equal(out["QL"], np.eye(m))  # qr(0) = I
             np.testing.assert_array_equal(out["QR"], np.eye(n))
@@ -318,5 +319,5 @@ def test_nonfinite_gradient_flags_and_propagates(ctx):
                           precision="bf16", **HP)
     out = {k: _np(v) for k, v in ds[1].items() if k != "G"}
     for fac, q in (("L", "QL"), ("R", "QR")):
-        basis_gate(out[q], emu[fac] @ S[q].astype(np.float64))
+        basis_gate(out[q], emu[fac], S[q])
     assert np.isfinite(out["W"]).all()

@@ -67,7 +67,7 @@ def check(S, G, t, out, **kw):
         res[fac] = rel(out[fac], emu[fac])
         assert res[fac] <= 1e-4, res
         Q = out[q]
-        sel, _ = basis_gate(Q, emu[fac] @ S[q].astype(np.float64))   # qr(L Q_old), column by column
+        sel, _ = basis_gate(Q, emu[fac], S[q])   # qr(L Q_old), column by column
         if sel.all():
             res[q] = rel(Q, emu[q])
             assert res[q] <= 5e-3, res

@@ -95,9 +95,9 @@ int choose_band(int bm, int tiles_m, long long M, long long N, long long kseg, i
   return banded * 1.5 < plain ? g : tiles_m;
 }
 
-template <int BN, int A_MN, int B_MN, bool PAIR = false>
+template <int BN, int A_MN, int B_MN, bool PAIR = false, bool EPI2 = false>
 cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
-  using Cfg = GemmCfg<BN, PAIR>;
+  using Cfg = GemmCfg<BN, PAIR, EPI2>;
   constexpr int BM_T = PAIR ? 2 * GEMM_BM : GEMM_BM;
   CUtensorMap ta, tb, tc;
   std::memset(&tc, 0, sizeof(tc));
@@ -153,7 +153,7 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
     p.c_tma = 1;
   }
 
-  auto kern = gemm_bf16_kernel<BN, A_MN, B_MN, PAIR>;
+  auto kern = gemm_bf16_kernel<BN, A_MN, B_MN, PAIR, EPI2>;
   cudaError_t ea = ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES);
   if (ea != cudaSuccess) return ea;
   // tiles enumerated per matrix: all, or those touching the upper triangle
@@ -175,7 +175,7 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   // executed tensor-core flops: computed tiles x 128 x BN x padded K x 2
   const double flops = 2.0 * tiles * p.batch * BM_T * BN * (double)round_up(p.K, GEMM_BK);
   ProfScope prof(op.kind, stream, flops);
-  return launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), Cfg::SMEM_BYTES, stream, PAIR, ta, tb, tc, p);
+  return launch_pdl(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, stream, PAIR, ta, tb, tc, p);
 }
 
 }  // namespace
@@ -237,7 +237,11 @@ cudaError_t launch_gemm(const GemmOp& op, int* status, cudaStream_t stream) {
       default: return launch_t<256, 1, 1, true>(op, status, stream);
     }
   }
-  const int sel = (narrow ? 4 : 0) | (op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0);
+  // two sets of epilogue warps when K is short: a tile's main loop (K / 64
+  // steps) is then no longer than one set's epilogue, which would otherwise
+  // leave the tensor pipe idle between tiles
+  const bool epi2 = op.K <= 2048;
+  const int sel = (epi2 ? 8 : 0) | (narrow ? 4 : 0) | (op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0);
   switch (sel) {
     case 0: return launch_t<256, 0, 0>(op, status, stream);
     case 1: return launch_t<256, 0, 1>(op, status, stream);
@@ -246,7 +250,15 @@ cudaError_t launch_gemm(const GemmOp& op, int* status, cudaStream_t stream) {
     case 4: return launch_t<128, 0, 0>(op, status, stream);
     case 5: return launch_t<128, 0, 1>(op, status, stream);
     case 6: return launch_t<128, 1, 0>(op, status, stream);
-    default: return launch_t<128, 1, 1>(op, status, stream);
+    case 7: return launch_t<128, 1, 1>(op, status, stream);
+    case 8: return launch_t<256, 0, 0, false, true>(op, status, stream);
+    case 9: return launch_t<256, 0, 1, false, true>(op, status, stream);
+    case 10: return launch_t<256, 1, 0, false, true>(op, status, stream);
+    case 11: return launch_t<256, 1, 1, false, true>(op, status, stream);
+    case 12: return launch_t<128, 0, 0, false, true>(op, status, stream);
+    case 13: return launch_t<128, 0, 1, false, true>(op, status, stream);
+    case 14: return launch_t<128, 1, 0, false, true>(op, status, stream);
+    default: return launch_t<128, 1, 1, false, true>(op, status, stream);
   }
 }
 

@@ -86,21 +86,28 @@ enum { EPI_AXPBY = 0, EPI_ADAM = 1, EPI_APPLY = 2 };
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;
-constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_THREADS = 192;        // producer, MMA issuer, 4 epilogue warps
+constexpr int GEMM_THREADS_EPI2 = 320;   // the same with two sets of 4 epilogue warps
 
 // PAIR: a cluster of two CTAs computes a 256 x BN tile with cta_group::2
 // MMAs; each CTA stages its 128 rows of A and BN/2 rows (columns of the
 // product) of B, so a stage is 32 KB instead of 48 KB per SM.
-template <int BN, bool PAIR = false>
+// EPI2: two sets of four epilogue warps, set s draining accumulator s (the
+// MMA issuer alternates the two accumulators tile by tile), for products
+// with a short K whose main loop per tile is not longer than one set's
+// epilogue; their staging takes one TMA stage fewer.
+template <int BN, bool PAIR = false, bool EPI2 = false>
 struct GemmCfg {
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
   static constexpr int BN_LOCAL = PAIR ? BN / 2 : BN;
   static constexpr int B_BYTES = BN_LOCAL * GEMM_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = PAIR ? 6 : (BN == 256 ? 4 : 6);
+  static constexpr int STAGES = PAIR ? 6 : (BN == 256 ? (EPI2 ? 3 : 4) : (EPI2 ? 4 : 6));
   static constexpr int TMEM_COLS = 2 * BN;          // two fp32 accumulators
   static constexpr int BAR_BYTES = 1024;            // mbarriers; keeps the epilogue stage 1 KB aligned
-  static constexpr int EPI_BYTES = 4 * 8192;        // per epilogue warp: output block (or C), its transpose
+  static constexpr int EPI_WARPS = EPI2 ? 8 : 4;
+  static constexpr int EPI_BYTES = EPI_WARPS * 8192;  // per epilogue warp: output block (or C), its transpose
+  static constexpr int THREADS = EPI2 ? GEMM_THREADS_EPI2 : GEMM_THREADS;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + EPI_BYTES + 1024;
 };
 
@@ -461,11 +468,12 @@ __device__ __forceinline__ void stage_store32_f32_diag(uint8_t* stg, int lane, c
   }
 }
 
-template <int BN, int A_MN, int B_MN, bool PAIR = false>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+template <int BN, int A_MN, int B_MN, bool PAIR = false, bool EPI2 = false>
+__global__ void __launch_bounds__(GemmCfg<BN, PAIR, EPI2>::THREADS, 1) __maxnreg__(EPI2 ? 200 : 255)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
-  using Cfg = GemmCfg<BN, PAIR>;
+  static_assert(!(PAIR && EPI2), "CTA pairs run one set of epilogue warps");
+  using Cfg = GemmCfg<BN, PAIR, EPI2>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int BM_T = PAIR ? 2 * GEMM_BM : GEMM_BM;     // rows per tile
   constexpr int BN_L = Cfg::BN_LOCAL;                     // B rows staged by this CTA
@@ -479,8 +487,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint64_t* cbar = drain + 1;                 // [4 warps][2]: C blocks read by TMA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 8);
+  uint64_t* cbar = drain + 1;                 // [epilogue warps][2]: C blocks read by TMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 2 * Cfg::EPI_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* consumed = abort_flag + 1;
 
@@ -501,7 +509,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(&acc_empty[a], PAIR ? 256 : 128);   // the epilogue threads of every CTA of the tile
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&cbar[i], 1);
+    for (int i = 0; i < 2 * Cfg::EPI_WARPS; ++i) mbar_init(&cbar[i], 1);
     *abort_flag = 0;
     *consumed = 0;
     fence_barrier_init();
@@ -642,13 +650,15 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int ew = warp - 2;                // epilogue warp index
+    const int eset = ew >> 2;               // EPI2: the accumulator this warp's set drains
     const int row_in_tile = q * 32 + lane;
-    uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES + q * 8192;
+    uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES + ew * 8192;
     uint8_t* stc = stg + 4096;              // staged 32 x 32 bf16 block of C
     // two 2 KB buffers (at stg + 4096 and + 6144, 1 KB aligned) for C blocks
     // that TMA writes in the 64-byte-swizzled layout stg_off() reads
     uint8_t* cbuf0 = stg + 4096;           // buffer bi at cbuf0 + 2048 bi
-    uint64_t* cb = cbar + 2 * q;
+    uint64_t* cb = cbar + 2 * ew;
     uint32_t cph = 0u;                      // bit bi: phase of buffer bi
     uint32_t cpend = 0u;                    // bit bi: a copy into buffer bi is in flight
     const bool plain_bf16 = !p.d_f32 && !p.d_split;
@@ -656,14 +666,17 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const bool has_c = p.C != nullptr || p.c_tab != nullptr;
     const bool adam = p.epi == EPI_ADAM;
     const bool apply = p.epi == EPI_APPLY;
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    int ntile = 0;                          // tiles of this CTA so far: accumulator ntile % 2
     // a pair's epilogue threads release the accumulator on the even CTA's barrier
     const uint32_t acc_empty_cl0 = PAIR ? mapa_shared(&acc_empty[0], 0) : 0u;
     const uint32_t acc_empty_cl1 = PAIR ? mapa_shared(&acc_empty[1], 0) : 0u;
     for (int t = unit; t < total; t += units) {
       int b, tm, tn;
       if (!gemm_decode(p, BN, t, b, tm, tn)) continue;
+      const int acc = ntile & 1;
+      const uint32_t acc_phase = (uint32_t)(ntile >> 1) & 1u;
+      ++ntile;
+      if (EPI2 && acc != eset) continue;    // the other set's tile
       const int r = tm * BM_T + (int)rank * GEMM_BM + row_in_tile;
       const bool row_ok = r < p.M;
       // this matrix's operands, resolved once per tile
@@ -933,8 +946,6 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       tc_fence_before();
       if constexpr (PAIR) mbar_arrive_cluster(acc ? acc_empty_cl1 : acc_empty_cl0);
       else mbar_arrive(&acc_empty[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
     }
     // C blocks requested for a tile that was abandoned must land before exit
     if (lane == 0)

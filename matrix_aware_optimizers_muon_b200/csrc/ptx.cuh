@@ -19,7 +19,7 @@
 // producer for a free stage) issues a few tests instead of spinning.
 // 0 = no hint (the hardware's own default limit).
 #ifndef MO_WAIT_HINT_NS
-#define MO_WAIT_HINT_NS 20000u
+#define MO_WAIT_HINT_NS 0u
 #endif
 
 namespace mo {

@@ -314,19 +314,23 @@ __global__ void __launch_bounds__(256) qr_chol_kernel(const float* C, long long 
   }
   if (tid == 0 && mp > 0.f) atomicMin(c.minpiv + b, __float_as_uint(mp));
   chol128_inverse(A, inv_diag, X, T);
+  // the inverse transposed: DinvT[p][c] = Dinv[c][p] (nonzero for c >= p), so
+  // that the panel kernel stages it with straight float4 copies
   float* dst = Dinv + (size_t)b * CB * CB;
 #pragma unroll 4
   for (int i = 0; i < 16; ++i) {
-    const int e = tid + 256 * i, r = e >> 5, c4 = (e & 31) * 4;
-    const float* x = X + r * CB_LD + c4;
-    reinterpret_cast<float4*>(dst)[e] = make_float4(c4 <= r ? x[0] : 0.f, c4 + 1 <= r ? x[1] : 0.f,
-                                                    c4 + 2 <= r ? x[2] : 0.f, c4 + 3 <= r ? x[3] : 0.f);
+    const int e = tid + 256 * i, pr = e >> 5, c4 = (e & 31) * 4;
+    const float* x = X + c4 * CB_LD + pr;
+    reinterpret_cast<float4*>(dst)[e] =
+        make_float4(c4 >= pr ? x[0] : 0.f, c4 + 1 >= pr ? x[CB_LD] : 0.f, c4 + 2 >= pr ? x[2 * CB_LD] : 0.f,
+                    c4 + 3 >= pr ? x[3 * CB_LD] : 0.f);
   }
 }
 
 // out = in * Dinv^T for 64 rows x 128 columns per CTA (256 threads):
 // thread (ty, tx) computes rows 4 ty .. +3 and columns 8 tx .. +7 from
-// transposed shared copies of the rows and of Dinv (lower: p <= c).
+// transposed shared copies of the rows and of Dinv (Dinv lower: p <= c;
+// its global copy is stored transposed).
 __global__ void __launch_bounds__(256) qr_panel_kernel(const PanelArgs a) {
   const int b = blockIdx.y;
   if (a.skip[b]) return;
@@ -339,29 +343,29 @@ __global__ void __launch_bounds__(256) qr_panel_kernel(const PanelArgs a) {
   const long long col0 = (long long)a.j * QR_B;
   const float* dinv = a.Dinv + (size_t)b * QR_B * QR_B;
   float* cy = a.CY + (size_t)b * a.mat_stride + col0;
-  // Dinv (4096 float4) and the 64 x 128 rows (2048 float4): 24 loads per
-  // thread, all issued before the transposing shared-memory stores
+  // DinvT (4096 float4, stored transposed by the diagonal-block kernel) and
+  // the 64 x 128 rows (2048 float4): 24 loads per thread, all issued before
+  // the shared-memory stores.  The rows are read with the lanes of a warp on
+  // consecutive rows (same 16 bytes of each), so that their transposing
+  // stores Rt[p][r] hit consecutive banks.
   {
     float4 d[16], y[8];
 #pragma unroll
     for (int i = 0; i < 16; ++i) d[i] = reinterpret_cast<const float4*>(dinv)[threadIdx.x + 256 * i];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int e = threadIdx.x + 256 * i, r = e >> 5, p4 = (e & 31) * 4;
+      const int e = threadIdx.x + 256 * i, r = e & 63, p4 = (e >> 6) * 4;
       y[i] = (r0 + r < a.r1) ? *reinterpret_cast<const float4*>(cy + (long long)(r0 + r) * a.ld + p4)
                              : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int e = threadIdx.x + 256 * i, cc = e >> 5, p4 = (e & 31) * 4;     // Dinv[cc][p4 ..]
-      Dt[(p4 + 0) * LDD + cc] = d[i].x;
-      Dt[(p4 + 1) * LDD + cc] = d[i].y;
-      Dt[(p4 + 2) * LDD + cc] = d[i].z;
-      Dt[(p4 + 3) * LDD + cc] = d[i].w;
+      const int e = threadIdx.x + 256 * i, pr = e >> 5, c4 = (e & 31) * 4;     // DinvT[pr][c4 ..]
+      *reinterpret_cast<float4*>(&Dt[pr * LDD + c4]) = d[i];
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int e = threadIdx.x + 256 * i, r = e >> 5, p4 = (e & 31) * 4;
+      const int e = threadIdx.x + 256 * i, r = e & 63, p4 = (e >> 6) * 4;
       Rt[(p4 + 0) * LDR + r] = y[i].x;
       Rt[(p4 + 1) * LDR + r] = y[i].y;
       Rt[(p4 + 2) * LDR + r] = y[i].z;

@@ -140,8 +140,8 @@ void launch_qr_control(const float* C, long long ld, long long mat_stride, int q
 // Diagonal block j of each matrix's Cholesky factor: C[b] + (128 j)(ld + 1)
 // holds the 128 x 128 Schur complement block; factor it with the matrix's
 // pivot floor, record the smallest pivot, and write the inverse of the
-// lower factor to Dinv[b] (128 x 128).  A pivot at or below the floor sets
-// fail[b] and skip[b].
+// lower factor, transposed (an upper-triangular 128 x 128 matrix), to
+// Dinv[b].  A pivot at or below the floor sets fail[b] and skip[b].
 void launch_qr_chol(const float* C, long long ld, long long mat_stride, int q, int j, float* Dinv,
                     const QrCtl& c, cudaStream_t s);
 

@@ -208,7 +208,17 @@ def test_cold_start_square_two_sided(ctx):
             ratio_emu = np.linalg.norm(emu["dW"]) / (HP["lr"] * np.sqrt(m * n))
             assert abs(ratio - ratio_emu) <= 1e-2, (ratio, ratio_emu)
         else:
-            assert rel(dW, emu["dW"]) <= 2e-2, (t, rel(dW, emu["dW"]))
+            # the refresh is gated column by column above; the rest of the
+            # step (rotations, Adam in the basis, rotation back, apply) is
+            # checked against the emulation run with the GPU's refreshed
+            # bases.  (Compared with the emulation's own bases instead, the
+            # update would differ by a few percent at these early steps: V is
+            # still tiny, so Adam magnifies the fp32-level differences of the
+            # bases' ill-determined columns.)
+            given = osoap.soap_step(S["W"], G, S["M"], S["V"], S["L"], out["QL"], S["R"], out["QR"], t=t,
+                                    precision="bf16", refresh=False, **HP)
+            assert rel(dW, given["dW"]) <= 1e-2, (t, rel(dW, given["dW"]))
+            assert rel(out["V"], given["V"]) <= 1e-2, (t, rel(out["V"], given["V"]))
         S = {k: out[k].astype(np.float32) for k in S}
 
 

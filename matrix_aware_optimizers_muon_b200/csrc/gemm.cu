@@ -11,6 +11,11 @@
 #include "profile.h"
 #include "runtime.h"
 
+// products with K up to this many columns use two sets of epilogue warps
+#ifndef MO_EPI2_MAX_K
+#define MO_EPI2_MAX_K 2048
+#endif
+
 namespace mo {
 
 namespace {
@@ -237,10 +242,13 @@ cudaError_t launch_gemm(const GemmOp& op, int* status, cudaStream_t stream) {
       default: return launch_t<256, 1, 1, true>(op, status, stream);
     }
   }
-  // two sets of epilogue warps when K is short: a tile's main loop (K / 64
-  // steps) is then no longer than one set's epilogue, which would otherwise
-  // leave the tensor pipe idle between tiles
-  const bool epi2 = op.K <= 2048;
+  // two sets of epilogue warps when K is short and every CTA gets at least
+  // two tiles: a tile's main loop (K / 64 steps) is then no longer than one
+  // set's epilogue, which would otherwise leave the tensor pipe idle
+  // between tiles
+  const int bn = narrow ? 128 : 256;
+  const long long tiles = (long long)((op.M + GEMM_BM - 1) / GEMM_BM) * ((op.N + bn - 1) / bn) * op.batch;
+  const bool epi2 = op.K <= MO_EPI2_MAX_K && tiles >= 2LL * device_sm_count();
   const int sel = (epi2 ? 8 : 0) | (narrow ? 4 : 0) | (op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0);
   switch (sel) {
     case 0: return launch_t<256, 0, 0>(op, status, stream);

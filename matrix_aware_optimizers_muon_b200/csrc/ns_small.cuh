@@ -25,6 +25,7 @@ struct SmallArgs {
   float* const* out;
   int32_t* const* flag;       // null or table (entries may be null)
   int* status;
+  uint32_t cols_magic;        // set by the launcher: ceil(2^32 / cols), row = umulhi(index, magic)
 };
 
 // Uploads `n` entries of four pointer tables (in, mom, out, flag) into device

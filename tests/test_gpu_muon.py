@@ -219,6 +219,9 @@ def test_ns_coefficient_variants(ctx, coeffs, steps, band):
     [(64, 200)] * 170 + [(200, 64)] * 130,    # one bucket, both orientations, > 148 per launch
     [(128, 256), (256, 128), (128, 128)],     # the largest shapes the fused kernel takes
     [(1, 1), (5, 250), (33, 100), (100, 33), (127, 255)],   # ragged tails
+    # bulk-copied loads and stores (n' <= 128, rows of 16-byte multiples),
+    # wide and tall, more matrices than CTAs (several per CTA)
+    [(96, 128)] * 500 + [(128, 96)] * 470 + [(128, 128)] * 460,
 ])
 def test_small_fused_batches(ctx, shapes):
     rng = wl.rng_of("small-fused", len(shapes), shapes[0])
@@ -233,6 +236,23 @@ def test_small_fused_batches(ctx, shapes):
     Wr, Br, _ = run_gpu_muon(ctx, Ws, Gs, Bs)
     for i in pick:
         np.testing.assert_array_equal(Wr[i], Wg[i])   # bitwise repeatable
+
+
+def test_small_ns_bulk_many(ctx):
+    """Plain NS through the fused kernel's bulk-copy path with several
+    matrices per CTA: a padded wide shape, its transpose, and full tiles;
+    matrices taken from the first and later rounds of a CTA."""
+    rng = wl.rng_of("small-ns-bulk")
+    shapes = [(100, 128)] * 500 + [(128, 100)] * 500 + [(128, 128)] * 450
+    mats = [wl.gaussian(rng, s, 1.0) for s in shapes]
+    outs = ctx.ns_orthogonalize([_cuda(m) for m in mats])
+    assert ctx.device_status() == 0
+    for i in (0, 449, 499, 500, 950, 999, 1000, 1449):
+        G = mats[i]
+        U, s, Vt = np.linalg.svd(G.astype(np.float64), full_matrices=False)
+        t = s / (np.linalg.norm(s) + 1e-7)
+        exact = (U * ons.scalar_map(t)) @ Vt
+        ns_gate(G, _np(outs[i]), exact, ons.newton_schulz_bf16(G), svd=(U, s, Vt))
 
 
 @pytest.mark.parametrize("kw", [dict(nesterov=False), dict(momentum_ema=True), dict(ns_steps=3),

@@ -15,6 +15,10 @@
 #ifndef MO_EPI2_MAX_K
 #define MO_EPI2_MAX_K 2048
 #endif
+// 1: outputs of non-symmetric products with a TMA-read C leave by TMA stores
+#ifndef MO_GEMM_DTMA
+#define MO_GEMM_DTMA 1
+#endif
 
 namespace mo {
 
@@ -104,8 +108,9 @@ template <int BN, int A_MN, int B_MN, bool PAIR = false, bool EPI2 = false>
 cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   using Cfg = GemmCfg<BN, PAIR, EPI2>;
   constexpr int BM_T = PAIR ? 2 * GEMM_BM : GEMM_BM;
-  CUtensorMap ta, tb, tc;
+  CUtensorMap ta, tb, tc, td;
   std::memset(&tc, 0, sizeof(tc));
+  std::memset(&td, 0, sizeof(td));
   const int nseg = op.nseg > 1 ? op.nseg : 1;
   if (nseg > 8 || (nseg > 1 && op.K % (nseg * GEMM_BK) != 0)) return cudaErrorInvalidValue;
   const long long kseg = op.K / nseg;
@@ -157,6 +162,15 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
     if (!encode_bf16_c(&tc, op.C, op.M, op.N, op.ldc, op.strideC, op.batch)) return cudaErrorInvalidValue;
     p.c_tma = 1;
   }
+  // ... and then a strided bf16 D of a non-symmetric plain product is
+  // written by TMA stores from the slots its C blocks arrived in
+  p.d_tma = 0;
+  if (p.c_tma && op.epi == EPI_AXPBY && !op.sym && op.d_tab == nullptr && op.D != nullptr &&
+      (op.batch == 1 || op.strideD % 8 == 0) && op.ldd % 8 == 0 && (reinterpret_cast<uintptr_t>(op.D) & 15) == 0 &&
+      MO_GEMM_DTMA) {
+    if (!encode_bf16_c(&td, op.D, op.M, op.N, op.ldd, op.strideD, op.batch)) return cudaErrorInvalidValue;
+    p.d_tma = 1;
+  }
 
   auto kern = gemm_bf16_kernel<BN, A_MN, B_MN, PAIR, EPI2>;
   cudaError_t ea = ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES);
@@ -180,7 +194,7 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   // executed tensor-core flops: computed tiles x 128 x BN x padded K x 2
   const double flops = 2.0 * tiles * p.batch * BM_T * BN * (double)round_up(p.K, GEMM_BK);
   ProfScope prof(op.kind, stream, flops);
-  return launch_pdl(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, stream, PAIR, ta, tb, tc, p);
+  return launch_pdl(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, stream, PAIR, ta, tb, tc, td, p);
 }
 
 }  // namespace

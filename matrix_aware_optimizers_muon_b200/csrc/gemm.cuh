@@ -66,6 +66,10 @@ struct GemmParams {
   const int* skip;
   // bf16 C read by TMA (tensor map tmC, 32 x 32 boxes, 64-byte swizzle)
   int c_tma;
+  // with c_tma, non-symmetric: the bf16 D blocks are written by TMA stores
+  // (tensor map tmD, same boxes) from the shared-memory slot their C block
+  // arrived in
+  int d_tma;
   // tile order: bands of `band` row tiles, each band column by column; a
   // band of tiles_m rows (or more) is the plain column order
   int band;
@@ -471,7 +475,8 @@ __device__ __forceinline__ void stage_store32_f32_diag(uint8_t* stg, int lane, c
 template <int BN, int A_MN, int B_MN, bool PAIR = false, bool EPI2 = false>
 __global__ void __launch_bounds__(GemmCfg<BN, PAIR, EPI2>::THREADS, 1) __maxnreg__(EPI2 ? 200 : 255)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+                 const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
+                 const GemmParams p) {
   static_assert(!(PAIR && EPI2), "CTA pairs run one set of epilogue warps");
   using Cfg = GemmCfg<BN, PAIR, EPI2>;
   constexpr int STAGES = Cfg::STAGES;
@@ -487,8 +492,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint64_t* cbar = drain + 1;                 // [epilogue warps][2]: C blocks read by TMA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 2 * Cfg::EPI_WARPS);
+  uint64_t* cbar = drain + 1;                 // [epilogue warps][4]: C blocks read by TMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 4 * Cfg::EPI_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* consumed = abort_flag + 1;
 
@@ -509,7 +514,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(&acc_empty[a], PAIR ? 256 : 128);   // the epilogue threads of every CTA of the tile
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < 2 * Cfg::EPI_WARPS; ++i) mbar_init(&cbar[i], 1);
+    for (int i = 0; i < 4 * Cfg::EPI_WARPS; ++i) mbar_init(&cbar[i], 1);
     *abort_flag = 0;
     *consumed = 0;
     fence_barrier_init();
@@ -655,12 +660,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int row_in_tile = q * 32 + lane;
     uint8_t* stg = smem + STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES + ew * 8192;
     uint8_t* stc = stg + 4096;              // staged 32 x 32 bf16 block of C
-    // two 2 KB buffers (at stg + 4096 and + 6144, 1 KB aligned) for C blocks
-    // that TMA writes in the 64-byte-swizzled layout stg_off() reads
-    uint8_t* cbuf0 = stg + 4096;           // buffer bi at cbuf0 + 2048 bi
-    uint64_t* cb = cbar + 2 * ew;
-    uint32_t cph = 0u;                      // bit bi: phase of buffer bi
-    uint32_t cpend = 0u;                    // bit bi: a copy into buffer bi is in flight
+    // C blocks that TMA writes in the 64-byte-swizzled layout stg_off()
+    // reads go to 2 KB slots (1 KB aligned) at stg + 2048 slot: slots 2 and
+    // 3 while stg holds the output staging rows, all four when the output
+    // leaves by TMA stores from the C slots themselves
+    uint64_t* cb = cbar + 4 * ew;
+    uint32_t cph = 0u;                      // bit i: phase of slot i
+    uint32_t cpend = 0u;                    // bit i: a copy into slot i is in flight
     const bool plain_bf16 = !p.d_f32 && !p.d_split;
     const bool plain_f32 = p.d_f32 && !p.d_split;
     const bool has_c = p.C != nullptr || p.c_tab != nullptr;
@@ -724,16 +730,29 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const bool wvec = wfull && !wtall && p.ap_vec;
       const bool wtr = wfull && wtall;
       const bool ctma = p.c_tma && !adam && plain_bf16 && n0 + BN <= p.N && __all_sync(0xffffffffu, row_ok);
-      auto issue_c = [&](int bi, int cc) {
-        mbar_arrive_expect_tx(&cb[bi], 32 * 32 * 2);
-        tma_load_3d(cbuf0 + 2048 * bi, &tmC, &cb[bi], n0 + cc, r0, b);
-        cpend |= 1u << bi;
+      // output blocks by TMA store, written over their C block's slot;
+      // C requested three blocks ahead
+      const bool dtma = ctma && p.d_tma;
+      auto issue_c = [&](int slot, int cc) {
+        mbar_arrive_expect_tx(&cb[slot], 32 * 32 * 2);
+        tma_load_3d(stg + 2048 * slot, &tmC, &cb[slot], n0 + cc, r0, b);
+        cpend |= 1u << slot;
       };
       if (ctma && lane == 0) {
-        fence_proxy_async_smem();              // earlier reads of the buffers come first
-        if (cc_begin < BN) issue_c(0, cc_begin);
-        if (cc_begin + 32 < BN) issue_c(1, cc_begin + 32);
+        fence_proxy_async_smem();              // earlier reads of the slots come first
+        if (dtma) {
+          bulk_wait_read();                    // the previous tile's stores have read their slots
+          for (int i = 0; i < 3; ++i)
+            if (cc_begin + 32 * i < BN) issue_c(i, cc_begin + 32 * i);
+        } else {
+          if (cc_begin < BN) issue_c(2, cc_begin);
+          if (cc_begin + 32 < BN) issue_c(3, cc_begin + 32);
+        }
       }
+      // with TMA stores in the launch, the previous tile's stores must have
+      // read their slots before any lane writes the staging area again (the
+      // vote after the accumulator wait orders the other lanes after this)
+      if (p.d_tma && lane == 0) bulk_wait_read();
       // warp-uniform: tcgen05.ld below must be executed by all 32 lanes
       const bool ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status, DEV_TIMEOUT_ACC_FULL);
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -837,13 +856,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
               x[4 * u + 3] = fmaf(beta, w.w, x[4 * u + 3]);
             }
           } else if (ctma) {
-            const int bi = kk & 1;
+            const int bi = dtma ? (kk & 3) : 2 + (kk & 1);
             mbar_wait(&cb[bi], (cph >> bi) & 1u, abort_flag, p.status, DEV_TIMEOUT_ACC_FULL);
             cph ^= 1u << bi;
             cpend &= ~(1u << bi);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              const uint4 w = *reinterpret_cast<const uint4*>(cbuf0 + 2048 * bi + stg_off(lane, u));
+              const uint4 w = *reinterpret_cast<const uint4*>(stg + 2048 * bi + stg_off(lane, u));
               const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
@@ -852,10 +871,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 x[8 * u + 2 * j + 1] = fmaf(beta, f.y, x[8 * u + 2 * j + 1]);
               }
             }
-            __syncwarp();                 // every lane has read the buffer
-            if (lane == 0) {
-              fence_proxy_async_smem();
-              if (cc + 64 < BN) issue_c(bi, cc + 64);
+            if (!dtma) {
+              __syncwarp();               // every lane has read the buffer
+              if (lane == 0) {
+                fence_proxy_async_smem();
+                if (cc + 64 < BN) issue_c(bi, cc + 64);
+              }
             }
           } else if (cpre) {
             __syncwarp();                 // the previous block's reads of stc are done
@@ -928,6 +949,30 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             float* d32 = reinterpret_cast<float*>(dbase);
             stage_store32_f32(stg, lane, x, d32 + (long long)r0 * p.ldd + c0,
                               p.sym ? d32 + (long long)c0 * p.ldd + r0 : nullptr, p.ldd);
+          } else if (fast && dtma) {
+            // this lane's row of bf16 output over the row of C it read, then
+            // one TMA store of the block; the slot of the previous block is
+            // free once its store has read it and takes the C block three
+            // ahead
+            uint8_t* slot = stg + 2048 * (kk & 3);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint32_t w[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(x[8 * u + 2 * j], x[8 * u + 2 * j + 1]);
+                w[j] = *reinterpret_cast<const uint32_t*>(&h);
+              }
+              *reinterpret_cast<uint4*>(slot + stg_off(lane, u)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tmD, slot, n0 + cc, r0, b);
+              bulk_commit();
+              bulk_wait_read_but1();
+              if (cc + 96 < BN) issue_c((kk + 3) & 3, cc + 96);
+            }
           } else if (fast) {
             __nv_bfloat16* d16 = reinterpret_cast<__nv_bfloat16*>(dbase);
             stage_store32(stg, lane, x, d16 + (long long)r0 * p.ldd + c0,
@@ -947,10 +992,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       if constexpr (PAIR) mbar_arrive_cluster(acc ? acc_empty_cl1 : acc_empty_cl0);
       else mbar_arrive(&acc_empty[acc]);
     }
-    // C blocks requested for a tile that was abandoned must land before exit
-    if (lane == 0)
-      for (int bi = 0; bi < 2; ++bi)
+    // C blocks requested for a tile that was abandoned must land before
+    // exit, and the output stores must be complete
+    if (lane == 0) {
+      for (int bi = 0; bi < 4; ++bi)
         if ((cpend >> bi) & 1u) mbar_wait_drain(&cb[bi], (cph >> bi) & 1u, p.status);
+      bulk_wait_all();
+    }
   }
 
   __syncthreads();

@@ -15,6 +15,17 @@
 #ifndef MO_EPI2_MAX_K
 #define MO_EPI2_MAX_K 2048
 #endif
+// 1: short-K products with two epilogue sets take 128-wide tiles and four
+// accumulators
+#ifndef MO_SHORTK_NARROW
+#define MO_SHORTK_NARROW 0
+#endif
+// 1: short-K products with two epilogue sets and more than one row tile run
+// on CTA pairs (256 x 256 tiles, each CTA staging half of B: a third fewer
+// bytes from L2 per flop, the bound of these products)
+#ifndef MO_SHORTK_PAIR
+#define MO_SHORTK_PAIR 1
+#endif
 // 1: outputs of non-symmetric products with a TMA-read C leave by TMA stores
 #ifndef MO_GEMM_DTMA
 #define MO_GEMM_DTMA 1
@@ -247,15 +258,7 @@ cudaError_t launch_gemm(const GemmOp& op, int* status, cudaStream_t stream) {
   // by the per-tile epilogue, which narrower tiles spread over more SMs);
   // 256 otherwise
   const long long wide_tiles = (long long)((op.M + GEMM_BM - 1) / GEMM_BM) * ((op.N + 255) / 256) * op.batch;
-  const bool narrow = op.N <= 128 || wide_tiles * 4 < device_sm_count();
-  if (!narrow && op.M > GEMM_BM && pairs_enabled()) {
-    switch ((op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0)) {
-      case 0: return launch_t<256, 0, 0, true>(op, status, stream);
-      case 1: return launch_t<256, 0, 1, true>(op, status, stream);
-      case 2: return launch_t<256, 1, 0, true>(op, status, stream);
-      default: return launch_t<256, 1, 1, true>(op, status, stream);
-    }
-  }
+  bool narrow = op.N <= 128 || wide_tiles * 4 < device_sm_count();
   // two sets of epilogue warps when K is short and every CTA gets at least
   // two tiles: a tile's main loop (K / 64 steps) is then no longer than one
   // set's epilogue, which would otherwise leave the tensor pipe idle
@@ -263,6 +266,21 @@ cudaError_t launch_gemm(const GemmOp& op, int* status, cudaStream_t stream) {
   const int bn = narrow ? 128 : 256;
   const long long tiles = (long long)((op.M + GEMM_BM - 1) / GEMM_BM) * ((op.N + bn - 1) / bn) * op.batch;
   const bool epi2 = op.K <= MO_EPI2_MAX_K && tiles >= 2LL * device_sm_count();
+  if (!narrow && op.M > GEMM_BM && (pairs_enabled() || (epi2 && MO_SHORTK_PAIR))) {
+    switch ((epi2 ? 4 : 0) | (op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0)) {
+      case 0: return launch_t<256, 0, 0, true>(op, status, stream);
+      case 1: return launch_t<256, 0, 1, true>(op, status, stream);
+      case 2: return launch_t<256, 1, 0, true>(op, status, stream);
+      case 3: return launch_t<256, 1, 1, true>(op, status, stream);
+      case 4: return launch_t<256, 0, 0, true, true>(op, status, stream);
+      case 5: return launch_t<256, 0, 1, true, true>(op, status, stream);
+      case 6: return launch_t<256, 1, 0, true, true>(op, status, stream);
+      default: return launch_t<256, 1, 1, true, true>(op, status, stream);
+    }
+  }
+  // with two epilogue sets, 128-wide tiles get four accumulators: a tile's
+  // epilogue then no longer holds up the main loop of the tile after next
+  if (epi2 && MO_SHORTK_NARROW) narrow = true;
   const int sel = (epi2 ? 8 : 0) | (narrow ? 4 : 0) | (op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0);
   switch (sel) {
     case 0: return launch_t<256, 0, 0>(op, status, stream);

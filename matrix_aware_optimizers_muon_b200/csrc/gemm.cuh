@@ -106,8 +106,12 @@ struct GemmCfg {
   static constexpr int BN_LOCAL = PAIR ? BN / 2 : BN;
   static constexpr int B_BYTES = BN_LOCAL * GEMM_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = PAIR ? 6 : (BN == 256 ? (EPI2 ? 3 : 4) : (EPI2 ? 4 : 6));
-  static constexpr int TMEM_COLS = 2 * BN;          // two fp32 accumulators
+  static constexpr int STAGES = PAIR ? (EPI2 ? 5 : 6) : (BN == 256 ? (EPI2 ? 3 : 4) : (EPI2 ? 5 : 6));
+  // fp32 accumulators in tensor memory: two, or four 128-column ones with
+  // two epilogue sets (each set then drains every other accumulator, and a
+  // tile's epilogue overlaps the next three tiles' main loops)
+  static constexpr int NACC = (EPI2 && BN == 128) ? 4 : 2;
+  static constexpr int TMEM_COLS = NACC * BN;
   static constexpr int BAR_BYTES = 1024;            // mbarriers; keeps the epilogue stage 1 KB aligned
   static constexpr int EPI_WARPS = EPI2 ? 8 : 4;
   static constexpr int EPI_BYTES = EPI_WARPS * 8192;  // per epilogue warp: output block (or C), its transpose
@@ -477,7 +481,6 @@ __global__ void __launch_bounds__(GemmCfg<BN, PAIR, EPI2>::THREADS, 1) __maxnreg
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                  const GemmParams p) {
-  static_assert(!(PAIR && EPI2), "CTA pairs run one set of epilogue warps");
   using Cfg = GemmCfg<BN, PAIR, EPI2>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int BM_T = PAIR ? 2 * GEMM_BM : GEMM_BM;     // rows per tile
@@ -490,8 +493,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* acc_empty = acc_full + Cfg::NACC;
+  uint64_t* drain = acc_empty + Cfg::NACC;
   uint64_t* cbar = drain + 1;                 // [epilogue warps][4]: C blocks read by TMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 4 * Cfg::EPI_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -509,7 +512,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < Cfg::NACC; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], PAIR ? 256 : 128);   // the epilogue threads of every CTA of the tile
     }
@@ -642,8 +645,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         if (!ok) break;
         if constexpr (PAIR) tc_commit_pair(&acc_full[acc], 3);     // both CTAs' epilogues
         else tc_commit(&acc_full[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == Cfg::NACC) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       if (any) {
         // every MMA issued by this thread must finish before TMEM is freed
@@ -672,17 +677,17 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const bool has_c = p.C != nullptr || p.c_tab != nullptr;
     const bool adam = p.epi == EPI_ADAM;
     const bool apply = p.epi == EPI_APPLY;
-    int ntile = 0;                          // tiles of this CTA so far: accumulator ntile % 2
+    int ntile = 0;                          // tiles of this CTA so far: accumulator ntile % NACC
     // a pair's epilogue threads release the accumulator on the even CTA's barrier
     const uint32_t acc_empty_cl0 = PAIR ? mapa_shared(&acc_empty[0], 0) : 0u;
     const uint32_t acc_empty_cl1 = PAIR ? mapa_shared(&acc_empty[1], 0) : 0u;
     for (int t = unit; t < total; t += units) {
       int b, tm, tn;
       if (!gemm_decode(p, BN, t, b, tm, tn)) continue;
-      const int acc = ntile & 1;
-      const uint32_t acc_phase = (uint32_t)(ntile >> 1) & 1u;
+      const int acc = ntile % Cfg::NACC;
+      const uint32_t acc_phase = (uint32_t)(ntile / Cfg::NACC) & 1u;
       ++ntile;
-      if (EPI2 && acc != eset) continue;    // the other set's tile
+      if (EPI2 && (acc & 1) != eset) continue;    // the other set's tile
       const int r = tm * BM_T + (int)rank * GEMM_BM + row_in_tile;
       const bool row_ok = r < p.M;
       // this matrix's operands, resolved once per tile

@@ -173,10 +173,12 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
     if (!encode_bf16_c(&tc, op.C, op.M, op.N, op.ldc, op.strideC, op.batch)) return cudaErrorInvalidValue;
     p.c_tma = 1;
   }
-  // ... and then a strided bf16 D of a non-symmetric plain product is
-  // written by TMA stores from the slots its C blocks arrived in
+  // a strided bf16 D of a plain product whose C (if any) comes by TMA is
+  // written by TMA stores: from the slots its C blocks arrived in
+  // (non-symmetric with C), else from staging slots
   p.d_tma = 0;
-  if (p.c_tma && op.epi == EPI_AXPBY && !op.sym && op.d_tab == nullptr && op.D != nullptr &&
+  if ((p.c_tma || (op.C == nullptr && op.c_tab == nullptr)) && op.epi == EPI_AXPBY && !op.d_f32 && !op.d_split && op.d_tab == nullptr &&
+      op.D != nullptr &&
       (op.batch == 1 || op.strideD % 8 == 0) && op.ldd % 8 == 0 && (reinterpret_cast<uintptr_t>(op.D) & 15) == 0 &&
       MO_GEMM_DTMA) {
     if (!encode_bf16_c(&td, op.D, op.M, op.N, op.ldd, op.strideD, op.batch)) return cudaErrorInvalidValue;

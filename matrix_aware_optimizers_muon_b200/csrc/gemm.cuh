@@ -66,9 +66,10 @@ struct GemmParams {
   const int* skip;
   // bf16 C read by TMA (tensor map tmC, 32 x 32 boxes, 64-byte swizzle)
   int c_tma;
-  // with c_tma, non-symmetric: the bf16 D blocks are written by TMA stores
-  // (tensor map tmD, same boxes) from the shared-memory slot their C block
-  // arrived in
+  // full 32 x 32 blocks of a plain bf16 D are written by TMA stores (tensor
+  // map tmD, same boxes): non-symmetric with c_tma, from the slot their C
+  // block arrived in; otherwise from staging slots (a symmetric product's
+  // mirror block by a second store)
   int d_tma;
   // tile order: bands of `band` row tiles, each band column by column; a
   // band of tiles_m rows (or more) is the plain column order
@@ -382,6 +383,47 @@ __device__ __forceinline__ void stage_store32(uint8_t* stg, int lane, const floa
 // takes the value computed above the diagonal (its own for c >= r, its
 // mirror's for c < r), so both halves are bit-equal, with the same coalesced
 // row stores.
+// For TMA stores of a 32 x 32 bf16 block: this lane's row into `own` and,
+// when `mir` is set, its transpose (the mirror block) into `mir`, both in
+// the 64-byte-swizzled rows of stg_off().
+__device__ __forceinline__ void stage_rows_tma(uint8_t* own, uint8_t* mir, int lane, const float (&x)[32]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(x[8 * u + 2 * j], x[8 * u + 2 * j + 1]);
+      w[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(own + stg_off(lane, u)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (mir) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      *reinterpret_cast<__nv_bfloat16*>(mir + stg_off(i, lane >> 3) + ((lane & 7) << 1)) = __float2bfloat16_rn(x[i]);
+  }
+}
+
+// A staged block on the diagonal of a symmetric product (own rows and their
+// transpose staged, then a __syncwarp): every element below the diagonal
+// takes its mirror's value, in place in `own`; each lane rewrites the
+// 16-byte units it reads.
+__device__ __forceinline__ void symmetrize_staged(uint8_t* own, const uint8_t* mir, int lane) {
+  const int u = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int R = 8 * j + (lane >> 2);
+    uint4 a = *reinterpret_cast<const uint4*>(own + stg_off(R, u));
+    const uint4 m = *reinterpret_cast<const uint4*>(mir + stg_off(R, u));
+    uint16_t* pa = reinterpret_cast<uint16_t*>(&a);
+    const uint16_t* pm = reinterpret_cast<const uint16_t*>(&m);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (8 * u + e < R) pa[e] = pm[e];
+    *reinterpret_cast<uint4*>(own + stg_off(R, u)) = a;
+  }
+}
+
 __device__ __forceinline__ void stage_store32_diag(uint8_t* stg, int lane, const float (&x)[32], __nv_bfloat16* drow,
                                                    long long ldd) {
   uint8_t* srow = stg;
@@ -737,7 +779,9 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const bool ctma = p.c_tma && !adam && plain_bf16 && n0 + BN <= p.N && __all_sync(0xffffffffu, row_ok);
       // output blocks by TMA store, written over their C block's slot;
       // C requested three blocks ahead
-      const bool dtma = ctma && p.d_tma;
+      const bool dtma = ctma && p.d_tma && !p.sym;
+      // ... or from the staging slots 0 (own block) and 1 (mirror block)
+      const bool dstg = p.d_tma && !dtma && n0 + BN <= p.N && (!has_c || ctma) && __all_sync(0xffffffffu, row_ok);
       auto issue_c = [&](int slot, int cc) {
         mbar_arrive_expect_tx(&cb[slot], 32 * 32 * 2);
         tma_load_3d(stg + 2048 * slot, &tmC, &cb[slot], n0 + cc, r0, b);
@@ -943,6 +987,24 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                   *w = fmaf(p.ap_decay, *w, -wstep * x[i]);
                 }
               }
+            }
+          } else if (dstg && (fast || (diag && plain_bf16))) {
+            // the previous block's stores have read the staging slots
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
+            uint8_t* own = stg;
+            uint8_t* mir = stg + 2048;
+            stage_rows_tma(own, (p.sym || diag) ? mir : nullptr, lane, x);
+            if (diag) {
+              __syncwarp();
+              symmetrize_staged(own, mir, lane);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tmD, own, c0, r0, b);
+              if (p.sym && !diag) tma_store_3d(&tmD, mir, r0, c0, b);
+              bulk_commit();
             }
           } else if (diag) {
             if (plain_f32)

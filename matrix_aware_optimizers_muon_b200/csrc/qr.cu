@@ -327,85 +327,96 @@ __global__ void __launch_bounds__(256) qr_chol_kernel(const float* C, long long 
   }
 }
 
-// out = in * Dinv^T for 64 rows x 128 columns per CTA (256 threads):
-// thread (ty, tx) computes rows 4 ty .. +3 and columns 8 tx .. +7 from
-// transposed shared copies of the rows and of Dinv (Dinv lower: p <= c;
-// its global copy is stored transposed).
-__global__ void __launch_bounds__(256) qr_panel_kernel(const PanelArgs a) {
+// out = in * Dinv^T for 128 rows x 128 columns per CTA (256 threads), from
+// transposed shared copies of the rows and of Dinv (Dinv lower: p <= c; its
+// global copy is stored transposed).  Column group g (8 columns) needs p <=
+// 8 g + 7 only; lane l of warp w computes rows 4 l .. 4 l + 3 for the groups
+// w and 15 - w in turn, so every warp runs the same 136 steps of the p loop
+// with all lanes on the same bound.
+constexpr int PANEL_ROWS = 128;
+constexpr int PANEL_LDD = QR_B + 4;           // Dt[p][c] = Dinv[c][p]
+constexpr int PANEL_LDR = PANEL_ROWS + 4;     // Rt[p][r] = in[r0 + r][p]
+constexpr int PANEL_SMEM = (QR_B * PANEL_LDD + QR_B * PANEL_LDR) * 4;
+
+__global__ void __launch_bounds__(256, 1) qr_panel_kernel(const PanelArgs a) {
   const int b = blockIdx.y;
   if (a.skip[b]) return;
   extern __shared__ float sm[];
-  constexpr int LDD = QR_B + 4;        // Dt[p][c] = Dinv[c][p]
-  constexpr int LDR = 64 + 4;          // Rt[p][r] = in[r0 + r][p]
   float* Dt = sm;
-  float* Rt = sm + QR_B * LDD;
-  const int r0 = a.r0 + blockIdx.x * 64;
+  float* Rt = sm + QR_B * PANEL_LDD;
+  const int r0 = a.r0 + blockIdx.x * PANEL_ROWS;
   const long long col0 = (long long)a.j * QR_B;
   const float* dinv = a.Dinv + (size_t)b * QR_B * QR_B;
   float* cy = a.CY + (size_t)b * a.mat_stride + col0;
-  // DinvT (4096 float4, stored transposed by the diagonal-block kernel) and
-  // the 64 x 128 rows (2048 float4): 24 loads per thread, all issued before
-  // the shared-memory stores.  The rows are read with the lanes of a warp on
+  // DinvT (4096 float4) and the 128 x 128 rows (4096 float4) in two halves
+  // of 8 + 8 loads per thread, each half's loads issued before its
+  // shared-memory stores.  The rows are read with the lanes of a warp on
   // consecutive rows (same 16 bytes of each), so that their transposing
   // stores Rt[p][r] hit consecutive banks.
-  {
-    float4 d[16], y[8];
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    float4 d[8], y[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) d[i] = reinterpret_cast<const float4*>(dinv)[threadIdx.x + 256 * i];
+    for (int i = 0; i < 8; ++i) d[i] = reinterpret_cast<const float4*>(dinv)[threadIdx.x + 256 * (8 * half + i)];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int e = threadIdx.x + 256 * i, r = e & 63, p4 = (e >> 6) * 4;
+      const int e = threadIdx.x + 256 * (8 * half + i), r = e & (PANEL_ROWS - 1), p4 = (e >> 7) * 4;
       y[i] = (r0 + r < a.r1) ? *reinterpret_cast<const float4*>(cy + (long long)(r0 + r) * a.ld + p4)
                              : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int e = threadIdx.x + 256 * i, pr = e >> 5, c4 = (e & 31) * 4;     // DinvT[pr][c4 ..]
-      *reinterpret_cast<float4*>(&Dt[pr * LDD + c4]) = d[i];
+    for (int i = 0; i < 8; ++i) {
+      const int e = threadIdx.x + 256 * (8 * half + i), pr = e >> 5, c4 = (e & 31) * 4;     // DinvT[pr][c4 ..]
+      *reinterpret_cast<float4*>(&Dt[pr * PANEL_LDD + c4]) = d[i];
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int e = threadIdx.x + 256 * i, r = e & 63, p4 = (e >> 6) * 4;
-      Rt[(p4 + 0) * LDR + r] = y[i].x;
-      Rt[(p4 + 1) * LDR + r] = y[i].y;
-      Rt[(p4 + 2) * LDR + r] = y[i].z;
-      Rt[(p4 + 3) * LDR + r] = y[i].w;
+      const int e = threadIdx.x + 256 * (8 * half + i), r = e & (PANEL_ROWS - 1), p4 = (e >> 7) * 4;
+      Rt[(p4 + 0) * PANEL_LDR + r] = y[i].x;
+      Rt[(p4 + 1) * PANEL_LDR + r] = y[i].y;
+      Rt[(p4 + 2) * PANEL_LDR + r] = y[i].z;
+      Rt[(p4 + 3) * PANEL_LDR + r] = y[i].w;
     }
   }
   __syncthreads();
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  float acc[4][8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
-  const int pmax = 8 * tx + 7;
-  for (int p = 0; p <= pmax; ++p) {
-    const float4 rv = *reinterpret_cast<const float4*>(&Rt[p * LDR + 4 * ty]);
-    const float4 d0 = *reinterpret_cast<const float4*>(&Dt[p * LDD + 8 * tx]);
-    const float4 d1 = *reinterpret_cast<const float4*>(&Dt[p * LDD + 8 * tx + 4]);
-    const float rr[4] = {rv.x, rv.y, rv.z, rv.w};
-    const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __half* lq = a.LQ + (size_t)b * a.mat_stride + col0;
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    const int g = h == 0 ? warp : 15 - warp;
+    float acc[4][8];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc[i][k] = fmaf(rr[i], dd[k], acc[i][k]);
-  }
-  __half* lq = a.LQ + (size_t)b * a.mat_stride + col0;
+      for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
+    const int pmax = 8 * g + 7;
+#pragma unroll 2
+    for (int p = 0; p <= pmax; ++p) {
+      const float4 rv = *reinterpret_cast<const float4*>(&Rt[p * PANEL_LDR + 4 * lane]);
+      const float4 d0 = *reinterpret_cast<const float4*>(&Dt[p * PANEL_LDD + 8 * g]);
+      const float4 d1 = *reinterpret_cast<const float4*>(&Dt[p * PANEL_LDD + 8 * g + 4]);
+      const float rr[4] = {rv.x, rv.y, rv.z, rv.w};
+      const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int row = r0 + 4 * ty + i;
-    if (row >= a.r1) continue;
-    const int c0 = 8 * tx;
-    if (row >= a.f32_from) {
-      float* o = cy + (long long)row * a.ld + c0;
-      reinterpret_cast<float4*>(o)[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-      reinterpret_cast<float4*>(o)[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[i][k] = fmaf(rr[i], dd[k], acc[i][k]);
     }
-    float xs[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) xs[k] = acc[i][k] * QR_PLANE_SCALE;
-    store_planes_h8(lq + (long long)row * a.ld + c0, a.plane_stride, xs);
+    for (int i = 0; i < 4; ++i) {
+      const int row = r0 + 4 * lane + i;
+      if (row >= a.r1) continue;
+      const int c0 = 8 * g;
+      if (row >= a.f32_from) {
+        float* o = cy + (long long)row * a.ld + c0;
+        reinterpret_cast<float4*>(o)[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        reinterpret_cast<float4*>(o)[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+      }
+      float xs[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) xs[k] = acc[i][k] * QR_PLANE_SCALE;
+      store_planes_h8(lq + (long long)row * a.ld + c0, a.plane_stride, xs);
+    }
   }
 }
 
@@ -498,10 +509,9 @@ void launch_qr_chol(const float* C, long long ld, long long mat_stride, int q, i
 void launch_qr_panel(const PanelArgs& a, cudaStream_t s) {
   if (a.r1 <= a.r0) return;
   ProfScope prof(PK_QR_ROWBLK, s);
-  const int smem = (QR_B * (QR_B + 4) + QR_B * (64 + 4)) * 4;
-  (void)ensure_smem_attr(reinterpret_cast<const void*>(qr_panel_kernel), smem);
-  dim3 grid((a.r1 - a.r0 + 63) / 64, a.q);
-  qr_panel_kernel<<<grid, 256, smem, s>>>(a);
+  (void)ensure_smem_attr(reinterpret_cast<const void*>(qr_panel_kernel), PANEL_SMEM);
+  dim3 grid((a.r1 - a.r0 + PANEL_ROWS - 1) / PANEL_ROWS, a.q);
+  qr_panel_kernel<<<grid, 256, PANEL_SMEM, s>>>(a);
 }
 
 void launch_qr_finish(const QrCtl& c, const FlagTable& flags, int q, float* Y, long long ld,

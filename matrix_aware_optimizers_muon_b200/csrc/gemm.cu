@@ -162,6 +162,8 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   p.ap_tall_from = op.ap_tall_from;
   p.ap_vec = op.ap_vec;
   p.ab_f16 = op.ab_f16;
+  p.gate = op.gate;
+  p.gate_n = op.gate_n;
   if (op.epi == EPI_APPLY && (op.sym || op.e_tab == nullptr || op.d_f32 || op.d_split))
     return cudaErrorInvalidValue;
   // a strided bf16 C of the plain (or Muon apply) epilogue is read by TMA

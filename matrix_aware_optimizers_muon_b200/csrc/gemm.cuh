@@ -82,6 +82,9 @@ struct GemmParams {
   float ap_step[2];
   int ap_tall_from;
   int ap_vec;               // every W of the launch: 16-byte aligned rows
+  // launch gate: no tiles when *gate >= gate_n
+  const int* gate;
+  int gate_n;
   // A and B hold fp16 (not bf16) values: the same kind::f16 MMA with the
   // operand type fields of the instruction descriptor set to f16
   int ab_f16;
@@ -530,6 +533,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM_T, BN, A_MN, B_MN);
   const uint32_t IDESC = p.ab_f16 ? idesc_as_f16(IDESC_BF16) : IDESC_BF16;
 
+  // a gated launch reads its gate first (after its predecessor) and, when
+  // closed, leaves before any setup; the whole grid reads the same word
+  if (p.gate != nullptr) {
+    pdl_wait();
+    if (*p.gate >= p.gate_n) return;
+  }
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);

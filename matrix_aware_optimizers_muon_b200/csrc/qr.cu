@@ -5,6 +5,7 @@
 
 #include "chol_block.cuh"
 #include "profile.h"
+#include "ptx.cuh"
 #include "qr.cuh"
 #include "runtime.h"
 
@@ -28,6 +29,8 @@ __global__ void qr_init_kernel(const QrCtl c, int q) {
   c.shift[b] = 0.f;
   c.minpiv[b] = 0x7f800000u;
   c.dev[b] = 0u;
+  if (b == 0)
+    for (int p = 0; p < QR_MAX_PASSES; ++p) c.pass_done[p] = 0;
 }
 
 // One CTA per matrix: the largest diagonal entry, then a power-of-two scale
@@ -92,12 +95,7 @@ __device__ __forceinline__ float hash_uniform(unsigned b, unsigned r, unsigned c
   return (float)(h >> 8) * (2.0f / 16777216.0f) - 1.0f;
 }
 
-__global__ void split16_kernel(const Split16Args a) {
-  const int b = blockIdx.z;
-  if (a.skip && a.skip[b]) return;
-  const int r = blockIdx.y;
-  const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
-  if (c0 >= a.cols_pad || r >= a.rows_pad) return;
+__device__ __forceinline__ void split16_row(const Split16Args& a, int b, int r, int c0) {
   const bool rv = r < a.rows_valid;
   const float* src = a.src[b] + (long long)r * a.lds;
   float x[8];
@@ -141,11 +139,26 @@ __global__ void split16_kernel(const Split16Args a) {
   store_planes_h8(a.dst + (size_t)b * a.mat_stride + (long long)r * a.ldd + c0, a.plane_stride, x);
 }
 
+__global__ void split16_kernel(const Split16Args a) {
+  pdl_wait();
+  pdl_trigger();
+  if (a.gate && *a.gate >= a.gate_n) return;
+  const int b = blockIdx.z;
+  if (a.skip && a.skip[b]) return;
+  const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (c0 >= a.cols_pad) return;
+  for (int r = blockIdx.y; r < a.rows_pad; r += gridDim.y) split16_row(a, b, r, c0);
+}
+
 // 32 columns x 8 row groups per CTA; the 8 partial sums of a column are
 // added in a fixed order (bitwise reproducible).
 __global__ void __launch_bounds__(256) colnorm2_kernel(const float* Y, long long ld, long long stride, int rows,
-                                                       int cols, float* inv_d, const int* skip) {
+                                                       int cols, float* inv_d, const int* skip, const int* gate,
+                                                       int gate_n) {
   __shared__ float part[8][33];
+  pdl_wait();
+  pdl_trigger();
+  if (gate && *gate >= gate_n) return;
   const int b = blockIdx.y;
   if (skip && skip[b]) return;
   const int cx = threadIdx.x & 31, g = threadIdx.x >> 5;
@@ -171,8 +184,11 @@ __global__ void __launch_bounds__(256) colnorm2_kernel(const float* Y, long long
 
 // Partial Gram statistics: block g of matrix b covers rows [g rpb, (g+1) rpb).
 __global__ void __launch_bounds__(256) qr_check_kernel(const float* C, long long ld, long long stride, int kp,
-                                                       const QrCtl c) {
+                                                       const QrCtl c, const int* gate, int gate_n) {
   __shared__ float red[8];
+  pdl_wait();
+  pdl_trigger();
+  if (gate && *gate >= gate_n) return;
   const int b = blockIdx.y;
   if (c.done[b]) return;
   const int rpb = (kp + QR_CHECK_BLOCKS - 1) / QR_CHECK_BLOCKS;
@@ -216,8 +232,10 @@ __global__ void __launch_bounds__(256) qr_check_kernel(const float* C, long long
 // One CTA per matrix: the outcome of the previous attempt, the check of this
 // pass's Gram, the mode of this pass, and the shift of the diagonal.
 __global__ void __launch_bounds__(256) qr_decide_kernel(float* C, long long ld, long long stride, int kp,
-                                                        const QrCtl c) {
+                                                        const QrCtl c, int pass) {
   __shared__ float s_shift;
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   if (threadIdx.x == 0) {
     float sh = 0.f;
@@ -257,6 +275,7 @@ __global__ void __launch_bounds__(256) qr_decide_kernel(float* C, long long ld, 
       }
       c.dev[b] = 0u;                        // the next pass's check accumulates from zero
     }
+    if (c.done[b]) atomicAdd(c.pass_done + pass, 1);
     s_shift = sh;
   }
   __syncthreads();
@@ -270,7 +289,10 @@ __global__ void __launch_bounds__(256) qr_decide_kernel(float* C, long long ld, 
 // One CTA (256 threads) per matrix: Cholesky of the diagonal block with the
 // matrix's pivot floor, then the inverse of its lower factor.
 __global__ void __launch_bounds__(256) qr_chol_kernel(const float* C, long long ld, long long stride, int k0,
-                                                      float* Dinv, const QrCtl c) {
+                                                      float* Dinv, const QrCtl c, const int* gate, int gate_n) {
+  pdl_wait();
+  pdl_trigger();
+  if (gate && *gate >= gate_n) return;
   const int b = blockIdx.x;
   if (c.skip[b]) return;
   extern __shared__ float sm[];
@@ -339,6 +361,9 @@ constexpr int PANEL_LDR = PANEL_ROWS + 4;     // Rt[p][r] = in[r0 + r][p]
 constexpr int PANEL_SMEM = (QR_B * PANEL_LDD + QR_B * PANEL_LDR) * 4;
 
 __global__ void __launch_bounds__(256, 1) qr_panel_kernel(const PanelArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  if (a.gate && *a.gate >= a.q) return;
   const int b = blockIdx.y;
   if (a.skip[b]) return;
   extern __shared__ float sm[];
@@ -463,6 +488,7 @@ QrCtl qr_ctl_at(char* base, int q) {
   c.dev = reinterpret_cast<unsigned*>(base + 9 * w);
   c.fscale = reinterpret_cast<float*>(base + 10 * w);
   c.fiscale = reinterpret_cast<float*>(base + 11 * w);
+  c.pass_done = reinterpret_cast<int*>(base + 12 * w);     // QR_MAX_PASSES <= 256 words
   c.part = reinterpret_cast<float*>(base + 13 * w);
   return c;
 }
@@ -480,30 +506,37 @@ void launch_factor_scale(const FactorScaleArgs& a, const QrCtl& c, cudaStream_t 
 void launch_split16(const Split16Args& a, cudaStream_t s) {
   ProfScope prof(PK_SOAP_QR, s);
   const int per_block = 256 * 8;
-  dim3 grid((a.cols_pad + per_block - 1) / per_block, a.rows_pad, a.count);
-  split16_kernel<<<grid, 256, 0, s>>>(a);
+  // up to 256 row groups per matrix, each CTA looping over its rows: a
+  // gated-off launch then has few CTAs to retire
+  const int ry = a.rows_pad < 256 ? a.rows_pad : 256;
+  dim3 grid((a.cols_pad + per_block - 1) / per_block, ry, a.count);
+  (void)launch_pdl(split16_kernel, grid, dim3(256), 0, s, false, a);
 }
 
 void launch_colnorm2(const float* Y, long long ld, long long mat_stride, int count, int rows, int cols,
-                     float* inv_d, const int* skip, cudaStream_t s) {
+                     float* inv_d, const int* skip, const int* gate, int gate_n, cudaStream_t s) {
   ProfScope prof(PK_SOAP_QR, s);
   dim3 grid((cols + 31) / 32, count);
-  colnorm2_kernel<<<grid, 256, 0, s>>>(Y, ld, mat_stride, rows, cols, inv_d, skip);
+  (void)launch_pdl(colnorm2_kernel, grid, dim3(256), 0, s, false, Y, ld, mat_stride, rows, cols, inv_d, skip, gate,
+                   gate_n);
 }
 
 void launch_qr_control(const float* C, long long ld, long long mat_stride, int q, int kp, const QrCtl& c,
-                       cudaStream_t s) {
+                       int pass, const int* gate, cudaStream_t s) {
   ProfScope prof(PK_SOAP_QR, s);
-  qr_check_kernel<<<dim3(QR_CHECK_BLOCKS, q), 256, 0, s>>>(C, ld, mat_stride, kp, c);
-  qr_decide_kernel<<<q, 256, 0, s>>>(const_cast<float*>(C), ld, mat_stride, kp, c);
+  (void)launch_pdl(qr_check_kernel, dim3(QR_CHECK_BLOCKS, q), dim3(256), 0, s, false, C, ld, mat_stride, kp, c, gate,
+                   q);
+  (void)launch_pdl(qr_decide_kernel, dim3(q), dim3(256), 0, s, false, const_cast<float*>(C), ld, mat_stride, kp, c,
+                   pass);
 }
 
 void launch_qr_chol(const float* C, long long ld, long long mat_stride, int q, int j, float* Dinv,
-                    const QrCtl& c, cudaStream_t s) {
+                    const QrCtl& c, const int* gate, cudaStream_t s) {
   ProfScope prof(PK_QR_CHOL, s);
   const int smem = (2 * CB * CB_LD + 32 * CB_T_LD + CB) * 4;
   (void)ensure_smem_attr(reinterpret_cast<const void*>(qr_chol_kernel), smem);
-  qr_chol_kernel<<<q, 256, smem, s>>>(C, ld, mat_stride, j * QR_B, Dinv, c);
+  (void)launch_pdl(qr_chol_kernel, dim3(q), dim3(256), (size_t)smem, s, false, C, ld, mat_stride, j * QR_B, Dinv, c,
+                   gate, q);
 }
 
 void launch_qr_panel(const PanelArgs& a, cudaStream_t s) {
@@ -511,7 +544,7 @@ void launch_qr_panel(const PanelArgs& a, cudaStream_t s) {
   ProfScope prof(PK_QR_ROWBLK, s);
   (void)ensure_smem_attr(reinterpret_cast<const void*>(qr_panel_kernel), PANEL_SMEM);
   dim3 grid((a.r1 - a.r0 + PANEL_ROWS - 1) / PANEL_ROWS, a.q);
-  qr_panel_kernel<<<grid, 256, PANEL_SMEM, s>>>(a);
+  (void)launch_pdl(qr_panel_kernel, grid, dim3(256), (size_t)PANEL_SMEM, s, false, a);
 }
 
 void launch_qr_finish(const QrCtl& c, const FlagTable& flags, int q, float* Y, long long ld,

@@ -73,6 +73,7 @@ struct QrCtl {
   float* part;          // [q][QR_CHECK_BLOCKS] partial sums of C_ij^2
   float* fscale;        // power step: scale 2^e of the factor's planes
   float* fiscale;       // and its inverse
+  int* pass_done;       // [QR_MAX_PASSES]: matrices done after pass p's decision
 };
 
 // Bytes of the control arrays for q matrices (1024-byte aligned pieces).
@@ -120,6 +121,8 @@ struct Split16Args {
   const int* noise_on = nullptr;
   float noise_amp = 0.f;
   unsigned noise_seed = 0u;
+  const int* gate = nullptr;          // launch gate (see launch_qr_control)
+  int gate_n = 0;
 };
 // The padded diagonal (pad_identity) is written as min(scale, 2^14) in the
 // planes, whatever the scale, so that it never overflows fp16; write_back
@@ -129,13 +132,21 @@ void launch_split16(const Split16Args& a, cudaStream_t s);
 // inv_d[b][c] = 1 / ||Y[b][:, c]|| (0 for a zero column, NaN for an
 // infinite norm) over the first `rows` rows; skips matrices with skip[b].
 void launch_colnorm2(const float* Y, long long ld, long long mat_stride, int count, int rows, int cols,
-                     float* inv_d, const int* skip, cudaStream_t s);
+                     float* inv_d, const int* skip, const int* gate, int gate_n, cudaStream_t s);
 
+// Launch gate (optional, device): the launch does nothing when *gate >=
+// gate_n (every matrix of the refresh already done).  The refresh kernels
+// launch with programmatic stream serialization: each waits for its
+// predecessor before its first global access, so a gated-off pass costs a
+// few microseconds per launch.
+// pass_done[pass] counts the matrices done after this pass's decision: the
+// gate of this pass's block steps and of the next pass's launches.
+//
 // The Gram check and the pass decision: max |C - I| and sum C^2 of each kp x
-// kp Gram (fixed-order partial sums), then per matrix the decision above,
-// with the shift added to C's diagonal.
+// kp Gram (fixed-order partial sums; the check is gated by `gate`), then per
+// matrix the decision above, with the shift added to C's diagonal.
 void launch_qr_control(const float* C, long long ld, long long mat_stride, int q, int kp, const QrCtl& c,
-                       cudaStream_t s);
+                       int pass, const int* gate, cudaStream_t s);
 
 // Diagonal block j of each matrix's Cholesky factor: C[b] + (128 j)(ld + 1)
 // holds the 128 x 128 Schur complement block; factor it with the matrix's
@@ -143,7 +154,7 @@ void launch_qr_control(const float* C, long long ld, long long mat_stride, int q
 // lower factor, transposed (an upper-triangular 128 x 128 matrix), to
 // Dinv[b].  A pivot at or below the floor sets fail[b] and skip[b].
 void launch_qr_chol(const float* C, long long ld, long long mat_stride, int q, int j, float* Dinv,
-                    const QrCtl& c, cudaStream_t s);
+                    const QrCtl& c, const int* gate, cudaStream_t s);
 
 // Rows [r0, r1) of each matrix's stacked [C; Y] (row stride ld), block
 // column j: x = row * Dinv^T (128 wide).  Its fp16 planes (scale
@@ -155,6 +166,7 @@ struct PanelArgs {
   const float* Dinv;
   __half* LQ; long long plane_stride;     // planes: same ld and mat_stride as CY
   const int* skip;
+  const int* gate = nullptr;              // launch gate: nothing when *gate >= q
 };
 void launch_qr_panel(const PanelArgs& a, cudaStream_t s);
 

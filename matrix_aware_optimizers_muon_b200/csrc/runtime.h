@@ -128,6 +128,10 @@ struct GemmOp {
   const int* skip = nullptr;
   // A and B hold fp16 values (both; the MMA takes one type for the two)
   int ab_f16 = 0;
+  // optional launch gate (device): the whole launch does nothing when
+  // *gate >= gate_n (every matrix of a refresh pass already done)
+  const int* gate = nullptr;
+  int gate_n = 0;
 };
 
 // Launch the tcgen05 GEMM.  Returns cudaSuccess or the launch/encode error.

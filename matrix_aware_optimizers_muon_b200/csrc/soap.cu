@@ -372,9 +372,14 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
 
       const int nb = (int)(kp / QR_B);
       for (int pass = 0; pass < QR_MAX_PASSES; ++pass) {
+        // launch gates: a pass whose matrices were all done by the previous
+        // pass's decision, and block steps after this pass's decision found
+        // them all done, take no part (decided on the device)
+        const int* gate_in = pass > 0 ? ctl.pass_done + (pass - 1) : nullptr;
+        const int* gate_steps = ctl.pass_done + pass;
         // normalise Y's columns (a zero column becomes e_c), planes of the
         // result into the Q part of [L; Q], C = Y^T Y into the C part
-        launch_colnorm2(CY + kk, kp, ms, q, (int)kp, (int)kp, invd, ctl.done, s);
+        launch_colnorm2(CY + kk, kp, ms, q, (int)kp, (int)kp, invd, ctl.done, gate_in, q, s);
         Split16Args sy;
         sy.count = q; sy.rows_valid = sy.cols_valid = sy.rows_pad = sy.cols_pad = (int)kp;
         for (int j = 0; j < q; ++j) sy.src[j] = CY + (size_t)j * ms + kk;
@@ -385,6 +390,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
         sy.noise_on = ctl.fail;                  // set by a failed attempt of the previous pass
         sy.noise_amp = QR_NOISE;
         sy.noise_seed = (unsigned)pass;
+        sy.gate = gate_in; sy.gate_n = q;
         launch_split16(sy, s);
         {
           GemmOp g;
@@ -397,10 +403,11 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
           g.D = CY; g.ldd = kp; g.strideD = ms; g.d_f32 = 1;
           g.kind = PK_SOAP_QR;
           g.skip = ctl.done;
+          g.gate = gate_in; g.gate_n = q;
           if ((e = launch_gemm(g, status, s)) != cudaSuccess) return e;
         }
         // done / plain / shifted per matrix, the shift on C's diagonal
-        launch_qr_control(CY, kp, ms, q, (int)kp, ctl, s);
+        launch_qr_control(CY, kp, ms, q, (int)kp, ctl, pass, gate_in, s);
         for (int j = 0; j < nb; ++j) {
           const long long r0 = (long long)j * QR_B;
           if (j > 0) {     // [C; Y][r0 :, j] -= [L; Q][r0 :, < j] L[j, < j]^T
@@ -415,13 +422,15 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
             t.D = CY + r0 * kp + r0; t.ldd = kp; t.strideD = ms; t.d_f32 = 1;
             t.kind = PK_QR_TRAIL;
             t.skip = ctl.skip;
+            t.gate = gate_steps; t.gate_n = q;
             if ((e = launch_gemm(t, status, s)) != cudaSuccess) return e;
           }
-          launch_qr_chol(CY, kp, ms, q, j, Dinv, ctl, s);
+          launch_qr_chol(CY, kp, ms, q, j, Dinv, ctl, gate_steps, s);
           PanelArgs pa;
           pa.q = q; pa.j = j; pa.r0 = (int)(r0 + QR_B); pa.r1 = (int)(2 * kp); pa.f32_from = (int)kp;
           pa.CY = CY; pa.ld = kp; pa.mat_stride = ms; pa.Dinv = Dinv;
           pa.LQ = LQ; pa.plane_stride = pst; pa.skip = ctl.skip;
+          pa.gate = gate_steps;
           launch_qr_panel(pa, s);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -82,9 +82,10 @@ struct GemmParams {
   float ap_step[2];
   int ap_tall_from;
   int ap_vec;               // every W of the launch: 16-byte aligned rows
-  // launch gate: no tiles when *gate >= gate_n
+  // launch gate: nothing when gate[gate_idx ? *gate_idx : 0] >= gate_n
   const int* gate;
   int gate_n;
+  const int* gate_idx;
   // A and B hold fp16 (not bf16) values: the same kind::f16 MMA with the
   // operand type fields of the instruction descriptor set to f16
   int ab_f16;
@@ -537,7 +538,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   // closed, leaves before any setup; the whole grid reads the same word
   if (p.gate != nullptr) {
     pdl_wait();
-    if (*p.gate >= p.gate_n) return;
+    if (p.gate[p.gate_idx ? *p.gate_idx : 0] >= p.gate_n) return;
   }
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

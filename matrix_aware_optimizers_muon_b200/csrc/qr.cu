@@ -29,8 +29,10 @@ __global__ void qr_init_kernel(const QrCtl c, int q) {
   c.shift[b] = 0.f;
   c.minpiv[b] = 0x7f800000u;
   c.dev[b] = 0u;
-  if (b == 0)
+  if (b == 0) {
     for (int p = 0; p < QR_MAX_PASSES; ++p) c.pass_done[p] = 0;
+    *c.npass = 0;
+  }
 }
 
 // One CTA per matrix: the largest diagonal entry, then a power-of-two scale
@@ -95,7 +97,7 @@ __device__ __forceinline__ float hash_uniform(unsigned b, unsigned r, unsigned c
   return (float)(h >> 8) * (2.0f / 16777216.0f) - 1.0f;
 }
 
-__device__ __forceinline__ void split16_row(const Split16Args& a, int b, int r, int c0) {
+__device__ __forceinline__ void split16_row(const Split16Args& a, int b, int r, int c0, unsigned seed) {
   const bool rv = r < a.rows_valid;
   const float* src = a.src[b] + (long long)r * a.lds;
   float x[8];
@@ -121,7 +123,7 @@ __device__ __forceinline__ void split16_row(const Split16Args& a, int b, int r, 
         const float s = a.col_scale[(size_t)b * a.cols_pad + c];
         x[i] = s == 0.f ? (r == c ? 1.f : 0.f) : x[i] * s;     // a zero column becomes e_c
       }
-      if (noisy) x[i] = fmaf(namp, hash_uniform(b, r, c, a.noise_seed), x[i]);
+      if (noisy) x[i] = fmaf(namp, hash_uniform(b, r, c, seed), x[i]);
     } else {
       pad[i] = a.pad_identity && r == c;
       x[i] = pad[i] ? 1.f : 0.f;
@@ -147,7 +149,8 @@ __global__ void split16_kernel(const Split16Args a) {
   if (a.skip && a.skip[b]) return;
   const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (c0 >= a.cols_pad) return;
-  for (int r = blockIdx.y; r < a.rows_pad; r += gridDim.y) split16_row(a, b, r, c0);
+  const unsigned seed = a.seed_dev ? (unsigned)*a.seed_dev : a.noise_seed;
+  for (int r = blockIdx.y; r < a.rows_pad; r += gridDim.y) split16_row(a, b, r, c0, seed);
 }
 
 // 32 columns x 8 row groups per CTA; the 8 partial sums of a column are
@@ -232,10 +235,11 @@ __global__ void __launch_bounds__(256) qr_check_kernel(const float* C, long long
 // One CTA per matrix: the outcome of the previous attempt, the check of this
 // pass's Gram, the mode of this pass, and the shift of the diagonal.
 __global__ void __launch_bounds__(256) qr_decide_kernel(float* C, long long ld, long long stride, int kp,
-                                                        const QrCtl c, int pass) {
+                                                        const QrCtl c, int pass_host, const int* pass_dev) {
   __shared__ float s_shift;
   pdl_wait();
   pdl_trigger();
+  const int pass = pass_dev ? *pass_dev : pass_host;
   const int b = blockIdx.x;
   if (threadIdx.x == 0) {
     float sh = 0.f;
@@ -289,10 +293,11 @@ __global__ void __launch_bounds__(256) qr_decide_kernel(float* C, long long ld, 
 // One CTA (256 threads) per matrix: Cholesky of the diagonal block with the
 // matrix's pivot floor, then the inverse of its lower factor.
 __global__ void __launch_bounds__(256) qr_chol_kernel(const float* C, long long ld, long long stride, int k0,
-                                                      float* Dinv, const QrCtl c, const int* gate, int gate_n) {
+                                                      float* Dinv, const QrCtl c, const int* gate,
+                                                      const int* gate_idx, int gate_n) {
   pdl_wait();
   pdl_trigger();
-  if (gate && *gate >= gate_n) return;
+  if (gate && gate[gate_idx ? *gate_idx : 0] >= gate_n) return;
   const int b = blockIdx.x;
   if (c.skip[b]) return;
   extern __shared__ float sm[];
@@ -363,7 +368,7 @@ constexpr int PANEL_SMEM = (QR_B * PANEL_LDD + QR_B * PANEL_LDR) * 4;
 __global__ void __launch_bounds__(256, 1) qr_panel_kernel(const PanelArgs a) {
   pdl_wait();
   pdl_trigger();
-  if (a.gate && *a.gate >= a.q) return;
+  if (a.gate && a.gate[a.gate_idx ? *a.gate_idx : 0] >= a.q) return;
   const int b = blockIdx.y;
   if (a.skip[b]) return;
   extern __shared__ float sm[];
@@ -445,6 +450,14 @@ __global__ void __launch_bounds__(256, 1) qr_panel_kernel(const PanelArgs a) {
   }
 }
 
+__global__ void qr_loop_kernel(const QrCtl c, int q, cudaGraphConditionalHandle h) {
+  pdl_wait();
+  const int p = *c.npass;
+  const bool more = c.pass_done[p] < q && p + 1 < QR_MAX_PASSES;
+  *c.npass = p + 1;
+  cudaGraphSetConditional(h, more ? 1u : 0u);
+}
+
 __global__ void qr_finish_flags_kernel(const QrCtl c, const FlagTable f, int q) {
   const int b = threadIdx.x;
   if (b < q && !c.done[b] && f.f[b] != nullptr) *f.f[b] = 1;
@@ -488,7 +501,8 @@ QrCtl qr_ctl_at(char* base, int q) {
   c.dev = reinterpret_cast<unsigned*>(base + 9 * w);
   c.fscale = reinterpret_cast<float*>(base + 10 * w);
   c.fiscale = reinterpret_cast<float*>(base + 11 * w);
-  c.pass_done = reinterpret_cast<int*>(base + 12 * w);     // QR_MAX_PASSES <= 256 words
+  c.pass_done = reinterpret_cast<int*>(base + 12 * w);     // QR_MAX_PASSES + 1 <= 256 words
+  c.npass = c.pass_done + QR_MAX_PASSES;
   c.part = reinterpret_cast<float*>(base + 13 * w);
   return c;
 }
@@ -522,21 +536,21 @@ void launch_colnorm2(const float* Y, long long ld, long long mat_stride, int cou
 }
 
 void launch_qr_control(const float* C, long long ld, long long mat_stride, int q, int kp, const QrCtl& c,
-                       int pass, const int* gate, cudaStream_t s) {
+                       int pass, const int* pass_dev, const int* gate, cudaStream_t s) {
   ProfScope prof(PK_SOAP_QR, s);
   (void)launch_pdl(qr_check_kernel, dim3(QR_CHECK_BLOCKS, q), dim3(256), 0, s, false, C, ld, mat_stride, kp, c, gate,
                    q);
   (void)launch_pdl(qr_decide_kernel, dim3(q), dim3(256), 0, s, false, const_cast<float*>(C), ld, mat_stride, kp, c,
-                   pass);
+                   pass, pass_dev);
 }
 
 void launch_qr_chol(const float* C, long long ld, long long mat_stride, int q, int j, float* Dinv,
-                    const QrCtl& c, const int* gate, cudaStream_t s) {
+                    const QrCtl& c, const int* gate, const int* gate_idx, cudaStream_t s) {
   ProfScope prof(PK_QR_CHOL, s);
   const int smem = (2 * CB * CB_LD + 32 * CB_T_LD + CB) * 4;
   (void)ensure_smem_attr(reinterpret_cast<const void*>(qr_chol_kernel), smem);
   (void)launch_pdl(qr_chol_kernel, dim3(q), dim3(256), (size_t)smem, s, false, C, ld, mat_stride, j * QR_B, Dinv, c,
-                   gate, q);
+                   gate, gate_idx, q);
 }
 
 void launch_qr_panel(const PanelArgs& a, cudaStream_t s) {
@@ -545,6 +559,11 @@ void launch_qr_panel(const PanelArgs& a, cudaStream_t s) {
   (void)ensure_smem_attr(reinterpret_cast<const void*>(qr_panel_kernel), PANEL_SMEM);
   dim3 grid((a.r1 - a.r0 + PANEL_ROWS - 1) / PANEL_ROWS, a.q);
   (void)launch_pdl(qr_panel_kernel, grid, dim3(256), (size_t)PANEL_SMEM, s, false, a);
+}
+
+void launch_qr_loop(const QrCtl& c, int q, cudaGraphConditionalHandle h, cudaStream_t s) {
+  ProfScope prof(PK_SOAP_QR, s);
+  (void)launch_pdl(qr_loop_kernel, dim3(1), dim3(1), 0, s, false, c, q, h);
 }
 
 void launch_qr_finish(const QrCtl& c, const FlagTable& flags, int q, float* Y, long long ld,

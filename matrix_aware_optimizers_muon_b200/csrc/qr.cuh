@@ -74,6 +74,7 @@ struct QrCtl {
   float* fscale;        // power step: scale 2^e of the factor's planes
   float* fiscale;       // and its inverse
   int* pass_done;       // [QR_MAX_PASSES]: matrices done after pass p's decision
+  int* npass;           // passes run so far (the pass loop recorded as a graph reads it)
 };
 
 // Bytes of the control arrays for q matrices (1024-byte aligned pieces).
@@ -123,6 +124,7 @@ struct Split16Args {
   unsigned noise_seed = 0u;
   const int* gate = nullptr;          // launch gate (see launch_qr_control)
   int gate_n = 0;
+  const int* seed_dev = nullptr;      // optional: the noise seed read from device memory
 };
 // The padded diagonal (pad_identity) is written as min(scale, 2^14) in the
 // planes, whatever the scale, so that it never overflows fp16; write_back
@@ -145,8 +147,14 @@ void launch_colnorm2(const float* Y, long long ld, long long mat_stride, int cou
 // The Gram check and the pass decision: max |C - I| and sum C^2 of each kp x
 // kp Gram (fixed-order partial sums; the check is gated by `gate`), then per
 // matrix the decision above, with the shift added to C's diagonal.
+// `pass_dev` (optional) replaces `pass` by a device word.
 void launch_qr_control(const float* C, long long ld, long long mat_stride, int q, int kp, const QrCtl& c,
-                       int pass, const int* gate, cudaStream_t s);
+                       int pass, const int* pass_dev, const int* gate, cudaStream_t s);
+
+// End of one pass of the pass loop recorded as a graph (a conditional while
+// node): npass += 1, and the loop goes on while a matrix is not done and
+// fewer than QR_MAX_PASSES passes have run.
+void launch_qr_loop(const QrCtl& c, int q, cudaGraphConditionalHandle h, cudaStream_t s);
 
 // Diagonal block j of each matrix's Cholesky factor: C[b] + (128 j)(ld + 1)
 // holds the 128 x 128 Schur complement block; factor it with the matrix's
@@ -154,7 +162,7 @@ void launch_qr_control(const float* C, long long ld, long long mat_stride, int q
 // lower factor, transposed (an upper-triangular 128 x 128 matrix), to
 // Dinv[b].  A pivot at or below the floor sets fail[b] and skip[b].
 void launch_qr_chol(const float* C, long long ld, long long mat_stride, int q, int j, float* Dinv,
-                    const QrCtl& c, const int* gate, cudaStream_t s);
+                    const QrCtl& c, const int* gate, const int* gate_idx, cudaStream_t s);
 
 // Rows [r0, r1) of each matrix's stacked [C; Y] (row stride ld), block
 // column j: x = row * Dinv^T (128 wide).  Its fp16 planes (scale
@@ -166,7 +174,8 @@ struct PanelArgs {
   const float* Dinv;
   __half* LQ; long long plane_stride;     // planes: same ld and mat_stride as CY
   const int* skip;
-  const int* gate = nullptr;              // launch gate: nothing when *gate >= q
+  const int* gate = nullptr;              // launch gate: nothing when gate[gate_idx ? *gate_idx : 0] >= q
+  const int* gate_idx = nullptr;
 };
 void launch_qr_panel(const PanelArgs& a, cudaStream_t s);
 

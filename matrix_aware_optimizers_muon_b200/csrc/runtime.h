@@ -46,9 +46,18 @@ cudaError_t ensure_smem_attr(const void* func, int bytes);
 // Launch `kern` with programmatic stream serialization (and, with cluster2,
 // clusters of two CTAs): it may start while the previous kernel of the
 // stream runs, so it must call pdl_wait() before touching global memory.
+// Per host thread: launches made by launch_pdl leave out programmatic
+// stream serialization while set (graph bodies recorded by the library).
+inline bool& pdl_off() {
+  static thread_local bool off = false;
+  return off;
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                        bool cluster2, Args&&... args) {
+  // programmatic serialization unless this thread is recording a graph body
+  // that must hold plain kernel nodes (pdl_off())
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -56,9 +65,11 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   int n = 0;
-  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[n].val.programmaticStreamSerializationAllowed = 1;
-  ++n;
+  if (!pdl_off()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
   if (cluster2) {
     attr[n].id = cudaLaunchAttributeClusterDimension;
     attr[n].val.clusterDim.x = 2;
@@ -132,6 +143,7 @@ struct GemmOp {
   // *gate >= gate_n (every matrix of a refresh pass already done)
   const int* gate = nullptr;
   int gate_n = 0;
+  const int* gate_idx = nullptr;     // optional device index: the gate word is gate[*gate_idx]
 };
 
 // Launch the tcgen05 GEMM.  Returns cudaSuccess or the launch/encode error.

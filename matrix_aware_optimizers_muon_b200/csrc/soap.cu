@@ -20,7 +20,9 @@
 #include <algorithm>
 #include <cmath>
 #include <map>
+#include <mutex>
 #include <tuple>
+#include <vector>
 
 #include "ns_plan.h"
 #include "profile.h"
@@ -35,6 +37,88 @@ namespace {
 
 constexpr size_t AL = 1024;
 size_t al(size_t x) { return (x + AL - 1) / AL * AL; }
+
+// The refresh's pass loop as a CUDA graph: a conditional while node whose
+// body is one pass ending in launch_qr_loop, so that only the passes a step
+// needs are executed (a warm step needs two of the eight allowed).  One
+// instantiated graph per (device, workspace, bucket layout), kept while the
+// same workspace and shapes come back; its kernels hold workspace pointers
+// only.
+struct PassGraph {
+  int dev = -1;
+  const char* ws = nullptr;
+  size_t cy = 0, lq = 0, dinv = 0, invd = 0, ctl = 0;
+  int q = 0;
+  long long kp = 0, k = 0;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+};
+std::mutex g_pass_graph_mu;
+std::vector<PassGraph> g_pass_graphs;                  // most recent last, at most 16
+constexpr size_t PASS_GRAPH_KEEP = 16;
+
+cudaStream_t pass_capture_stream(int dev) {
+  static cudaStream_t streams[64] = {};
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (streams[dev] == nullptr && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) {
+    streams[dev] = nullptr;
+    (void)cudaGetLastError();
+  }
+  return streams[dev];
+}
+
+// Launches the pass-loop graph of `key` on s, recording it first with
+// `record(stream, handle)` when it is not cached.  Returns false (nothing
+// launched, errors cleared) when a graph cannot be made, so that the caller
+// launches the passes directly.
+template <class Record>
+bool launch_pass_graph(PassGraph key, Record&& record, cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(g_pass_graph_mu);
+  for (size_t i = 0; i < g_pass_graphs.size(); ++i) {
+    const PassGraph& g = g_pass_graphs[i];
+    if (g.dev == key.dev && g.ws == key.ws && g.cy == key.cy && g.lq == key.lq && g.dinv == key.dinv &&
+        g.invd == key.invd && g.ctl == key.ctl && g.q == key.q && g.kp == key.kp && g.k == key.k)
+      return cudaGraphLaunch(g.exec, s) == cudaSuccess || ((void)cudaGetLastError(), false);
+  }
+  cudaStream_t cs = pass_capture_stream(key.dev);
+  if (cs == nullptr) return false;
+  cudaGraph_t graph = nullptr;
+  if (cudaGraphCreate(&graph, 0) != cudaSuccess) return (void)cudaGetLastError(), false;
+  auto give_up = [&]() {
+    cudaGraphDestroy(graph);
+    (void)cudaGetLastError();
+    return false;
+  };
+  cudaGraphConditionalHandle h;
+  if (cudaGraphConditionalHandleCreate(&h, graph, 1u, cudaGraphCondAssignDefault) != cudaSuccess) return give_up();
+  cudaGraphNodeParams np = {};
+  np.type = cudaGraphNodeTypeConditional;
+  np.conditional.handle = h;
+  np.conditional.type = cudaGraphCondTypeWhile;
+  np.conditional.size = 1;
+  cudaGraphNode_t node;
+  if (cudaGraphAddNode(&node, graph, nullptr, 0, &np) != cudaSuccess) return give_up();
+  cudaGraph_t body = np.conditional.phGraph_out[0];
+  if (cudaStreamBeginCaptureToGraph(cs, body, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+    return give_up();
+  pdl_off() = true;
+  const cudaError_t er = record(cs, h);
+  pdl_off() = false;
+  cudaGraph_t captured = nullptr;
+  const cudaError_t ec = cudaStreamEndCapture(cs, &captured);
+  if (er != cudaSuccess || ec != cudaSuccess) return give_up();
+  cudaGraphExec_t exec = nullptr;
+  if (cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) return give_up();
+  key.graph = graph;
+  key.exec = exec;
+  if (g_pass_graphs.size() >= PASS_GRAPH_KEEP) {
+    cudaGraphExecDestroy(g_pass_graphs.front().exec);
+    cudaGraphDestroy(g_pass_graphs.front().graph);
+    g_pass_graphs.erase(g_pass_graphs.begin());
+  }
+  g_pass_graphs.push_back(key);
+  return cudaGraphLaunch(exec, s) == cudaSuccess || ((void)cudaGetLastError(), false);
+}
 
 // two-plane products: x = h + l, x y ~ lh + hl + hh (bf16 planes for the
 // rotations, fp16 planes with ab_f16 for the refresh).  The small products
@@ -371,15 +455,19 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
       }
 
       const int nb = (int)(kp / QR_B);
-      for (int pass = 0; pass < QR_MAX_PASSES; ++pass) {
-        // launch gates: a pass whose matrices were all done by the previous
-        // pass's decision, and block steps after this pass's decision found
-        // them all done, take no part (decided on the device)
-        const int* gate_in = pass > 0 ? ctl.pass_done + (pass - 1) : nullptr;
-        const int* gate_steps = ctl.pass_done + pass;
+      // One CholeskyQR pass.  Launched directly (pass >= 0), later launches
+      // are gated on the device by the matrices done after the previous
+      // pass's decision; recorded into the pass-loop graph (pass < 0), the
+      // pass index is the device word ctl.npass and the loop itself stops.
+      auto enqueue_pass = [&](int pass, cudaStream_t st) -> cudaError_t {
+        const bool graph = pass < 0;
+        const int* gate_in = (!graph && pass > 0) ? ctl.pass_done + (pass - 1) : nullptr;
+        const int* gate_steps = graph ? ctl.pass_done : ctl.pass_done + pass;
+        const int* gate_idx = graph ? ctl.npass : nullptr;
+        cudaError_t er;
         // normalise Y's columns (a zero column becomes e_c), planes of the
         // result into the Q part of [L; Q], C = Y^T Y into the C part
-        launch_colnorm2(CY + kk, kp, ms, q, (int)kp, (int)kp, invd, ctl.done, gate_in, q, s);
+        launch_colnorm2(CY + kk, kp, ms, q, (int)kp, (int)kp, invd, ctl.done, gate_in, q, st);
         Split16Args sy;
         sy.count = q; sy.rows_valid = sy.cols_valid = sy.rows_pad = sy.cols_pad = (int)kp;
         for (int j = 0; j < q; ++j) sy.src[j] = CY + (size_t)j * ms + kk;
@@ -389,9 +477,10 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
         sy.skip = ctl.done;
         sy.noise_on = ctl.fail;                  // set by a failed attempt of the previous pass
         sy.noise_amp = QR_NOISE;
-        sy.noise_seed = (unsigned)pass;
+        sy.noise_seed = graph ? 0u : (unsigned)pass;
+        sy.seed_dev = graph ? ctl.npass : nullptr;
         sy.gate = gate_in; sy.gate_n = q;
-        launch_split16(sy, s);
+        launch_split16(sy, st);
         {
           GemmOp g;
           g.A = LQ + kk; g.lda = kp; g.strideA = ms; g.a_mn = 1;
@@ -404,10 +493,10 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
           g.kind = PK_SOAP_QR;
           g.skip = ctl.done;
           g.gate = gate_in; g.gate_n = q;
-          if ((e = launch_gemm(g, status, s)) != cudaSuccess) return e;
+          if ((er = launch_gemm(g, status, st)) != cudaSuccess) return er;
         }
         // done / plain / shifted per matrix, the shift on C's diagonal
-        launch_qr_control(CY, kp, ms, q, (int)kp, ctl, pass, gate_in, s);
+        launch_qr_control(CY, kp, ms, q, (int)kp, ctl, graph ? 0 : pass, graph ? ctl.npass : nullptr, gate_in, st);
         for (int j = 0; j < nb; ++j) {
           const long long r0 = (long long)j * QR_B;
           if (j > 0) {     // [C; Y][r0 :, j] -= [L; Q][r0 :, < j] L[j, < j]^T
@@ -422,19 +511,43 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
             t.D = CY + r0 * kp + r0; t.ldd = kp; t.strideD = ms; t.d_f32 = 1;
             t.kind = PK_QR_TRAIL;
             t.skip = ctl.skip;
-            t.gate = gate_steps; t.gate_n = q;
-            if ((e = launch_gemm(t, status, s)) != cudaSuccess) return e;
+            t.gate = gate_steps; t.gate_n = q; t.gate_idx = gate_idx;
+            if ((er = launch_gemm(t, status, st)) != cudaSuccess) return er;
           }
-          launch_qr_chol(CY, kp, ms, q, j, Dinv, ctl, gate_steps, s);
+          launch_qr_chol(CY, kp, ms, q, j, Dinv, ctl, gate_steps, gate_idx, st);
           PanelArgs pa;
           pa.q = q; pa.j = j; pa.r0 = (int)(r0 + QR_B); pa.r1 = (int)(2 * kp); pa.f32_from = (int)kp;
           pa.CY = CY; pa.ld = kp; pa.mat_stride = ms; pa.Dinv = Dinv;
           pa.LQ = LQ; pa.plane_stride = pst; pa.skip = ctl.skip;
-          pa.gate = gate_steps;
-          launch_qr_panel(pa, s);
+          pa.gate = gate_steps; pa.gate_idx = gate_idx;
+          launch_qr_panel(pa, st);
         }
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        return cudaGetLastError();
+      };
+      // the graph holds no event brackets: with profiling on, or inside a
+      // caller's capture, the passes are launched directly
+      cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+      const bool direct_passes = g_prof != nullptr || cudaStreamIsCapturing(s, &cap) != cudaSuccess ||
+                                 cap != cudaStreamCaptureStatusNone;
+      bool in_graph = false;
+      if (!direct_passes) {
+        PassGraph key;
+        (void)cudaGetDevice(&key.dev);
+        key.ws = ws; key.cy = bk.cy; key.lq = bk.lq; key.dinv = bk.dinv; key.invd = bk.invd; key.ctl = bk.ctl;
+        key.q = q; key.kp = kp; key.k = k;
+        in_graph = launch_pass_graph(
+            key,
+            [&](cudaStream_t cs, cudaGraphConditionalHandle h) -> cudaError_t {
+              cudaError_t er = enqueue_pass(-1, cs);
+              if (er != cudaSuccess) return er;
+              launch_qr_loop(ctl, q, h, cs);
+              return cudaGetLastError();
+            },
+            s);
       }
+      if (!in_graph)
+        for (int pass = 0; pass < QR_MAX_PASSES; ++pass)
+          if ((e = enqueue_pass(pass, s)) != cudaSuccess) return e;
       {
         const float* qold[SOAP_MAXB];
         for (int j = 0; j < q; ++j) qold[j] = basis_of(j);

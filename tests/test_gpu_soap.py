@@ -331,3 +331,33 @@ def test_nonfinite_gradient_flags_and_propagates(ctx):
     for fac, q in (("L", "QL"), ("R", "QR")):
         basis_gate(out[q], emu[fac], S[q])
     assert np.isfinite(out["W"]).all()
+
+
+def test_pass_loop_graph_equals_direct_launches(ctx):
+    """The refresh's pass loop runs as a graph with a conditional while node
+    in eager calls, and as directly launched gated passes under profiling (or
+    a caller's stream capture): the same kernels in the same order, so every
+    output is bit-equal, including a cold start that needs several passes."""
+    import torch
+    for steps, (m, n, left, right) in ((0, (96, 160, True, True)), (6, (128, 96, True, False))):
+        if steps == 0:
+            st = wl.SpikeStream("graph-vs-direct", "warm", 1, m, n, wl.CFG4_MINI)
+            S = dict(W=st.W.astype(np.float32), M=np.zeros((m, n), np.float32), V=np.zeros((m, n), np.float32),
+                     L=np.zeros((m, m), np.float32), QL=np.eye(m, dtype=np.float32),
+                     R=np.zeros((n, n), np.float32), QR=np.eye(n, dtype=np.float32))
+            G, t = st.next(), 1
+        else:
+            S, G, t = warm_state(m, n, left, right, steps, "graph-vs-direct")
+        outs = []
+        for prof in (False, True):
+            ctx.profile(prof)
+            try:
+                flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+                outs.append((run_gpu(ctx, S, G, t, flags=flags), int(flags.item())))
+            finally:
+                ctx.profile(False)
+        (a, fa), (b, fb) = outs
+        assert fa == fb
+        for k in a:
+            if a[k] is not None:
+                np.testing.assert_array_equal(a[k], b[k], err_msg=k)

@@ -77,8 +77,13 @@ bool launch_pass_graph(PassGraph key, Record&& record, cudaStream_t s) {
   for (size_t i = 0; i < g_pass_graphs.size(); ++i) {
     const PassGraph& g = g_pass_graphs[i];
     if (g.dev == key.dev && g.ws == key.ws && g.cy == key.cy && g.lq == key.lq && g.dinv == key.dinv &&
-        g.invd == key.invd && g.ctl == key.ctl && g.q == key.q && g.kp == key.kp && g.k == key.k)
-      return cudaGraphLaunch(g.exec, s) == cudaSuccess || ((void)cudaGetLastError(), false);
+        g.invd == key.invd && g.ctl == key.ctl && g.q == key.q && g.kp == key.kp && g.k == key.k) {
+      if (cudaGraphLaunch(g.exec, s) == cudaSuccess) return true;
+      // a graph that no longer launches (its context was reset) is dropped
+      (void)cudaGetLastError();
+      g_pass_graphs.erase(g_pass_graphs.begin() + (long)i);
+      return false;
+    }
   }
   cudaStream_t cs = pass_capture_stream(key.dev);
   if (cs == nullptr) return false;

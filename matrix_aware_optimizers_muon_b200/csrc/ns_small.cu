@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(SM_THREADS, 3) ns_small_kernel(const SmallArgs
       ok = workers_all(ok);
       if (ok) {
         float* out = a.out[mat];
-        if constexpr (BULK) {
+        if (BULK && a.mode == 1) {
           // rounds of 32 KB: fp32 O (or, in Muon mode, W <- decay W - step O
           // on W brought in by a bulk load) staged in A, then one bulk store
           float4* st4 = reinterpret_cast<float4*>(A);

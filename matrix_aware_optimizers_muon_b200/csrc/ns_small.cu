@@ -167,7 +167,42 @@ __global__ void __launch_bounds__(SM_THREADS, 3) ns_small_kernel(const SmallArgs
       float* B = a.mom ? a.mom[mat] : nullptr;
       const int total = a.rows * a.cols;
       float ss = 0.f;
-      if constexpr (BULK) {
+      if (BULK && a.mode == 0) {
+        // plain NS: 16 float4 loads in flight per thread, straight into
+        // registers (no staging traffic in the shared memory the SM's CTAs
+        // share): two rounds for a 128 x 128 matrix
+        constexpr int RU = 16;
+        const float4* G4 = reinterpret_cast<const float4*>(G);
+        const int total4 = total >> 2;
+        for (int e0 = tid; e0 < total4; e0 += 128 * RU) {
+          float4 g[RU];
+#pragma unroll
+          for (int u = 0; u < RU; ++u) {
+            const int e = e0 + u * 128;
+            g[u] = e < total4 ? __ldg(G4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < RU; ++u) {
+            const int e4 = e0 + u * 128;
+            if (e4 >= total4) break;
+            const float nv[4] = {g[u].x, g[u].y, g[u].z, g[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) ss = fmaf(nv[j], nv[j], ss);
+            const int e = 4 * e4;
+            const int r = (int)__umulhi((uint32_t)e, a.cols_magic), c = e - r * a.cols;
+            if (!a.tall) {
+              const __nv_bfloat162 lo = __floats2bfloat162_rn(nv[0], nv[1]);
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(nv[2], nv[3]);
+              *reinterpret_cast<uint2*>(X + swz(r, c)) =
+                  make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<__nv_bfloat16*>(X + swz(c + j, r)) = __float2bfloat16_rn(nv[j]);
+            }
+          }
+        }
+      } else if constexpr (BULK) {
         // per round: `per` floats of G (and of B in Muon mode) into A
         const int per = a.mode == 1 ? STAGE_F / 2 : STAGE_F;
         const float* sg = reinterpret_cast<const float*>(A);

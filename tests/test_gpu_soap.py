@@ -361,3 +361,34 @@ def test_pass_loop_graph_equals_direct_launches(ctx):
         for k in a:
             if a[k] is not None:
                 np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+def test_cuda_graph_capture_matches_eager(ctx):
+    """A SOAP step (refresh included) captured in a caller's CUDA graph and
+    replayed gives bitwise the eager result: inside a capture the refresh
+    launches its passes directly, gated on the device."""
+    import torch
+    S, G, t = warm_state(96, 160, True, True, 6, "graph-capture")
+    eager = run_gpu(ctx, S, G, t)
+    d = {k: _cuda(v) for k, v in S.items()}
+    d["G"] = _cuda(G)
+    call = lambda: ctx.soap_step([d], t, reserve=False, **HP)
+    ctx.soap_step([d], t, **HP)                       # reserves the workspace (state reset below)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call()                                        # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for k, v in S.items():                            # reset the state, then replay once
+        if v is not None:
+            d[k].copy_(_cuda(v))
+    graph.replay()
+    torch.cuda.synchronize()
+    assert ctx.device_status() == 0
+    for k, v in eager.items():
+        if v is not None:
+            np.testing.assert_array_equal(_np(d[k]), v, err_msg=k)
+    del graph

@@ -569,7 +569,9 @@ def soap_bench(ctx, dev, steps=3, warm=10, side=4096):
                               "useful_TFLOP/s": round(rot / (rot_ms / 1e3) / 1e12, 1) if rot_ms else None,
                               "executed_TFLOP/s": round(rot_exec / (rot_ms / 1e3) / 1e12, 1) if rot_ms else None,
                               "note": "two-plane operands: 3 bf16 MMAs per useful product"},
-            "kernels_note": "kernels_ms_per_step: further steps with per-launch events (their overhead included)",
+            "kernels_note": ("kernels_ms_per_step: further steps with per-launch events (their overhead included); "
+                             "with the events on, the refresh launches all 16 passes, the unneeded ones gated off "
+                             "on the device (qr_chol, qr_rowblock, qr_trail include those launches)"),
             "gpu_launches": int(sum(v[2] for v in prof.values()) / steps)}
 
 

@@ -263,7 +263,7 @@ typedef struct {
   int bias_correction;  /* 1: divide by 1 - beta^t (default) */
   int32_t* nonfinite;   /* optional device int32[n]: 1 when a basis refresh did
                            not reach an orthonormal basis (non-finite input,
-                           or more CholeskyQR passes needed than allowed); that
+                           or more than 16 CholeskyQR passes needed); that
                            matrix then keeps its previous basis */
   int skip_refresh;     /* 1: update L, R but keep Q_L, Q_R this step (the steps
                            between refreshes when the basis is refreshed only

@@ -49,7 +49,7 @@
 
 namespace mo {
 
-constexpr int QR_MAX_PASSES = 8;
+constexpr int QR_MAX_PASSES = 16;
 constexpr int QR_CHECK_BLOCKS = 64;    // partial sums per matrix for the Gram check
 constexpr float QR_TAU_DONE = 5e-5f;
 constexpr float QR_PLAIN_FLOOR = 1e-4f;

@@ -558,31 +558,24 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
         for (int j = 0; j < q; ++j) qold[j] = basis_of(j);
         launch_qr_finish(ctl, flags, q, CY + kk, kp, ms, (int)k, (int)kp, qold, s);
       }
-      // the new bases: fp32 into the caller's Q, bf16 into the group buffers
-      CopyOutArgs co;
-      co.count = q; co.k = (int)k; co.Y = CY + kk; co.ld = kp; co.mat_stride = ms;
-      for (int j = 0; j < q; ++j) {
-        const mo_soap_mat& m = items[bk.jobs[j].item].m;
-        co.dst[j] = bk.jobs[j].left ? m.QL : m.QR;
-      }
-      launch_copy_out(co, s);
-      // two bf16 planes of each new basis into its group's buffer (one launch
-      // per job: the group buffers are not uniformly strided across the bucket)
+      BasisOutArgs bo;
+      bo.count = q; bo.k = (int)k; bo.kpad_max = 0;
+      bo.Y = CY + kk; bo.ld = kp; bo.mat_stride = ms;
       for (int j = 0; j < q; ++j) {
         const Job& jb = bk.jobs[j];
         const Group& g = P.groups[jb.group];
+        const mo_soap_mat& m = items[jb.item].m;
         const long long kpad = jb.left ? g.mpad : g.npad;
-        SplitArgs one;
-        one.count = 1; one.rows_valid = (int)k; one.cols_valid = (int)k;
-        one.rows_pad = (int)kpad; one.cols_pad = (int)kpad;
-        one.src[0] = CY + (size_t)j * ms + kk; one.lds = kp;
-        one.col_scale = nullptr; one.write_back = nullptr; one.ldw = 0; one.wb_stride = 0;
-        one.dst = at<__nv_bfloat16>(ws, jb.left ? g.qlp : g.qrp) + (size_t)jb.pos * kpad * kpad;
-        one.ldd = kpad; one.mat_stride = 0;
-        one.plane_stride = (long long)g.items.size() * kpad * kpad;
-        one.nplanes = 2; one.pad_identity = 0;
-        launch_split(one, s);
+        bo.q[j] = jb.left ? m.QL : m.QR;
+        bo.vec[j] = (k % 4 == 0 && (reinterpret_cast<uintptr_t>(bo.q[j]) & 15) == 0) ? 1 : 0;
+        bo.kpad[j] = (int)kpad;
+        bo.planes[j] = at<__nv_bfloat16>(ws, jb.left ? g.qlp : g.qrp) + (size_t)jb.pos * kpad * kpad;
+        bo.pst[j] = (long long)g.items.size() * kpad * kpad;
+        bo.kpad_max = std::max(bo.kpad_max, (int)kpad);
       }
+      // the new bases: fp32 into the caller's Q, two bf16 planes into the
+      // group buffers for the rotations, in one pass
+      launch_basis_out(bo, s);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaGetLastError();

@@ -134,11 +134,44 @@ __global__ void __launch_bounds__(256) damping_kernel(const DampArgs a) {
   if (threadIdx.x == 0) a.delta[b] = part[0] != 0.f ? a.rho * part[0] : 1.0f;
 }
 
-__global__ void copy_out_kernel(const CopyOutArgs a) {
+// four columns per thread: one float4 read of Y (rows are 16-byte aligned,
+// ld a multiple of 128), the fp32 copy, and four bf16 of each plane
+__global__ void basis_out_kernel(const BasisOutArgs a) {
   const int b = blockIdx.z;
   const int r = blockIdx.y;
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c < a.k) a.dst[b][(long long)r * a.k + c] = a.Y[(size_t)b * a.mat_stride + (long long)r * a.ld + c];
+  const int kpad = a.kpad[b];
+  const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (r >= kpad || c0 >= kpad) return;
+  const int k = a.k;
+  float x[4] = {0.f, 0.f, 0.f, 0.f};
+  if (r < k) {
+    const float* y = a.Y + (size_t)b * a.mat_stride + (long long)r * a.ld + c0;
+    if (c0 + 4 <= k) {
+      const float4 v = *reinterpret_cast<const float4*>(y);
+      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x[j] = c0 + j < k ? y[j] : 0.f;
+    }
+    float* q = a.q[b] + (long long)r * k + c0;
+    if (a.vec[b] && c0 + 4 <= k) {
+      *reinterpret_cast<float4*>(q) = make_float4(x[0], x[1], x[2], x[3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (c0 + j < k) q[j] = x[j];
+    }
+  }
+  __nv_bfloat162 h01 = __floats2bfloat162_rn(x[0], x[1]);
+  __nv_bfloat162 h23 = __floats2bfloat162_rn(x[2], x[3]);
+  const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+  __nv_bfloat162 l01 = __floats2bfloat162_rn(x[0] - f01.x, x[1] - f01.y);
+  __nv_bfloat162 l23 = __floats2bfloat162_rn(x[2] - f23.x, x[3] - f23.y);
+  __nv_bfloat16* d = a.planes[b] + (long long)r * kpad + c0;     // 8-byte aligned: kpad % 4 == 0
+  *reinterpret_cast<uint2*>(d) =
+      make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+  *reinterpret_cast<uint2*>(d + a.pst[b]) =
+      make_uint2(*reinterpret_cast<const uint32_t*>(&l01), *reinterpret_cast<const uint32_t*>(&l23));
 }
 
 __global__ void adam_identity_kernel(const AdamIdArgs a) {
@@ -216,10 +249,10 @@ void launch_damping(const DampArgs& a, cudaStream_t s) {
   damping_kernel<<<a.count, 256, 0, s>>>(a);
 }
 
-void launch_copy_out(const CopyOutArgs& a, cudaStream_t s) {
+void launch_basis_out(const BasisOutArgs& a, cudaStream_t s) {
   ProfScope prof(PK_SOAP_QR, s);
-  dim3 grid((a.k + 255) / 256, a.k, a.count);
-  copy_out_kernel<<<grid, 256, 0, s>>>(a);
+  dim3 grid((a.kpad_max + 1023) / 1024, a.kpad_max, a.count);
+  basis_out_kernel<<<grid, 256, 0, s>>>(a);
 }
 
 void launch_adam_identity(const AdamIdArgs& a, cudaStream_t s) {

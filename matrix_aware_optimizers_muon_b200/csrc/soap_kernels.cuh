@@ -64,12 +64,22 @@ struct FlagTable {
 };
 
 // Final basis: Qout[b] (caller fp32 k x k) = Y[b][:k, :k]
-struct CopyOutArgs {
-  int count, k;
+// The new bases out of the refresh, in one pass over them: job b's k x k
+// basis (rows of Y + b * mat_stride, row stride ld) into the caller's q[b]
+// (fp32, row stride k) and, zero-padded to kpad[b] x kpad[b] (a multiple of
+// 4), as two bf16 planes h = bf16(x), l = bf16(x - h) at planes[b] (row
+// stride kpad[b], plane stride pst[b]) for the rotations.  vec[b]: q[b] is
+// 16-byte aligned and k % 4 == 0 (float4 stores).
+struct BasisOutArgs {
+  int count, k, kpad_max;
   const float* Y; long long ld, mat_stride;
-  float* dst[SOAP_MAXB];
+  float* q[SOAP_MAXB];
+  __nv_bfloat16* planes[SOAP_MAXB];
+  int kpad[SOAP_MAXB];
+  long long pst[SOAP_MAXB];
+  unsigned char vec[SOAP_MAXB];
 };
-void launch_copy_out(const CopyOutArgs& a, cudaStream_t s);
+void launch_basis_out(const BasisOutArgs& a, cudaStream_t s);
 
 // Adam step with identity bases (both sides) fused with the apply:
 // V <- b2 V + (1-b2) G^2 ; W <- decay W - lr (M / bc1) / (sqrt(V / bc2) + eps)

@@ -905,9 +905,9 @@ def gemm_vs_cublas(args, local):
     D8 = torch.empty(s8, s8, device=dev, dtype=torch.bfloat16)
     f_prod = 2.0 * m * m * n * bt                   # Gram or update, full product
     ops = [
-        ("update aX + PX", "ours", f_prod,
-         lambda: ctx.gemm_bf16(P, X, Y, M=m, N=n, K=m, batch=bt, b_mn=True, alpha=1.0, beta=3.4445, C=X)),
-        ("update aX + PX", "cublas", f_prod, lambda: torch.bmm(P, X, out=Y)),
+        ("update P X", "ours", f_prod,
+         lambda: ctx.gemm_bf16(P, X, Y, M=m, N=n, K=m, batch=bt, b_mn=True)),
+        ("update P X", "cublas", f_prod, lambda: torch.bmm(P, X, out=Y)),
         ("Gram X X^T", "ours (symmetric)", f_prod,
          lambda: ctx.gemm_bf16(X, X, A, M=m, N=m, K=n, batch=bt, sym=True)),
         ("Gram X X^T", "ours (full)", f_prod, lambda: ctx.gemm_bf16(X, X, A, M=m, N=m, K=n, batch=bt)),

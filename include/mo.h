@@ -115,8 +115,8 @@ MO_API mo_status mo_device_status(mo_ctx* ctx, void* stream, int32_t* status);
  * synchronises those events and returns, per kernel kind k < nkinds (host
  * arrays), the summed elapsed milliseconds, the executed tensor-core flops
  * and the launch count, then forgets the records.  Kinds: 0 Muon momentum /
- * cast, 1 norm finalize, 2 Gram X X^T, 3 polynomial b A + c A A, 4 update
- * a X + P X, 5 apply / store, 6 SOAP elementwise, 7 SOAP rotations, 8 SOAP
+ * cast, 1 norm finalize, 2 Gram X X^T, 3 polynomial a I + b A + c A A,
+ * 4 update P X, 5 apply / store, 6 SOAP elementwise, 7 SOAP rotations, 8 SOAP
  * power step and QR (other), 9 mo_gemm_bf16, 10 SOAP factor EMAs, 11 QR
  * diagonal Cholesky blocks, 12 QR row-block solves, 13 QR trailing updates,
  * 14 fused small-matrix Newton-Schulz / Muon. */

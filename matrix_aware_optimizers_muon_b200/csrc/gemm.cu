@@ -165,6 +165,8 @@ cudaError_t launch_t(const GemmOp& op, int* status, cudaStream_t stream) {
   p.gate = op.gate;
   p.gate_n = op.gate_n;
   p.gate_idx = op.gate_idx;
+  p.diag = op.diag_add;
+  if (op.diag_add != 0.f && op.epi != EPI_AXPBY) return cudaErrorInvalidValue;
   if (op.epi == EPI_APPLY && (op.sym || op.e_tab == nullptr || op.d_f32 || op.d_split))
     return cudaErrorInvalidValue;
   // a strided bf16 C of the plain (or Muon apply) epilogue is read by TMA

@@ -86,6 +86,9 @@ struct GemmParams {
   const int* gate;
   int gate_n;
   const int* gate_idx;
+  // added to the diagonal elements (row == column) of each matrix's
+  // output, before rounding (epilogue AXPBY)
+  float diag;
   // A and B hold fp16 (not bf16) values: the same kind::f16 MMA with the
   // operand type fields of the instruction descriptor set to f16
   int ab_f16;
@@ -959,6 +962,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             load_row32(cbase, p.c_f32, (long long)r * p.ldc + c0, full ? 32 : p.N - c0, c);
 #pragma unroll
             for (int i = 0; i < 32; ++i) x[i] = fmaf(beta, c[i], x[i]);
+          }
+          if (p.diag != 0.f && c0 < r0 + 32 && r0 < c0 + 32) {
+            // the block meets the diagonal: lane r adds to its element (r, r)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c0 + i == r) x[i] += p.diag;
           }
           if (apply) {
             // O = bf16(x), as the plain output would hold it; then the Muon

@@ -3,9 +3,10 @@
 //   prep (momentum, Nesterov, bf16 cast + orientation, tile partials of N^2)
 //   finalize (||N||_F -> 1 / (||N||_F + eps))
 //   ns_steps x { A = X X^T          (symmetric: upper tiles + mirror)
-//                P = b A + c A A    (symmetric: upper tiles + mirror)
-//                X' = a X + P X }   (iteration 0 folds the 1/(||N||+eps)
-//                                    scale into the fp32 epilogues)
+//                P = a I + b A + c A A  (symmetric: upper tiles + mirror)
+//                X' = P X }         (= a X + (b A + c A A) X; iteration 0
+//                                    folds the 1/(||N||+eps) scale into the
+//                                    fp32 epilogues)
 //   apply (W <- (1 - lr wd) W - lr s O, un-oriented; or out = O); for Muon
 //   the apply runs in the epilogue of the last update product instead, so
 //   O is never stored
@@ -251,23 +252,24 @@ cudaError_t ns_run_at(const std::vector<NsItem>& items, const NsCall& call, int*
         e = launch_gemm(g, status, stream);
         if (e != cudaSuccess) return e;
 
-        GemmOp q;                      // P = b A + c A A   (A symmetric: A A = A A^T)
+        // P = a I + b A + c A A   (A symmetric: A A = A A^T); a on the
+        // diagonal lets the update X' = a X + (b A + c A A) X be one product
+        GemmOp q;
         q.A = A; q.lda = L.lda; q.strideA = L.astride; q.a_mn = 0;
         q.B = A; q.ldb = L.lda; q.strideB = L.astride; q.b_mn = 0;
         q.M = (int)s.mp; q.N = (int)s.mp; q.K = (int)s.mp; q.batch = cnt; q.sym = 1;
-        q.alpha = call.c; q.beta = call.b;
+        q.alpha = call.c; q.beta = call.b; q.diag_add = call.a;
         q.C = A; q.ldc = L.lda; q.strideC = L.astride; q.c_f32 = 0;
         q.D = P; q.ldd = L.lda; q.strideD = L.astride; q.d_f32 = 0; q.kind = PK_POLY;
         e = launch_gemm(q, status, stream);
         if (e != cudaSuccess) return e;
 
-        GemmOp u;                      // X' = a X + P X   (X stored [K = m'][N = n'])
+        GemmOp u;                      // X' = P X   (X stored [K = m'][N = n'])
         u.A = P; u.lda = L.lda; u.strideA = L.astride; u.a_mn = 0;
         u.B = Xc; u.ldb = L.ldx; u.strideB = L.xstride; u.b_mn = 1;
         u.M = (int)s.mp; u.N = (int)s.np; u.K = (int)s.mp; u.batch = cnt; u.sym = 0;
-        u.alpha = 1.f; u.beta = call.a;
-        u.scale = inv; u.alpha_pow = it == 0 ? 1 : 0; u.beta_pow = it == 0 ? 1 : 0;
-        u.C = Xc; u.ldc = L.ldx; u.strideC = L.xstride; u.c_f32 = 0;
+        u.alpha = 1.f; u.beta = 0.f;
+        u.scale = inv; u.alpha_pow = it == 0 ? 1 : 0;
         u.D = Xn; u.ldd = L.ldx; u.strideD = L.xstride; u.d_f32 = 0; u.kind = PK_UPDATE;
         if (fused_apply && it == call.steps - 1) {
           u.epi = 2;                   // Muon apply epilogue

@@ -14,8 +14,8 @@ enum ProfKind {
   PK_PREP = 0,       // Muon momentum / cast / partial norms
   PK_NORM = 1,       // norm finalize
   PK_GRAM = 2,       // A = X X^T
-  PK_POLY = 3,       // P = b A + c A A
-  PK_UPDATE = 4,     // X' = a X + P X
+  PK_POLY = 3,       // P = a I + b A + c A A
+  PK_UPDATE = 4,     // X' = P X  (P = a I + b A + c A A; small kernel: a X + P X)
   PK_APPLY = 5,      // W update / output store
   PK_SOAP_EW = 6,    // SOAP elementwise kernels
   PK_SOAP_GEMM = 7,  // SOAP tensor-core products

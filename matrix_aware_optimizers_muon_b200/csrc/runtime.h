@@ -144,6 +144,8 @@ struct GemmOp {
   const int* gate = nullptr;
   int gate_n = 0;
   const int* gate_idx = nullptr;     // optional device index: the gate word is gate[*gate_idx]
+  // added to each matrix's diagonal (row == column) before D is rounded
+  float diag_add = 0.f;
 };
 
 // Launch the tcgen05 GEMM.  Returns cudaSuccess or the launch/encode error.

@@ -15,8 +15,8 @@ Two modes:
 
 * ``newton_schulz`` - the iteration in float64, nothing rounded.
 * ``newton_schulz_bf16`` - the same iteration with bfloat16 rounding at the
-  points the GPU path declares (operands bf16, products accumulated wide,
-  every stored matrix rounded to bf16 with ties-to-even):
+  points of a bf16-operand product chain (operands bf16, products
+  accumulated wide, every stored matrix rounded to bf16 with ties-to-even):
 
       Nb  = bf16(N)                      (the cast happens before scaling, as
       s   = ||N||_F,  inv = 1/(s + eps)   in the pages' reference code; the
@@ -30,8 +30,10 @@ Two modes:
                      X = bf16(a X + P X)
 
   In exact arithmetic both modes compute the same X_k (X_0 = inv * Nb when
-  Nb = N); the emulation exists so that the GPU result can be compared with
-  what its own rounding points imply.
+  Nb = N); the emulation gives the noise floor that a bf16 path's result is
+  held to.  (A path may round at other points with the same iteration, e.g.
+  store bf16(a I + b A + c A A) and form X = bf16(P X); its error is then
+  held to this same floor.)
 """
 
 import numpy as np

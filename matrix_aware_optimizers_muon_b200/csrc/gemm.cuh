@@ -825,7 +825,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       // otherwise bf16 C of full blocks (pointer tables): loaded one block
       // ahead with coalesced 16-byte loads (eight 64-byte rows per
       // instruction), then transposed to row-per-lane through shared memory
-      const bool cpre = !ctma && has_c && !adam && !p.c_f32 && plain_bf16 && n0 + BN <= p.N &&
+      const bool cpre = !EPI2 && !ctma && has_c && !adam && !p.c_f32 && plain_bf16 && n0 + BN <= p.N &&
                         __all_sync(0xffffffffu, row_ok);
       const __nv_bfloat16* c16 = reinterpret_cast<const __nv_bfloat16*>(cbase);
       uint4 cnext[4];
@@ -842,9 +842,32 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const bool cf32 = has_c && !adam && p.c_f32 && !p.d_split && n0 + BN <= p.N &&
                         __all_sync(0xffffffffu, row_ok);
       const float* c32 = reinterpret_cast<const float*>(cbase);
+      // a full tile of a plain product (no C, no mirror, bf16 out by TMA
+      // stores): a compact loop, away from the general one's many cases
+      const bool plain_tile = dstg && !has_c && !p.sym && !adam && !apply && p.diag == 0.f;
+      if (plain_tile) {
+#pragma unroll 1
+        for (int cc = 0; cc < BN; cc += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + cc, v);
+          tmem_ld_wait();
+          float x[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = alpha * __uint_as_float(v[i]);
+          if (lane == 0) bulk_wait_read();         // the previous block's store has read the slot
+          __syncwarp();
+          stage_rows_tma(stg, nullptr, lane, x);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmD, stg, n0 + cc, r0, b);
+            bulk_commit();
+          }
+        }
+      }
       int kk = 0;                                // 32-column blocks done in this tile
 #pragma unroll 1
-      for (int cc = cc_begin; cc < BN; cc += 32, ++kk) {
+      for (int cc = plain_tile ? BN : cc_begin; cc < BN; cc += 32, ++kk) {
         uint4 ccur[4];
         if (cpre) {
 #pragma unroll

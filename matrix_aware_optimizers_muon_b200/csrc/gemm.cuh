@@ -865,9 +865,68 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
         }
       }
+      // a full tile of a symmetric product (Gram; polynomial with C by TMA
+      // in slots 2 and 3): blocks on or above the diagonal, each stored with
+      // its mirror image (a diagonal block symmetrised in place)
+      const bool sym_tile = dstg && p.sym && !adam && !apply;
+      if (sym_tile) {
+        int kq = 0;
+#pragma unroll 1
+        for (int cc = cc_begin; cc < BN; cc += 32, ++kq) {
+          const int c0 = n0 + cc;
+          const bool dg = c0 == r0;
+          uint32_t v[32];
+          tmem_ld32(taddr + cc, v);
+          tmem_ld_wait();
+          float x[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = alpha * __uint_as_float(v[i]);
+          if (ctma) {
+            const int bi = 2 + (kq & 1);
+            mbar_wait(&cb[bi], (cph >> bi) & 1u, abort_flag, p.status, DEV_TIMEOUT_ACC_FULL);
+            cph ^= 1u << bi;
+            cpend &= ~(1u << bi);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint4 w = *reinterpret_cast<const uint4*>(stg + 2048 * bi + stg_off(lane, u));
+              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ws[j]));
+                x[8 * u + 2 * j] = fmaf(beta, f.x, x[8 * u + 2 * j]);
+                x[8 * u + 2 * j + 1] = fmaf(beta, f.y, x[8 * u + 2 * j + 1]);
+              }
+            }
+            __syncwarp();                         // every lane has read the slot
+            if (lane == 0) {
+              fence_proxy_async_smem();
+              if (cc + 64 < BN) issue_c(bi, cc + 64);
+            }
+          }
+          if (dg && p.diag != 0.f) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c0 + i == r) x[i] += p.diag;
+          }
+          if (lane == 0) bulk_wait_read();         // the previous block's stores have read slots 0 and 1
+          __syncwarp();
+          stage_rows_tma(stg, stg + 2048, lane, x);
+          if (dg) {
+            __syncwarp();
+            symmetrize_staged(stg, stg + 2048, lane);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmD, stg, c0, r0, b);
+            if (!dg) tma_store_3d(&tmD, stg + 2048, r0, c0, b);
+            bulk_commit();
+          }
+        }
+      }
       int kk = 0;                                // 32-column blocks done in this tile
 #pragma unroll 1
-      for (int cc = plain_tile ? BN : cc_begin; cc < BN; cc += 32, ++kk) {
+      for (int cc = (plain_tile || sym_tile) ? BN : cc_begin; cc < BN; cc += 32, ++kk) {
         uint4 ccur[4];
         if (cpre) {
 #pragma unroll

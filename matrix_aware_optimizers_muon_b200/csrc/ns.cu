@@ -4,9 +4,11 @@
 //   finalize (||N||_F -> 1 / (||N||_F + eps))
 //   ns_steps x { A = X X^T          (symmetric: upper tiles + mirror)
 //                P = a I + b A + c A A  (symmetric: upper tiles + mirror)
-//                X' = P X }         (= a X + (b A + c A A) X; iteration 0
-//                                    folds the 1/(||N||+eps) scale into the
-//                                    fp32 epilogues)
+//                X' = P X }         (= a X + (b A + c A A) X; with fewer
+//                                    than 128 rows P = b A + c A A and
+//                                    X' = a X + P X; iteration 0 folds the
+//                                    1/(||N||+eps) scale into the fp32
+//                                    epilogues)
 //   apply (W <- (1 - lr wd) W - lr s O, un-oriented; or out = O); for Muon
 //   the apply runs in the epilogue of the last update product instead, so
 //   O is never stored
@@ -253,23 +255,29 @@ cudaError_t ns_run_at(const std::vector<NsItem>& items, const NsCall& call, int*
         if (e != cudaSuccess) return e;
 
         // P = a I + b A + c A A   (A symmetric: A A = A A^T); a on the
-        // diagonal lets the update X' = a X + (b A + c A A) X be one product
+        // diagonal lets the update X' = a X + (b A + c A A) X be one product.
+        // With fewer than 128 rows a row of X carries a large share of the
+        // norm, P's diagonal is of the order of a, and rounding a + P_ii to
+        // bf16 costs more than it does with a X kept apart: there P =
+        // b A + c A A and the update reads X as C
+        const bool fold = s.mp >= 128;
         GemmOp q;
         q.A = A; q.lda = L.lda; q.strideA = L.astride; q.a_mn = 0;
         q.B = A; q.ldb = L.lda; q.strideB = L.astride; q.b_mn = 0;
         q.M = (int)s.mp; q.N = (int)s.mp; q.K = (int)s.mp; q.batch = cnt; q.sym = 1;
-        q.alpha = call.c; q.beta = call.b; q.diag_add = call.a;
+        q.alpha = call.c; q.beta = call.b; q.diag_add = fold ? call.a : 0.f;
         q.C = A; q.ldc = L.lda; q.strideC = L.astride; q.c_f32 = 0;
         q.D = P; q.ldd = L.lda; q.strideD = L.astride; q.d_f32 = 0; q.kind = PK_POLY;
         e = launch_gemm(q, status, stream);
         if (e != cudaSuccess) return e;
 
-        GemmOp u;                      // X' = P X   (X stored [K = m'][N = n'])
+        GemmOp u;                      // X' = P X, or a X + P X   (X stored [K = m'][N = n'])
         u.A = P; u.lda = L.lda; u.strideA = L.astride; u.a_mn = 0;
         u.B = Xc; u.ldb = L.ldx; u.strideB = L.xstride; u.b_mn = 1;
         u.M = (int)s.mp; u.N = (int)s.np; u.K = (int)s.mp; u.batch = cnt; u.sym = 0;
-        u.alpha = 1.f; u.beta = 0.f;
-        u.scale = inv; u.alpha_pow = it == 0 ? 1 : 0;
+        u.alpha = 1.f; u.beta = fold ? 0.f : call.a;
+        u.scale = inv; u.alpha_pow = it == 0 ? 1 : 0; u.beta_pow = (!fold && it == 0) ? 1 : 0;
+        if (!fold) { u.C = Xc; u.ldc = L.ldx; u.strideC = L.xstride; u.c_f32 = 0; }
         u.D = Xn; u.ldd = L.ldx; u.strideD = L.xstride; u.d_f32 = 0; u.kind = PK_UPDATE;
         if (fused_apply && it == call.steps - 1) {
           u.epi = 2;                   // Muon apply epilogue

@@ -150,20 +150,25 @@ extern "C" MO_API mo_status ns_orthogonalize_static(mo_ctx* ctx, const float* in
     g.D = A; g.ldd = lda; g.strideD = astride;
     e = mo::launch_gemm(g, status, s);
     if (e != cudaSuccess) break;
-    mo::GemmOp q;                                  // P = a I + b A + c A A
+    const bool fold = mp >= 128;                   // as in the workspace path
+    mo::GemmOp q;                                  // P = a I + b A + c A A (or b A + c A A)
     q.A = A; q.lda = lda; q.strideA = astride;
     q.B = A; q.ldb = lda; q.strideB = astride;
     q.M = (int)mp; q.N = (int)mp; q.K = (int)mp; q.sym = 1;
-    q.alpha = cfg->c; q.beta = cfg->b; q.diag_add = cfg->a;
+    q.alpha = cfg->c; q.beta = cfg->b; q.diag_add = fold ? cfg->a : 0.f;
     q.C = A; q.ldc = lda; q.strideC = astride;
     q.D = P; q.ldd = lda; q.strideD = astride;
     e = mo::launch_gemm(q, status, s);
     if (e != cudaSuccess) break;
-    mo::GemmOp u;                                  // X' = P X = a X + (b A + c A A) X
+    mo::GemmOp u;                                  // X' = P X (or a X + P X)
     u.A = P; u.lda = lda; u.strideA = astride;
     u.B = Xc; u.ldb = ldx; u.strideB = xstride; u.b_mn = 1;
     u.M = (int)mp; u.N = (int)np; u.K = (int)mp;
     u.scale = inv; u.alpha_pow = it == 0 ? 1 : 0;
+    if (!fold) {
+      u.beta = cfg->a; u.beta_pow = it == 0 ? 1 : 0;
+      u.C = Xc; u.ldc = ldx; u.strideC = xstride;
+    }
     u.D = Xn; u.ldd = ldx; u.strideD = xstride;
     e = mo::launch_gemm(u, status, s);
     Xc = Xn;

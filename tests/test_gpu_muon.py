@@ -77,7 +77,7 @@ def test_cfg1_two_steps_deterministic(ctx):
 
 
 @pytest.mark.parametrize("shape", [(128, 384), (384, 128), (300, 300), (130, 257), (257, 130),
-                                   (64, 1000), (7, 3), (1, 40), (40, 1)])
+                                   (64, 1000), (7, 3), (1, 40), (40, 1), (3, 1000), (512, 8)])
 def test_ragged_shapes_full_rank(ctx, shape):
     m, n = shape
     rng = wl.rng_of("ragged", m, n)

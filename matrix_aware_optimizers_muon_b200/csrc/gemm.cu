@@ -245,10 +245,12 @@ int device_sm_count() {
 
 namespace {
 // CTA pairs (256 x 256 tiles over two SMs) for products with more than 128
-// rows and N > 128, when MO_GEMM_PAIR=1 is set in the environment.  They do
-// the same work in fewer cycles, but under the B200's power cap the clock
-// drops by as much and the step takes as long (measured), so single-CTA
-// 128 x 256 tiles are the default.
+// rows and N > 128: for short K with two epilogue sets, for products that
+// ask for them (GemmOp::pair, the SOAP products), and for all when
+// MO_GEMM_PAIR=1 is set in the environment.  They do the same work in fewer
+// cycles, but under the B200's power cap the clock drops by as much or more
+// on the Newton-Schulz chain's long-K products (measured), so single-CTA
+// 128 x 256 tiles are the default there.
 bool pairs_enabled() {
   static const bool on = [] {
     const char* v = std::getenv("MO_GEMM_PAIR");
@@ -273,7 +275,7 @@ cudaError_t launch_gemm(const GemmOp& op, int* status, cudaStream_t stream) {
   const int bn = narrow ? 128 : 256;
   const long long tiles = (long long)((op.M + GEMM_BM - 1) / GEMM_BM) * ((op.N + bn - 1) / bn) * op.batch;
   const bool epi2 = op.K <= MO_EPI2_MAX_K && tiles >= 2LL * device_sm_count();
-  if (!narrow && op.M > GEMM_BM && (pairs_enabled() || (epi2 && MO_SHORTK_PAIR))) {
+  if (!narrow && op.M > GEMM_BM && (pairs_enabled() || op.pair || (epi2 && MO_SHORTK_PAIR))) {
     switch ((epi2 ? 4 : 0) | (op.a_mn ? 2 : 0) | (op.b_mn ? 1 : 0)) {
       case 0: return launch_t<256, 0, 0, true>(op, status, stream);
       case 1: return launch_t<256, 0, 1, true>(op, status, stream);

@@ -146,6 +146,10 @@ struct GemmOp {
   const int* gate_idx = nullptr;     // optional device index: the gate word is gate[*gate_idx]
   // added to each matrix's diagonal (row == column) before D is rounded
   float diag_add = 0.f;
+  // CTA pairs (256 x 256 tiles over two SMs) where the shape allows them,
+  // whatever K (measured faster for the SOAP products, slower for the
+  // Newton-Schulz chain's long-K products at the power cap)
+  int pair = 0;
 };
 
 // Launch the tcgen05 GEMM.  Returns cudaSuccess or the launch/encode error.

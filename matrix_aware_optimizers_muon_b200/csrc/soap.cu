@@ -346,6 +346,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       if (g.left) {          // L <- bs L + (1 - bs) Gb Gb^T   (Gb = plane h of G)
         GemmOp op;
+        op.pair = 1;
         op.A = pa.Gp; op.lda = g.npad; op.strideA = pn;
         op.B = pa.Gp; op.ldb = g.npad; op.strideB = pn;
         op.M = (int)g.m; op.N = (int)g.m; op.K = (int)g.n; op.batch = c; op.sym = 1;
@@ -357,6 +358,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
       }
       if (g.right) {         // R <- bs R + (1 - bs) Gb^T Gb
         GemmOp op;
+        op.pair = 1;
         op.A = pa.Gp; op.lda = g.npad; op.strideA = pn; op.a_mn = 1;
         op.B = pa.Gp; op.ldb = g.npad; op.strideB = pn; op.b_mn = 1;
         op.M = (int)g.n; op.N = (int)g.n; op.K = (int)g.m; op.batch = c; op.sym = 1;
@@ -448,6 +450,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
       launch_split16(sp, s);
       {
         GemmOp op;
+        op.pair = 1;
         op.A = LQ; op.lda = kp; op.strideA = ms;                           // F [i][p]: K-major
         op.B = LQ + kk; op.ldb = kp; op.strideB = ms; op.b_mn = 1;        // Q_old [p][j]: MN-major
         set_planes2(op, pst, pst);
@@ -488,6 +491,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
         launch_split16(sy, st);
         {
           GemmOp g;
+          g.pair = 1;
           g.A = LQ + kk; g.lda = kp; g.strideA = ms; g.a_mn = 1;
           g.B = LQ + kk; g.ldb = kp; g.strideB = ms; g.b_mn = 1;
           set_planes2(g, pst, pst);
@@ -506,6 +510,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
           const long long r0 = (long long)j * QR_B;
           if (j > 0) {     // [C; Y][r0 :, j] -= [L; Q][r0 :, < j] L[j, < j]^T
             GemmOp t;
+            t.pair = 1;
             t.A = LQ + r0 * kp; t.lda = kp; t.strideA = ms;
             t.B = LQ + r0 * kp; t.ldb = kp; t.strideB = ms;
             set_planes2(t, pst, pst);
@@ -631,10 +636,12 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
       // rotate X into the basis: M' (fp32) or, with the Adam epilogue, V and Dbar
       auto rotate_in = [&](const __nv_bfloat16* X, bool adam) -> cudaError_t {
         GemmOp op;
+        op.pair = 1;
         op.kind = PK_SOAP_GEMM;
         op.batch = c;
         if (g.left && g.right) {
           GemmOp t;                       // T = QL^T X, kept as two planes
+          t.pair = 1;
           t.kind = PK_SOAP_GEMM; t.batch = c;
           left_t(t, X);
           to_planes(t, Tp);
@@ -662,6 +669,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
       if ((e = rotate_in(Gp, true)) != cudaSuccess) return e;      // G', V, Dbar
       // rotate back and apply: W <- decay W - lr QL Dbar QR^T
       GemmOp op;
+      op.pair = 1;
       op.kind = PK_SOAP_GEMM;
       op.batch = c;
       auto left_n = [&](GemmOp& g2, const __nv_bfloat16* X) {      // QL X
@@ -678,6 +686,7 @@ cudaError_t soap_run(const std::vector<SoapItem>& items, const mo_soap_cfg& cfg,
       };
       if (g.left && g.right) {
         GemmOp t;                         // S = QL Dbar, kept as two planes
+        t.pair = 1;
         t.kind = PK_SOAP_GEMM; t.batch = c;
         left_n(t, Dp);
         to_planes(t, Tp);

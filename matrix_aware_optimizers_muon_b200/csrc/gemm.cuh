@@ -390,6 +390,27 @@ __device__ __forceinline__ void stage_store32(uint8_t* stg, int lane, const floa
 // takes the value computed above the diagonal (its own for c >= r, its
 // mirror's for c < r), so both halves are bit-equal, with the same coalesced
 // row stores.
+// The transpose of the staged 32 x 32 bf16 block `own` into `mir` (both in
+// the rows of stg_off(); every lane's row of `own` written before the
+// call).  Each 8 x 8 sub-block (I, J) is one 16-byte unit J of rows 8I..8I+7:
+// a transposing ldmatrix takes the four sub-blocks (I, 0..3), and stmatrix
+// writes sub-block (I, J)^T as rows 8J..8J+7, unit I, of the mirror.
+__device__ __forceinline__ void stage_mirror_trans(const uint8_t* own, uint8_t* mir, int lane) {
+#pragma unroll
+  for (int I = 0; I < 4; ++I) {
+    uint32_t r0, r1, r2, r3;
+    const uint32_t src = smem_u32(own + stg_off(8 * I + (lane & 7), lane >> 3));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(src)
+                 : "memory");
+    const uint32_t dst = smem_u32(mir + stg_off(lane, I));
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(r0), "r"(r1),
+                 "r"(r2), "r"(r3)
+                 : "memory");
+  }
+}
+
 // For TMA stores of a 32 x 32 bf16 block: this lane's row into `own` and,
 // when `mir` is set, its transpose (the mirror block) into `mir`, both in
 // the 64-byte-swizzled rows of stg_off().
@@ -405,9 +426,8 @@ __device__ __forceinline__ void stage_rows_tma(uint8_t* own, uint8_t* mir, int l
     *reinterpret_cast<uint4*>(own + stg_off(lane, u)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   if (mir) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      *reinterpret_cast<__nv_bfloat16*>(mir + stg_off(i, lane >> 3) + ((lane & 7) << 1)) = __float2bfloat16_rn(x[i]);
+    __syncwarp();                       // every row of `own` is staged
+    stage_mirror_trans(own, mir, lane);
   }
 }
 

@@ -315,9 +315,9 @@ def run_ours(args, world, rank, local):
             "frac": round(gemm_tf / peak_tf, 4) if gemm_tf else None,
             "peak_source": f"{peak_kind} bf16_tflops_sustained",
             # DRAM bytes of one update launch (an iteration before the last)
-            # on the 4096 x 14336 bucket (96 matrices): ncu captured 871.3 MB
+            # on the 4096 x 14336 bucket (96 matrices): ncu captured 864.1 MB
             # on the one-layer batch of 3; traffic grows with the matrices
-            "traffic": 871.3e6 * args.layers,
+            "traffic": 864.1e6 * args.layers,
             "traffic_kernel": "update GEMM, 4096x14336 bucket, one launch (ncu, scaled by matrices)",
             "alg_flops_per_step": flops_gemm,
             "exec_flops_per_step": gemm_exec / args.steps,
